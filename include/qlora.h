@@ -1,0 +1,197 @@
+/*
+ * libqlora -- the QLoRA adapted linear layer on NVIDIA B200 (sm_100a).
+ *
+ * A linear layer whose frozen weight W0 (in x out, stored row-major as (in, out))
+ * is kept as 4-bit NormalFloat (NF4) codes with one absmax per 64 consecutive
+ * weights, the absmax values themselves double-quantised to 8-bit E4M3 codes with
+ * one fp32 scale per 256 absmax values, plus trainable low-rank adapters
+ * A (in x r) and B (r x out):
+ *
+ *     forward   Y  = X deq(Wq) + (X A) B
+ *     backward  dX = dY deq(Wq)^T + (dY B^T) A^T
+ *               dA = X^T (dY B^T)            dB = (X A)^T dY
+ *
+ * Sources (pages of the method, cited by title and section):
+ *   "QLoRA (low-rank adapters on a quantized model)" -- "How it works" steps 1-5
+ *     (quantize once and freeze; W = Wq + A B with B = 0 at the start; dA = dW B^T,
+ *     dB = A^T dW; optional merge), "What QLoRA adds over LoRA" (NF4 levels at
+ *     normal quantiles, one absmax per block of 64, absmax quantised to 8 bits,
+ *     weights dequantised to bf16 for each matmul and never updated).
+ *   "LLMs · QLoRA" -- the blockwise quantiser: reshape to rows of 64, absmax per
+ *     row, nearest level by argmin, reconstruction level[idx] * scale.
+ *   "LoRA & QLoRA" -- "Mathematical Formulation" (h = W0 x + B(A x)),
+ *     "Double Quantization" (absmax constants to an 8-bit float).
+ *
+ * Conventions for every call:
+ *   - Pointers marked [device] are device memory of the CURRENT CUDA device,
+ *     allocated and owned by the caller; the library keeps no pointer after return.
+ *     The library allocates no memory.  Pointers marked [host] are host memory.
+ *   - bf16 tensors are passed as uint16_t bit patterns (bfloat16).
+ *   - Every tensor is dense row-major, in the shapes stated, 16-byte aligned.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and return after enqueueing.  Argument checks run on the host
+ *     before any launch; a failed check returns an error and launches nothing.
+ *   - Inputs must not alias outputs.  W0 must be finite.
+ *   - No call writes to the frozen weight (codes, dq_codes, dq_scales).
+ *   - Errors: QLORA_ERR_CUDA if a launch fails; QLORA_ERR_UNSUPPORTED_DEVICE if
+ *     the current device is not compute capability 10.0 (there is no fallback).
+ */
+#ifndef QLORA_H
+#define QLORA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QLORA_API __attribute__((visibility("default")))
+#else
+#define QLORA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum qlora_status {
+  QLORA_OK = 0,
+  QLORA_ERR_INVALID_ARG = 1,        /* NULL where a tensor is required, bad enum, host pointer */
+  QLORA_ERR_SHAPE = 2,              /* a size constraint of the call is violated */
+  QLORA_ERR_ALIGNMENT = 3,          /* a tensor pointer is not 16-byte aligned */
+  QLORA_ERR_WORKSPACE = 4,          /* workspace NULL or smaller than qlora_workspace_bytes() */
+  QLORA_ERR_UNSUPPORTED_DEVICE = 5, /* current device is not sm_100 */
+  QLORA_ERR_CUDA = 6,               /* a CUDA runtime call or kernel launch failed */
+  QLORA_ERR_TIMEOUT = 7             /* a bounded wait inside a kernel gave up (qlora_ws_status) */
+} qlora_status;
+
+/* Output element type of qlora_dequantize / qlora_merge. */
+typedef enum qlora_dtype { QLORA_F32 = 0, QLORA_BF16 = 1 } qlora_dtype;
+
+/* Operation whose workspace size qlora_workspace_bytes() reports. */
+typedef enum qlora_op { QLORA_OP_FWD = 1, QLORA_OP_BWD = 2 } qlora_op;
+
+/* Fixed format constants. */
+#define QLORA_BLOCK 64   /* weights per absmax block */
+#define QLORA_GROUP 256  /* absmax values per double-quantisation fp32 scale */
+
+/*
+ * The frozen, quantised weight (non-owning view; all pointers [device]).
+ *   codes     : uint8[in*out/2]  NF4 codes of the flattened row-major (in, out) W0;
+ *               element 2k in the low nibble of byte k, element 2k+1 in the high nibble.
+ *   dq_codes  : uint8[in*out/64] E4M3 code of each block's absmax (block b = elements
+ *               64b .. 64b+63 of the flattened W0).
+ *   dq_scales : fp32[ceil(in*out/64/256)] scale of each group of 256 consecutive blocks.
+ *   in, out   : matrix shape.
+ * Dequantised weight ("What QLoRA adds over LoRA"; "LLMs · QLoRA" levels[idx]*scale):
+ *   absmax'_b = fl32(e4m3(dq_codes[b]) * dq_scales[b/256])
+ *   w'        = fl32(nf4_level[code] * absmax'_b)   (fl32 = IEEE binary32 round-to-nearest)
+ * and the matmuls use bf16(w') (round to nearest even).
+ */
+typedef struct qlora_nf4_weight {
+  const uint8_t* codes;
+  const uint8_t* dq_codes;
+  const float* dq_scales;
+  int64_t in;
+  int64_t out;
+} qlora_nf4_weight;
+
+/*
+ * Quantise W0 once ("How it works" step 1; "LLMs · QLoRA" quantiser; "What QLoRA
+ * adds over LoRA" NF4 and double quantisation).
+ *   W0        [device] fp32 (in, out).
+ *   codes     [device] out: uint8[in*out/2].
+ *   dq_codes  [device] out: uint8[in*out/64].
+ *   dq_scales [device] out: fp32[ceil(in*out/64/256)].
+ * Per block b: a_b = max |w| over the block; x = fl32(w / a_b) (IEEE division;
+ * an all-zero block gives x = 0); code = index of the nearest NF4 level, ties to
+ * the lower index.  Per group g of 256 blocks: s_g = fl32(max_b a_b / 448),
+ * dq_codes[b] = E4M3 round-to-nearest-even, saturating at 448, of fl32(a_b / s_g)
+ * (0 when s_g = 0).  Codes are bit-exact: they do not depend on launch shape.
+ * Requires in >= 1, out >= 1, in*out % 64 == 0.  W0, codes, dq_codes and dq_scales
+ * 16-byte aligned.
+ */
+QLORA_API qlora_status qlora_quantize_nf4(const float* W0, int64_t in, int64_t out, uint8_t* codes,
+                                uint8_t* dq_codes, float* dq_scales, void* stream);
+
+/*
+ * Dequantise the frozen weight to a dense (in, out) matrix: W_out[k][n] = w'
+ * (QLORA_F32) or bf16(w') (QLORA_BF16).  Bit-exact.
+ *   w      [host] descriptor of [device] tensors.
+ *   W_out  [device] out: fp32 or bf16 (in, out).
+ * Requires in*out % 64 == 0.
+ */
+QLORA_API qlora_status qlora_dequantize(const qlora_nf4_weight* w, void* W_out, int out_dtype, void* stream);
+
+/*
+ * Forward of the adapted layer ("How it works" steps 2-3; "LoRA & QLoRA"
+ * Mathematical Formulation h = W0 x + B(A x)):
+ *   V = bf16(X A)  (fp32 accumulation),   Y = bf16(X bf16(w') + V B)  (fp32 accumulation).
+ *   w      [host] descriptor of [device] tensors.
+ *   X      [device] bf16 (M, in).
+ *   A      [device] bf16 (in, r).          B [device] bf16 (r, out).
+ *   Y      [device] out: bf16 (M, out).
+ *   V_save [device] out: bf16 (M, r), the saved X A for the backward; may be NULL
+ *          (then V lives in the workspace).
+ *   ws     [device] workspace of at least qlora_workspace_bytes(QLORA_OP_FWD, ...)
+ *          bytes, initialised once by qlora_ws_init().
+ * Requires M >= 1, in % 64 == 0, out % 64 == 0, 8 <= r <= 256, r % 8 == 0.
+ */
+QLORA_API qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int64_t M,
+                              const uint16_t* A, const uint16_t* B, int r, uint16_t* Y,
+                              uint16_t* V_save, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Backward of the adapted layer ("How it works" step 4; "The code, line by line":
+ * dA = dW B^T, dB = A^T dW, here in the factored form that never forms dW):
+ *   U  = bf16(dY B^T)
+ *   dX = bf16(dY bf16(w')^T + U A^T)     (written only if dX != NULL)
+ *   dA = X^T U         (fp32, overwritten)
+ *   dB = V^T dY        (fp32, overwritten), V = X A (the saved V, or recomputed)
+ * The frozen weight receives no gradient.
+ *   X  [device] bf16 (M, in).   V [device] bf16 (M, r) from the forward, or NULL.
+ *   dY [device] bf16 (M, out).  A, B as in the forward.
+ *   dX [device] out: bf16 (M, in), or NULL.
+ *   dA [device] out: fp32 (in, r).   dB [device] out: fp32 (r, out).
+ *   ws [device] at least qlora_workspace_bytes(QLORA_OP_BWD, ...) bytes.
+ * Requires the forward's shape constraints.
+ */
+QLORA_API qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16_t* X, const uint16_t* V,
+                              const uint16_t* dY, int64_t M, const uint16_t* A,
+                              const uint16_t* B, int r, uint16_t* dX, float* dA, float* dB,
+                              void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Merge the adapters into a dense weight ("How it works" step 5):
+ *   W_out = w' + A B   (fp32 accumulation; QLORA_F32 or QLORA_BF16 output, (in, out)).
+ * Requires in % 64 == 0, out % 64 == 0, 8 <= r <= 256, r % 8 == 0.
+ */
+QLORA_API qlora_status qlora_merge(const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B, int r,
+                         void* W_out, int out_dtype, void* stream);
+
+/* ---------------------------------------------------------------- helpers */
+
+/* Bytes of workspace qlora_linear_fwd / qlora_linear_bwd need for these sizes
+ * (0 for an unknown op or invalid sizes).  Host only, no device access. */
+QLORA_API size_t qlora_workspace_bytes(int op, int64_t M, int64_t in, int64_t out, int r);
+
+/* Zero the workspace's status words (once, before the workspace's first use). */
+QLORA_API qlora_status qlora_ws_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, then report QLORA_ERR_TIMEOUT if a bounded wait in a
+ * kernel that used this workspace gave up since the last check (and clear it),
+ * else QLORA_OK.  Device work of a call that timed out left its outputs undefined. */
+QLORA_API qlora_status qlora_ws_status(void* ws, void* stream);
+
+/* The 16 NF4 levels, ascending (code = index) [host]. */
+QLORA_API void qlora_nf4_codebook(float out[16]);
+
+/* Adapter parameters of one layer: r (in + out) ("How it works", adapter size). */
+QLORA_API int64_t qlora_adapter_params(int64_t in, int64_t out, int r);
+
+/* Human-readable name of a status code (static string). */
+QLORA_API const char* qlora_status_string(qlora_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_H */

@@ -59,6 +59,13 @@ def backward(X, A, B, Wq, dY):
     return {"dX": dX, "dA": dA, "dB": dB, "U": U}
 
 
+def adapter_grads(X, A, B, dY):
+    """dA = X^T (dY B^T) and dB = (X A)^T dY alone (no dX), for large token counts."""
+    X, A, B, dY = _f64(X), _f64(A), _f64(B), _f64(dY)
+    U = dY @ B.T
+    return {"dA": X.T @ U, "dB": (X @ A).T @ dY}
+
+
 def backward_dense(X, A, B, dY):
     """The pages' own route: dW = X^T dY, dA = dW B^T, dB = A^T dW."""
     X, A, B, dY = _f64(X), _f64(A), _f64(B), _f64(dY)

@@ -1,0 +1,225 @@
+"""Python binding of libqlora, the QLoRA adapted linear layer for B200 (sm_100a).
+
+Argument marshalling only: every function passes device pointers, sizes and the
+current CUDA stream to the C ABI declared in ``include/qlora.h`` and raises
+``QLoRAError`` on a non-zero status.  PyTorch provides device memory and
+streams; all arithmetic runs in the library's CUDA kernels.  There is no CPU
+path: importing works without a GPU (for the build and host-side checks), but
+every call that launches work needs ``libqlora.so`` and an sm_100 device, and
+fails loudly otherwise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqlora.so")
+
+QLORA_F32, QLORA_BF16 = 0, 1
+QLORA_OP_FWD, QLORA_OP_BWD = 1, 2
+BLOCK, GROUP = 64, 256
+
+STATUS_NAMES = {
+    0: "QLORA_OK", 1: "QLORA_ERR_INVALID_ARG", 2: "QLORA_ERR_SHAPE", 3: "QLORA_ERR_ALIGNMENT",
+    4: "QLORA_ERR_WORKSPACE", 5: "QLORA_ERR_UNSUPPORTED_DEVICE", 6: "QLORA_ERR_CUDA",
+    7: "QLORA_ERR_TIMEOUT",
+}
+
+# Every symbol the header declares.
+EXPORTS = (
+    "qlora_quantize_nf4", "qlora_dequantize", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_merge",
+    "qlora_workspace_bytes", "qlora_ws_init", "qlora_ws_status", "qlora_nf4_codebook",
+    "qlora_adapter_params", "qlora_status_string",
+)
+
+
+class QLoRAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+class _Weight(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("dq_codes", ctypes.c_void_p), ("dq_scales", ctypes.c_void_p),
+                ("in_", ctypes.c_int64), ("out", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libqlora.so (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m quantized_rank_fine_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        wp = ctypes.POINTER(_Weight)
+        sig = {
+            "qlora_quantize_nf4": (i32, [vp, i64, i64, vp, vp, vp, vp]),
+            "qlora_dequantize": (i32, [wp, vp, i32, vp]),
+            "qlora_linear_fwd": (i32, [wp, vp, i64, vp, vp, i32, vp, vp, vp, sz, vp]),
+            "qlora_linear_bwd": (i32, [wp, vp, vp, vp, i64, vp, vp, i32, vp, vp, vp, vp, sz, vp]),
+            "qlora_merge": (i32, [wp, vp, vp, i32, vp, i32, vp]),
+            "qlora_workspace_bytes": (sz, [i32, i64, i64, i64, i32]),
+            "qlora_ws_init": (i32, [vp, sz, vp]),
+            "qlora_ws_status": (i32, [vp, vp]),
+            "qlora_nf4_codebook": (None, [ctypes.POINTER(ctypes.c_float)]),
+            "qlora_adapter_params": (i64, [i64, i64, i32]),
+            "qlora_status_string": (ctypes.c_char_p, [i32]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype, f.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise QLoRAError(status, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream=None):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+
+
+@dataclass
+class NF4Weight:
+    """The frozen quantised weight: packed codes, E4M3 absmax codes, fp32 group scales."""
+    codes: torch.Tensor       # uint8 [in*out/2]
+    dq_codes: torch.Tensor    # uint8 [in*out/64]
+    dq_scales: torch.Tensor   # float32 [ceil(in*out/64/256)]
+    n_in: int
+    n_out: int
+
+    def c_struct(self) -> _Weight:
+        return _Weight(_ptr(self.codes), _ptr(self.dq_codes), _ptr(self.dq_scales), self.n_in, self.n_out)
+
+
+def qlora_nf4_codebook() -> list:
+    buf = (ctypes.c_float * 16)()
+    lib().qlora_nf4_codebook(buf)
+    return list(buf)
+
+
+def qlora_adapter_params(n_in: int, n_out: int, r: int) -> int:
+    return lib().qlora_adapter_params(n_in, n_out, r)
+
+
+def qlora_status_string(status: int) -> str:
+    return lib().qlora_status_string(status).decode()
+
+
+def qlora_workspace_bytes(op: int, M: int, n_in: int, n_out: int, r: int) -> int:
+    return lib().qlora_workspace_bytes(op, M, n_in, n_out, r)
+
+
+class Workspace:
+    """Caller-owned scratch of the forward/backward calls (a device uint8 tensor),
+    grown on demand and initialised once through qlora_ws_init."""
+
+    def __init__(self, device=None):
+        self.device = torch.device(device or "cuda")
+        self.buf = None
+
+    def get(self, nbytes: int, stream=None) -> torch.Tensor:
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+            _check(lib().qlora_ws_init(_ptr(self.buf), self.buf.numel(), _stream(stream)), "qlora_ws_init")
+        return self.buf
+
+    def status(self, stream=None) -> int:
+        if self.buf is None:
+            return 0
+        return lib().qlora_ws_status(_ptr(self.buf), _stream(stream))
+
+
+def qlora_quantize_nf4(W0: torch.Tensor, stream=None, out: NF4Weight | None = None) -> NF4Weight:
+    """W0 fp32 (in, out) on the GPU -> NF4Weight (outputs allocated unless given)."""
+    n_in, n_out = W0.shape
+    n = n_in * n_out
+    if out is None:
+        dev = W0.device
+        out = NF4Weight(torch.empty(n // 2, dtype=torch.uint8, device=dev),
+                        torch.empty(n // BLOCK, dtype=torch.uint8, device=dev),
+                        torch.empty((n // BLOCK + GROUP - 1) // GROUP, dtype=torch.float32, device=dev),
+                        n_in, n_out)
+    _check(lib().qlora_quantize_nf4(_ptr(W0), n_in, n_out, _ptr(out.codes), _ptr(out.dq_codes),
+                                    _ptr(out.dq_scales), _stream(stream)), "qlora_quantize_nf4")
+    return out
+
+
+def qlora_dequantize(w: NF4Weight, dtype=torch.float32, stream=None, out=None) -> torch.Tensor:
+    code = QLORA_BF16 if dtype == torch.bfloat16 else QLORA_F32
+    if out is None:
+        out = torch.empty((w.n_in, w.n_out), dtype=dtype, device=w.codes.device)
+    ws = w.c_struct()
+    _check(lib().qlora_dequantize(ctypes.byref(ws), _ptr(out), code, _stream(stream)), "qlora_dequantize")
+    return out
+
+
+def qlora_merge(w: NF4Weight, A: torch.Tensor, B: torch.Tensor, dtype=torch.float32, stream=None,
+                out=None) -> torch.Tensor:
+    code = QLORA_BF16 if dtype == torch.bfloat16 else QLORA_F32
+    if out is None:
+        out = torch.empty((w.n_in, w.n_out), dtype=dtype, device=w.codes.device)
+    ws = w.c_struct()
+    _check(lib().qlora_merge(ctypes.byref(ws), _ptr(A), _ptr(B), A.shape[1], _ptr(out), code, _stream(stream)),
+           "qlora_merge")
+    return out
+
+
+def qlora_linear_fwd(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, workspace: Workspace,
+                     save_V: bool = True, stream=None, Y=None, V=None):
+    """Returns (Y, V) with V = X A (None when save_V is False)."""
+    M, r = X.shape[0], A.shape[1]
+    if Y is None:
+        Y = torch.empty((M, w.n_out), dtype=torch.bfloat16, device=X.device)
+    if save_V and V is None:
+        V = torch.empty((M, r), dtype=torch.bfloat16, device=X.device)
+    nb = qlora_workspace_bytes(QLORA_OP_FWD, M, w.n_in, w.n_out, r)
+    buf = workspace.get(nb, stream)
+    ws = w.c_struct()
+    _check(lib().qlora_linear_fwd(ctypes.byref(ws), _ptr(X), M, _ptr(A), _ptr(B), r, _ptr(Y),
+                                  _ptr(V) if save_V else None, _ptr(buf), buf.numel(), _stream(stream)),
+           "qlora_linear_fwd")
+    return Y, (V if save_V else None)
+
+
+def qlora_linear_bwd(w: NF4Weight, X: torch.Tensor, V, dY: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
+                     workspace: Workspace, need_dX: bool = True, stream=None, dX=None, dA=None, dB=None):
+    """Returns (dX or None, dA fp32 (in, r), dB fp32 (r, out))."""
+    M, r = X.shape[0], A.shape[1]
+    dev = X.device
+    if need_dX and dX is None:
+        dX = torch.empty((M, w.n_in), dtype=torch.bfloat16, device=dev)
+    if dA is None:
+        dA = torch.empty((w.n_in, r), dtype=torch.float32, device=dev)
+    if dB is None:
+        dB = torch.empty((r, w.n_out), dtype=torch.float32, device=dev)
+    nb = qlora_workspace_bytes(QLORA_OP_BWD, M, w.n_in, w.n_out, r)
+    buf = workspace.get(nb, stream)
+    ws = w.c_struct()
+    _check(lib().qlora_linear_bwd(ctypes.byref(ws), _ptr(X), _ptr(V), _ptr(dY), M, _ptr(A), _ptr(B), r,
+                                  _ptr(dX) if need_dX else None, _ptr(dA), _ptr(dB), _ptr(buf), buf.numel(),
+                                  _stream(stream)), "qlora_linear_bwd")
+    return (dX if need_dX else None), dA, dB

@@ -1,0 +1,272 @@
+// The C ABI of libqlora: host-side argument checks, workspace layout, launches.
+// Declarations, argument meaning, layouts and error behaviour: include/qlora.h.
+#include <cuda_runtime.h>
+#include <string.h>
+
+#include "../../include/qlora.h"
+#include "common.cuh"
+#include "kernels.h"
+
+using qlora::WeightView;
+
+namespace {
+
+constexpr size_t kStatusBytes = 256;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Current device must be compute capability 10.0 (B200 / sm_100).
+qlora_status check_device() {
+  static int checked[64] = {};   // 0 unknown, 1 ok, 2 unsupported
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return QLORA_ERR_UNSUPPORTED_DEVICE;
+  if (checked[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    checked[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  return checked[dev] == 1 ? QLORA_OK : QLORA_ERR_UNSUPPORTED_DEVICE;
+}
+
+// A required tensor: non-NULL, device (or managed) memory of the current device, 16-byte aligned.
+qlora_status check_ptr(const void* p, bool required = true) {
+  if (!p) return required ? QLORA_ERR_INVALID_ARG : QLORA_OK;
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_INVALID_ARG;
+  }
+  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return QLORA_ERR_INVALID_ARG;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (a.device != dev) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(p)) return QLORA_ERR_ALIGNMENT;
+  return QLORA_OK;
+}
+
+#define QLORA_TRY(expr)                  \
+  do {                                   \
+    qlora_status _s = (expr);            \
+    if (_s != QLORA_OK) return _s;       \
+  } while (0)
+
+#define QLORA_CUDA(expr)                                 \
+  do {                                                   \
+    if ((expr) != cudaSuccess) return QLORA_ERR_CUDA;    \
+  } while (0)
+
+bool rank_ok(int r) { return r >= 8 && r <= 256 && r % 8 == 0; }
+
+bool linear_shape_ok(int64_t M, int64_t in, int64_t out, int r) {
+  return M >= 1 && M <= (int64_t(1) << 31) - 1 && in >= 64 && out >= 64 && in % 64 == 0 && out % 64 == 0 &&
+         in <= (int64_t(1) << 24) && out <= (int64_t(1) << 24) && rank_ok(r);
+}
+
+qlora_status check_weight_shape(const qlora_nf4_weight* w) {
+  if (!w || !w->codes || !w->dq_codes || !w->dq_scales) return QLORA_ERR_INVALID_ARG;
+  if (w->in < 1 || w->out < 1 || w->in > (int64_t(1) << 40) / w->out || (w->in * w->out) % QLORA_BLOCK != 0)
+    return QLORA_ERR_SHAPE;
+  return QLORA_OK;
+}
+
+qlora_status check_weight(const qlora_nf4_weight* w) {
+  QLORA_TRY(check_weight_shape(w));
+  QLORA_TRY(check_ptr(w->codes));
+  QLORA_TRY(check_ptr(w->dq_codes));
+  QLORA_TRY(check_ptr(w->dq_scales));
+  return QLORA_OK;
+}
+
+WeightView view(const qlora_nf4_weight* w) { return WeightView{w->codes, w->dq_codes, w->dq_scales, w->in, w->out}; }
+
+// Workspace layout (byte offsets), shared by the size query and the calls.
+struct WsLayout {
+  size_t v_off, u_off, part_off, total;
+};
+
+WsLayout ws_layout(int op, int64_t M, int64_t in, int64_t out, int r) {
+  WsLayout L{};
+  const size_t mr = align256(static_cast<size_t>(M) * r * 2);
+  size_t off = kStatusBytes;
+  L.v_off = off;
+  off += mr;
+  size_t parts = 0;
+  if (op == QLORA_OP_FWD) {
+    L.u_off = 0;
+    parts = qlora::skinny_partial_floats(M, r, in);
+  } else {
+    L.u_off = off;
+    off += mr;
+    parts = std::max({qlora::skinny_partial_floats(M, r, in), qlora::skinny_partial_floats(M, r, out),
+                      qlora::skinny_partial_floats(in, r, M), qlora::skinny_partial_floats(out, r, M)});
+  }
+  L.part_off = off;
+  off += align256(parts * 4);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* qlora_status_string(qlora_status s) {
+  switch (s) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_INVALID_ARG: return "invalid argument";
+    case QLORA_ERR_SHAPE: return "unsupported shape";
+    case QLORA_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
+    case QLORA_ERR_UNSUPPORTED_DEVICE: return "device is not sm_100";
+    case QLORA_ERR_CUDA: return "CUDA error";
+    case QLORA_ERR_TIMEOUT: return "bounded wait in a kernel timed out";
+  }
+  return "unknown status";
+}
+
+void qlora_nf4_codebook(float out[16]) {
+  if (!out) return;
+  for (int i = 0; i < 16; ++i) out[i] = qlora::nf4_level(i);
+}
+
+int64_t qlora_adapter_params(int64_t in, int64_t out, int r) { return static_cast<int64_t>(r) * (in + out); }
+
+size_t qlora_workspace_bytes(int op, int64_t M, int64_t in, int64_t out, int r) {
+  if ((op != QLORA_OP_FWD && op != QLORA_OP_BWD) || !linear_shape_ok(M, in, out, r)) return 0;
+  return ws_layout(op, M, in, out, r).total;
+}
+
+qlora_status qlora_ws_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < kStatusBytes) return QLORA_ERR_WORKSPACE;
+  QLORA_TRY(check_device());
+  QLORA_TRY(check_ptr(ws));
+  QLORA_CUDA(cudaMemsetAsync(ws, 0, kStatusBytes, static_cast<cudaStream_t>(stream)));
+  return QLORA_OK;
+}
+
+qlora_status qlora_ws_status(void* ws, void* stream) {
+  if (!ws) return QLORA_ERR_WORKSPACE;
+  QLORA_TRY(check_device());
+  QLORA_TRY(check_ptr(ws));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  QLORA_CUDA(cudaStreamSynchronize(s));
+  uint32_t flag = 0;
+  QLORA_CUDA(cudaMemcpy(&flag, ws, sizeof(flag), cudaMemcpyDeviceToHost));
+  if (flag != 0) {
+    QLORA_CUDA(cudaMemset(ws, 0, sizeof(flag)));
+    return QLORA_ERR_TIMEOUT;
+  }
+  return QLORA_OK;
+}
+
+qlora_status qlora_quantize_nf4(const float* W0, int64_t in, int64_t out, uint8_t* codes, uint8_t* dq_codes,
+                                float* dq_scales, void* stream) {
+  if (!W0 || !codes || !dq_codes || !dq_scales) return QLORA_ERR_INVALID_ARG;
+  if (in < 1 || out < 1 || in > (int64_t(1) << 40) / out || (in * out) % QLORA_BLOCK != 0) return QLORA_ERR_SHAPE;
+  QLORA_TRY(check_device());
+  QLORA_TRY(check_ptr(W0));
+  QLORA_TRY(check_ptr(codes));
+  QLORA_TRY(check_ptr(dq_codes));
+  QLORA_TRY(check_ptr(dq_scales));
+  QLORA_CUDA(qlora::launch_quantize_nf4(W0, in * out, codes, dq_codes, dq_scales, static_cast<cudaStream_t>(stream)));
+  return QLORA_OK;
+}
+
+qlora_status qlora_dequantize(const qlora_nf4_weight* w, void* W_out, int out_dtype, void* stream) {
+  if (out_dtype != QLORA_F32 && out_dtype != QLORA_BF16 || !W_out) return QLORA_ERR_INVALID_ARG;
+  QLORA_TRY(check_weight_shape(w));
+  QLORA_TRY(check_device());
+  QLORA_TRY(check_weight(w));
+  QLORA_TRY(check_ptr(W_out));
+  QLORA_CUDA(qlora::launch_dequantize(w->codes, w->dq_codes, w->dq_scales, w->in * w->out, out_dtype == QLORA_BF16,
+                                      W_out, static_cast<cudaStream_t>(stream)));
+  return QLORA_OK;
+}
+
+qlora_status qlora_merge(const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B, int r, void* W_out,
+                         int out_dtype, void* stream) {
+  if (out_dtype != QLORA_F32 && out_dtype != QLORA_BF16 || !A || !B || !W_out) return QLORA_ERR_INVALID_ARG;
+  QLORA_TRY(check_weight_shape(w));
+  if (!linear_shape_ok(1, w->in, w->out, r) || w->in > (int64_t(1) << 21)) return QLORA_ERR_SHAPE;
+  QLORA_TRY(check_device());
+  QLORA_TRY(check_weight(w));
+  QLORA_TRY(check_ptr(A));
+  QLORA_TRY(check_ptr(B));
+  QLORA_TRY(check_ptr(W_out));
+  QLORA_CUDA(qlora::launch_merge(w->codes, w->dq_codes, w->dq_scales, A, B, r, w->in, w->out,
+                                 out_dtype == QLORA_BF16, W_out, static_cast<cudaStream_t>(stream)));
+  return QLORA_OK;
+}
+
+qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int64_t M, const uint16_t* A,
+                              const uint16_t* B, int r, uint16_t* Y, uint16_t* V_save, void* ws, size_t ws_bytes,
+                              void* stream) {
+  if (!X || !A || !B || !Y) return QLORA_ERR_INVALID_ARG;
+  QLORA_TRY(check_weight_shape(w));
+  if (!linear_shape_ok(M, w->in, w->out, r)) return QLORA_ERR_SHAPE;
+  if (!ws || ws_bytes < ws_layout(QLORA_OP_FWD, M, w->in, w->out, r).total) return QLORA_ERR_WORKSPACE;
+  QLORA_TRY(check_device());
+  QLORA_TRY(check_weight(w));
+  QLORA_TRY(check_ptr(X));
+  QLORA_TRY(check_ptr(A));
+  QLORA_TRY(check_ptr(B));
+  QLORA_TRY(check_ptr(Y));
+  QLORA_TRY(check_ptr(V_save, false));
+  const WsLayout L = ws_layout(QLORA_OP_FWD, M, w->in, w->out, r);
+  if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  QLORA_TRY(check_ptr(ws));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint32_t* status = reinterpret_cast<uint32_t*>(base);
+  uint16_t* V = V_save ? V_save : reinterpret_cast<uint16_t*>(base + L.v_off);
+  float* part = reinterpret_cast<float*>(base + L.part_off);
+  const WeightView wv = view(w);
+  QLORA_CUDA(qlora::launch_xa(X, A, M, w->in, r, V, part, s));
+  QLORA_CUDA(qlora::launch_fwd_gemm(wv, X, V, B, M, r, Y, status, s));
+  return QLORA_OK;
+}
+
+qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16_t* X, const uint16_t* V, const uint16_t* dY,
+                              int64_t M, const uint16_t* A, const uint16_t* B, int r, uint16_t* dX, float* dA,
+                              float* dB, void* ws, size_t ws_bytes, void* stream) {
+  if (!X || !dY || !A || !B || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  QLORA_TRY(check_weight_shape(w));
+  if (!linear_shape_ok(M, w->in, w->out, r)) return QLORA_ERR_SHAPE;
+  if (!ws || ws_bytes < ws_layout(QLORA_OP_BWD, M, w->in, w->out, r).total) return QLORA_ERR_WORKSPACE;
+  QLORA_TRY(check_device());
+  QLORA_TRY(check_weight(w));
+  QLORA_TRY(check_ptr(X));
+  QLORA_TRY(check_ptr(V, false));
+  QLORA_TRY(check_ptr(dY));
+  QLORA_TRY(check_ptr(A));
+  QLORA_TRY(check_ptr(B));
+  QLORA_TRY(check_ptr(dX, false));
+  QLORA_TRY(check_ptr(dA));
+  QLORA_TRY(check_ptr(dB));
+  const WsLayout L = ws_layout(QLORA_OP_BWD, M, w->in, w->out, r);
+  if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  QLORA_TRY(check_ptr(ws));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint32_t* status = reinterpret_cast<uint32_t*>(base);
+  uint16_t* U = reinterpret_cast<uint16_t*>(base + L.u_off);
+  float* part = reinterpret_cast<float*>(base + L.part_off);
+  const WeightView wv = view(w);
+  if (!V) {
+    uint16_t* Vw = reinterpret_cast<uint16_t*>(base + L.v_off);
+    QLORA_CUDA(qlora::launch_xa(X, A, M, w->in, r, Vw, part, s));
+    V = Vw;
+  }
+  QLORA_CUDA(qlora::launch_dybt(dY, B, M, w->out, r, U, part, s));
+  QLORA_CUDA(qlora::launch_vtdy(V, dY, M, w->out, r, dB, part, s));
+  QLORA_CUDA(qlora::launch_xtu(X, U, M, w->in, r, dA, part, s));
+  if (dX) QLORA_CUDA(qlora::launch_dx_gemm(wv, dY, U, A, M, r, dX, status, s));
+  return QLORA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,169 @@
+// Dense dequantisation and adapter merge of the frozen NF4 weight.
+//
+// dequantize ("LLMs · QLoRA": levels[idx] * scale; "What QLoRA adds over LoRA":
+// absmax quantised to 8 bits, weights dequantised to bf16):
+//   a'_b = fl32(e4m3(dq_code_b) * s_g),  w' = fl32(level[code] * a'_b),
+//   written as fp32 or as bf16(w').  Plain binary32 products, no FMA contraction,
+//   so the result is bit-exact.
+// merge ("QLoRA (low-rank adapters on a quantized model)", "How it works" step 5):
+//   W = w' + A B with fp32 accumulation over the rank.
+//
+// Both are HBM-bound streaming kernels: each thread handles 16 consecutive
+// weights (8 code bytes, one 64-byte fp32 or 32-byte bf16 output run), so every
+// warp reads 256 contiguous code bytes and writes 2 KB (fp32) contiguously.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace qlora {
+
+namespace {
+
+constexpr int kDqThreads = 256;
+
+template <bool kBf16>
+__global__ void __launch_bounds__(kDqThreads)
+dequantize_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ dq_codes,
+                  const float* __restrict__ dq_scales, int64_t n16, void* __restrict__ out) {
+  __shared__ float lv[16];
+  if (threadIdx.x < 16) lv[threadIdx.x] = nf4_level(threadIdx.x);
+  __syncthreads();
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kDqThreads + threadIdx.x;
+  if (t >= n16) return;
+  const int64_t blk = t >> 2;                       // 4 threads per 64-weight block
+  const float a = absmax_deq(dq_codes[blk], dq_scales[blk / kGroup]);
+  const uint2 c = __ldcs(reinterpret_cast<const uint2*>(codes) + t);
+  float w[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t word = (i < 4) ? c.x : c.y;
+    const uint32_t byte = (word >> (8 * (i & 3))) & 0xFFu;
+    w[2 * i] = mul_rn(lv[byte & 0xF], a);
+    w[2 * i + 1] = mul_rn(lv[byte >> 4], a);
+  }
+  if constexpr (kBf16) {
+    uint4* o = reinterpret_cast<uint4*>(out) + 2 * t;
+    uint4 p0, p1;
+    p0.x = pack_bf16x2(w[0], w[1]);   p0.y = pack_bf16x2(w[2], w[3]);
+    p0.z = pack_bf16x2(w[4], w[5]);   p0.w = pack_bf16x2(w[6], w[7]);
+    p1.x = pack_bf16x2(w[8], w[9]);   p1.y = pack_bf16x2(w[10], w[11]);
+    p1.z = pack_bf16x2(w[12], w[13]); p1.w = pack_bf16x2(w[14], w[15]);
+    __stcs(o, p0);
+    __stcs(o + 1, p1);
+  } else {
+    float4* o = reinterpret_cast<float4*>(out) + 4 * t;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      __stcs(o + i, make_float4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]));
+  }
+}
+
+// Merge: CTA tile of 32 rows x 256 columns; thread (ty, tx) owns columns
+// 8tx .. 8tx+7 of rows ty, ty+8, ty+16, ty+24.  The rank is consumed in slices
+// of 32 staged in shared memory as fp32.
+constexpr int kMgRows = 32, kMgCols = 256, kMgR = 32;
+
+template <bool kBf16>
+__global__ void __launch_bounds__(256)
+merge_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ dq_codes,
+             const float* __restrict__ dq_scales, const __nv_bfloat16* __restrict__ A,
+             const __nv_bfloat16* __restrict__ B, int r, int64_t n_in, int64_t n_out,
+             void* __restrict__ out) {
+  __shared__ float sA[kMgRows][kMgR + 1];
+  __shared__ __align__(16) float sB[kMgR][kMgCols];
+  __shared__ float lv[16];
+  const int tid = threadIdx.x, tx = tid & 31, ty = tid >> 5;
+  if (tid < 16) lv[tid] = nf4_level(tid);
+  const int64_t row0 = static_cast<int64_t>(blockIdx.y) * kMgRows;
+  const int64_t col0 = static_cast<int64_t>(blockIdx.x) * kMgCols;
+
+  float acc[4][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+
+  for (int j0 = 0; j0 < r; j0 += kMgR) {
+    __syncthreads();
+    for (int e = tid; e < kMgRows * kMgR; e += 256) {
+      const int rr = e / kMgR, jj = e % kMgR;
+      const int64_t row = row0 + rr;
+      sA[rr][jj] = (row < n_in && j0 + jj < r) ? __bfloat162float(A[row * r + j0 + jj]) : 0.0f;
+    }
+    for (int e = tid; e < kMgR * kMgCols; e += 256) {
+      const int jj = e / kMgCols, cc = e % kMgCols;
+      const int64_t col = col0 + cc;
+      sB[jj][cc] = (col < n_out && j0 + jj < r) ? __bfloat162float(B[(j0 + jj) * n_out + col]) : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int jj = 0; jj < kMgR; ++jj) {
+      float b[8];
+      const float4 b0 = *reinterpret_cast<const float4*>(&sB[jj][8 * tx]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&sB[jj][8 * tx + 4]);
+      b[0] = b0.x; b[1] = b0.y; b[2] = b0.z; b[3] = b0.w;
+      b[4] = b1.x; b[5] = b1.y; b[6] = b1.z; b[7] = b1.w;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float a = sA[ty + 8 * i][jj];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a, b[j], acc[i][j]);
+      }
+    }
+  }
+
+  const int64_t col = col0 + 8 * tx;
+  if (col >= n_out) return;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t row = row0 + ty + 8 * i;
+    if (row >= n_in) continue;
+    const int64_t e0 = row * n_out + col;                 // multiple of 8
+    const int64_t blk = e0 / kBlock;
+    const float a = absmax_deq(dq_codes[blk], dq_scales[blk / kGroup]);
+    const uint32_t c = *reinterpret_cast<const uint32_t*>(codes + e0 / 2);
+    float w[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) w[j] = __fadd_rn(mul_rn(lv[(c >> (4 * j)) & 0xF], a), acc[i][j]);
+    if constexpr (kBf16) {
+      uint4 p;
+      p.x = pack_bf16x2(w[0], w[1]); p.y = pack_bf16x2(w[2], w[3]);
+      p.z = pack_bf16x2(w[4], w[5]); p.w = pack_bf16x2(w[6], w[7]);
+      *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(out) + e0) = p;
+    } else {
+      float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + e0);
+      o[0] = make_float4(w[0], w[1], w[2], w[3]);
+      o[1] = make_float4(w[4], w[5], w[6], w[7]);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* dq_codes,
+                              const float* dq_scales, int64_t n, bool bf16, void* out,
+                              cudaStream_t stream) {
+  const int64_t n16 = n / 16;
+  if (n16 == 0) return cudaSuccess;
+  const unsigned grid = static_cast<unsigned>((n16 + kDqThreads - 1) / kDqThreads);
+  if (bf16)
+    dequantize_kernel<true><<<grid, kDqThreads, 0, stream>>>(codes, dq_codes, dq_scales, n16, out);
+  else
+    dequantize_kernel<false><<<grid, kDqThreads, 0, stream>>>(codes, dq_codes, dq_scales, n16, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge(const uint8_t* codes, const uint8_t* dq_codes, const float* dq_scales,
+                         const uint16_t* A, const uint16_t* B, int r, int64_t n_in,
+                         int64_t n_out, bool bf16, void* out, cudaStream_t stream) {
+  dim3 grid(static_cast<unsigned>((n_out + kMgCols - 1) / kMgCols),
+            static_cast<unsigned>((n_in + kMgRows - 1) / kMgRows));
+  const auto* a = reinterpret_cast<const __nv_bfloat16*>(A);
+  const auto* b = reinterpret_cast<const __nv_bfloat16*>(B);
+  if (bf16)
+    merge_kernel<true><<<grid, 256, 0, stream>>>(codes, dq_codes, dq_scales, a, b, r, n_in, n_out, out);
+  else
+    merge_kernel<false><<<grid, 256, 0, stream>>>(codes, dq_codes, dq_scales, a, b, r, n_in, n_out, out);
+  return cudaGetLastError();
+}
+
+}  // namespace qlora

@@ -1,0 +1,362 @@
+// Fused NF4-dequant GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM).
+//
+//   forward  Y  = [X | V] . [deq(Wq) ; B]      (M x out, K = in + r)
+//   dX       dX = [dY | U] . [deq(Wq)^T ; A^T] (M x in,  K = out + r)
+//
+// ("How it works" steps 2-4 and "What QLoRA adds over LoRA" of "QLoRA (low-rank
+// adapters on a quantized model)": the frozen weight is dequantised to bf16 for
+// each matmul; the adapter product (X A) B, and U A^T in the backward, is the
+// same contraction extended by r along K, so it lands in the same accumulator.)
+//
+// CTA tile 256 (M) x 256 (N), K step 64, 3-stage shared-memory ring, one CTA per
+// SM.  Two UMMA M=128 x N=256 accumulators fill the 512 TMEM columns; both use
+// the same dequantised weight tile, so each weight is dequantised M/256 times.
+// Warp roles (320 threads):
+//   warp 0     TMA producer: activation tile (256 x 64 bf16, 128B swizzle) and,
+//              for the adapter K-steps, the V/U tile and the B/A tile.
+//   warp 1     TMEM allocation + the single thread that issues tcgen05.mma.
+//   warps 2-9  dequant producers (one thread per 64-weight block per K-step):
+//              raw codes from global memory -> per-block 16-entry bf16 table ->
+//              byte-permute lookup -> 16-byte stores in the UMMA canonical
+//              layout; then the epilogue (TMEM -> registers -> bf16 -> global).
+// The weight tile is written MN-major for the forward (N contiguous in W) and
+// K-major for dX (K contiguous in W), so the dequant never transposes.
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+#include <cudaTypedefs.h>
+
+namespace qlora {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = 256, kBN = 256, kBK = 64, kStages = 3;
+constexpr int kThreads = 320;
+constexpr int kDeqWarps = 8;
+constexpr uint32_t kABytes = kBM * kBK * 2;     // 32 KB
+constexpr uint32_t kBBytes = kBN * kBK * 2;     // 32 KB
+constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 + 256;
+constexpr uint32_t kTmemCols = 512;
+
+struct GemmArgs {
+  const uint8_t* codes;
+  const uint8_t* dq_codes;
+  const float* dq_scales;
+  int64_t w_out;      // columns of the stored weight (out)
+  int64_t M, N, K;    // output M x N, weight reduction length K (multiple of 64)
+  int r;
+  uint16_t* D;        // bf16 (M, N)
+  uint32_t* status;
+};
+
+// Per-block table: v_j = bf16(fl32(level_j * a)) for j = 0..15, split into the
+// low bytes (lo[0..3]) and high bytes (hi[0..3]) of the 16 entries, 4 per word.
+struct BlockLut {
+  uint32_t lo[4], hi[4];
+};
+
+__device__ __forceinline__ BlockLut make_lut(float a) {
+  uint32_t pr[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    pr[i] = pack_bf16x2(mul_rn(nf4_level(2 * i), a), mul_rn(nf4_level(2 * i + 1), a));
+  BlockLut t;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    t.lo[q] = __byte_perm(pr[2 * q], pr[2 * q + 1], 0x6420);
+    t.hi[q] = __byte_perm(pr[2 * q], pr[2 * q + 1], 0x7531);
+  }
+  return t;
+}
+
+// Four 4-bit codes (nibbles of x, element order low to high) -> two bf16x2 words.
+__device__ __forceinline__ void lut4(const BlockLut& t, uint32_t x, uint32_t& o01, uint32_t& o23) {
+  const uint32_t s_lo = x & 0x7777u;                              // index within a half table
+  const uint32_t s_pick = 0x3210u | ((x >> 1) & 0x4444u);         // +4 where the code is >= 8
+  const uint32_t lo = __byte_perm(__byte_perm(t.lo[0], t.lo[1], s_lo),
+                                  __byte_perm(t.lo[2], t.lo[3], s_lo), s_pick);
+  const uint32_t hi = __byte_perm(__byte_perm(t.hi[0], t.hi[1], s_lo),
+                                  __byte_perm(t.hi[2], t.hi[3], s_lo), s_pick);
+  o01 = __byte_perm(lo, hi, 0x5140);
+  o23 = __byte_perm(lo, hi, 0x7362);
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
+template <bool kDX>
+__global__ void __launch_bounds__(kThreads, 1)
+nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_ext_a,
+                const __grid_constant__ CUtensorMap tm_ext_b, const GemmArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 1);
+  const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + kStages);
+  const uint32_t tmem_full = smem_addr(bars + 2 * kStages);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kBN;
+  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kBM;
+  const int nkb_w = static_cast<int>(p.K / kBK);
+  const int n_ext = (p.r + kBK - 1) / kBK;
+  const int nkb = nkb_w + n_ext;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full0 + 8 * s, 1 + kDeqWarps);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init(tmem_full, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_act);
+    tma_prefetch_desc(&tm_ext_a);
+    tma_prefetch_desc(&tm_ext_b);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % kStages;
+        const uint32_t ph = (kb / kStages) & 1;
+        if (!mbar_wait(empty0 + 8 * s, ph ^ 1, p.status, kFlagTimeoutProducer)) break;
+        const uint32_t a_dst = smem_addr(smem + s * kStageBytes);
+        const uint32_t b_dst = a_dst + kABytes;
+        if (kb < nkb_w) {
+          mbar_arrive_expect_tx(full0 + 8 * s, kABytes);
+          tma_load_2d(a_dst, &tm_act, full0 + 8 * s, kb * kBK, static_cast<int32_t>(m0));
+        } else {
+          const int j = kb - nkb_w;
+          mbar_arrive_expect_tx(full0 + 8 * s, kABytes + kBBytes);
+          tma_load_2d(a_dst, &tm_ext_a, full0 + 8 * s, j * kBK, static_cast<int32_t>(m0));
+          if (!kDX) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              tma_load_2d(b_dst + i * 8192, &tm_ext_b, full0 + 8 * s, static_cast<int32_t>(n0 + 64 * i), j * kBK);
+          } else {
+            tma_load_2d(b_dst, &tm_ext_b, full0 + 8 * s, j * kBK, static_cast<int32_t>(n0));
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, 256, false, !kDX);
+      bool ok = true;
+      for (int kb = 0; kb < nkb && ok; ++kb) {
+        const int s = kb % kStages;
+        const uint32_t ph = (kb / kStages) & 1;
+        if (!mbar_wait(full0 + 8 * s, ph, p.status, kFlagTimeoutMma)) { ok = false; break; }
+        tc_fence_after();
+        int nk16 = 4;
+        if (kb >= nkb_w) nk16 = min(4, (p.r - (kb - nkb_w) * kBK + 15) / 16);
+        const uint32_t a_base = smem_addr(smem + s * kStageBytes);
+        const uint32_t b_base = a_base + kABytes;
+        for (int kk = 0; kk < nk16; ++kk) {
+          const uint64_t bdesc = kDX ? smem_desc_sw128(b_base + kk * 32, 16, 1024)
+                                     : smem_desc_sw128(b_base + kk * 2048, 8192, 1024);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint64_t adesc = smem_desc_sw128(a_base + h * 16384 + kk * 32, 16, 1024);
+            umma_bf16(tmem_base + h * 256, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+        }
+        umma_commit(empty0 + 8 * s);
+      }
+      umma_commit(tmem_full);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ dequant producers
+    const int t = threadIdx.x - 64;                 // 0..255: one 64-weight block each
+    const int64_t blocks_per_row = p.w_out / kBlock;
+    int64_t blk;                                    // block index at kb = 0
+    bool valid;
+    uint32_t row_off;                               // byte offset of this thread's 8 chunks
+    int swz;
+    if (!kDX) {
+      const int kr = t >> 2, j = t & 3;             // k row in tile, 64-wide n block
+      valid = (n0 + 64 * j) < p.N;
+      blk = static_cast<int64_t>(kr) * blocks_per_row + (n0 >> 6) + j;
+      row_off = j * 8192 + (kr >> 3) * 1024 + (kr & 7) * 128;
+      swz = kr & 7;
+    } else {
+      const int nr = t;
+      valid = (n0 + nr) < p.N;
+      blk = (n0 + nr) * blocks_per_row;
+      row_off = nr * 128;
+      swz = nr & 7;
+    }
+    // K-step kb moves the block index by 64 rows (forward) or 1 block (dX).
+    const int64_t blk_step = kDX ? 1 : 64 * blocks_per_row;
+
+    uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0;
+    uint8_t dqc = 0;
+    float dqs = 0.0f;
+    if (valid && nkb_w > 0) {
+      const uint4* src = reinterpret_cast<const uint4*>(p.codes + blk * 32);
+      c0 = __ldg(src);
+      c1 = __ldg(src + 1);
+      dqc = __ldg(p.dq_codes + blk);
+      dqs = __ldg(p.dq_scales + blk / kGroup);
+    }
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % kStages;
+      const uint32_t ph = (kb / kStages) & 1;
+      // every lane waits; the warp leaves the loop together if the wait gave up
+      const bool got = mbar_wait(empty0 + 8 * s, ph ^ 1, p.status, kFlagTimeoutProducer);
+      if (!__all_sync(0xffffffffu, got)) break;
+      if (kb < nkb_w) {
+        const uint32_t dst = smem_addr(smem + s * kStageBytes + kABytes) + row_off;
+        const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const BlockLut lut = make_lut(valid ? absmax_deq(dqc, dqs) : 0.0f);
+        // prefetch the next K-step's block
+        if (valid && kb + 1 < nkb_w) {
+          const int64_t nb = blk + (kb + 1) * blk_step;
+          const uint4* src = reinterpret_cast<const uint4*>(p.codes + nb * 32);
+          c0 = __ldg(src);
+          c1 = __ldg(src + 1);
+          dqc = __ldg(p.dq_codes + nb);
+          dqs = __ldg(p.dq_scales + nb / kGroup);
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t o0, o1, o2, o3;
+          lut4(lut, w[c] & 0xFFFFu, o0, o1);
+          lut4(lut, w[c] >> 16, o2, o3);
+          st_shared_v4(dst + ((c ^ swz) << 4), o0, o1, o2, o3);
+        }
+        fence_proxy_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(full0 + 8 * s);
+    }
+
+    // ------------------------------------------------------------ epilogue
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(tmem_full, 0, p.status, kFlagTimeoutEpilogue));
+    tc_fence_after();
+    if (ok) {
+      const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
+      const int half = (warp - 2) >> 2;             // which M=128 accumulator
+      const int64_t row = m0 + half * 128 + quarter * 32 + lane;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + half * 256;
+#pragma unroll 1
+      for (int cb = 0; cb < kBN / 32; ++cb) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(taddr + cb * 32, v);
+        tmem_ld_wait();
+        const int64_t col = n0 + cb * 32;
+        if (row < p.M && col < p.N) {
+          uint4* dst = reinterpret_cast<uint4*>(p.D + row * p.N + col);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 o;
+            o.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
+            o.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
+            o.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
+            o.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
+            dst[q] = o;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// Row-major bf16 matrix (rows x cols) -> 2-D tensor map with a (box_cols x box_rows)
+// box and 128-byte swizzle; box_cols * 2 must be <= 128.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_cols, int box_rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols * 2)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult rc = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return rc == CUDA_SUCCESS;
+}
+
+template <bool kDX>
+cudaError_t launch_gemm(const CUtensorMap& act, const CUtensorMap& ea, const CUtensorMap& eb, const GemmArgs& a,
+                        cudaStream_t stream) {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(nf4_gemm_kernel<kDX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kSmemBytes));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  dim3 grid(static_cast<unsigned>((a.N + kBN - 1) / kBN), static_cast<unsigned>((a.M + kBM - 1) / kBM));
+  nf4_gemm_kernel<kDX><<<grid, kThreads, kSmemBytes, stream>>>(act, ea, eb, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// Y = X deq(W) + V B.
+cudaError_t launch_fwd_gemm(const WeightView& w, const uint16_t* X, const uint16_t* V, const uint16_t* B,
+                            int64_t M, int r, uint16_t* Y, uint32_t* status, cudaStream_t stream) {
+  CUtensorMap act, ea, eb;
+  if (!make_map(&act, X, M, w.in, 64, 256) || !make_map(&ea, V, M, r, 64, 256) ||
+      !make_map(&eb, B, r, w.out, 64, 64))
+    return cudaErrorInvalidValue;
+  GemmArgs a{w.codes, w.dq_codes, w.dq_scales, w.out, M, w.out, w.in, r, Y, status};
+  return launch_gemm<false>(act, ea, eb, a, stream);
+}
+
+// dX = dY deq(W)^T + U A^T.
+cudaError_t launch_dx_gemm(const WeightView& w, const uint16_t* dY, const uint16_t* U, const uint16_t* A,
+                           int64_t M, int r, uint16_t* dX, uint32_t* status, cudaStream_t stream) {
+  CUtensorMap act, ea, eb;
+  if (!make_map(&act, dY, M, w.out, 64, 256) || !make_map(&ea, U, M, r, 64, 256) ||
+      !make_map(&eb, A, w.in, r, 64, 256))
+    return cudaErrorInvalidValue;
+  GemmArgs a{w.codes, w.dq_codes, w.dq_scales, w.out, M, w.in, w.out, r, dX, status};
+  return launch_gemm<true>(act, ea, eb, a, stream);
+}
+
+}  // namespace qlora

@@ -1,0 +1,47 @@
+// Internal launch functions of libqlora (host side).  Every function enqueues
+// on `stream` and returns the launch status; arguments are already validated.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+namespace qlora {
+
+constexpr int kMaxSplits = 16;   // most K/M splits of the rank-r kernels
+
+struct WeightView {
+  const uint8_t* codes;
+  const uint8_t* dq_codes;
+  const float* dq_scales;
+  int64_t in, out;
+};
+
+cudaError_t launch_quantize_nf4(const float* W0, int64_t n, uint8_t* codes, uint8_t* dq_codes,
+                                float* dq_scales, cudaStream_t stream);
+cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* dq_codes, const float* dq_scales,
+                              int64_t n, bool bf16, void* out, cudaStream_t stream);
+cudaError_t launch_merge(const uint8_t* codes, const uint8_t* dq_codes, const float* dq_scales,
+                         const uint16_t* A, const uint16_t* B, int r, int64_t n_in, int64_t n_out,
+                         bool bf16, void* out, cudaStream_t stream);
+
+// Rank-r products; `part` is fp32 scratch of skinny_partial_floats(...) floats.
+size_t skinny_partial_floats(int64_t out_rows, int r, int64_t k_total);
+cudaError_t launch_xa(const uint16_t* X, const uint16_t* A, int64_t M, int64_t n_in, int r, uint16_t* V,
+                      float* part, cudaStream_t stream);
+cudaError_t launch_dybt(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t n_out, int r,
+                        uint16_t* U, float* part, cudaStream_t stream);
+cudaError_t launch_xtu(const uint16_t* X, const uint16_t* U, int64_t M, int64_t n_in, int r, float* dA,
+                       float* part, cudaStream_t stream);
+cudaError_t launch_vtdy(const uint16_t* V, const uint16_t* dY, int64_t M, int64_t n_out, int r,
+                        float* dB, float* part, cudaStream_t stream);
+
+// Fused dequant GEMMs (tcgen05); `status` is the workspace status word.
+cudaError_t launch_fwd_gemm(const WeightView& w, const uint16_t* X, const uint16_t* V, const uint16_t* B,
+                            int64_t M, int r, uint16_t* Y, uint32_t* status, cudaStream_t stream);
+cudaError_t launch_dx_gemm(const WeightView& w, const uint16_t* dY, const uint16_t* U, const uint16_t* A,
+                           int64_t M, int r, uint16_t* dX, uint32_t* status, cudaStream_t stream);
+
+}  // namespace qlora

@@ -1,0 +1,102 @@
+"""Host-side checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments before touching a device (CPU only)."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import quantized_rank_fine_b200 as q
+from oracle import nf4
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "qlora.h")
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qlora_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(q.LIB_PATH):
+        from quantized_rank_fine_b200 import build
+        build.build()
+    return q.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = header_functions()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(q.EXPORTS)
+
+
+def test_codebook_equals_oracle(L):
+    """The library's constant levels are the oracle's codebook, bit for bit."""
+    got = np.array(q.qlora_nf4_codebook(), dtype=np.float32)
+    assert np.array_equal(got.view(np.uint32), nf4.nf4_codebook().view(np.uint32))
+
+
+def test_adapter_params_and_status_strings(L):
+    assert q.qlora_adapter_params(4096, 4096, 16) == 131072
+    assert q.qlora_adapter_params(768, 2304, 8) == 24576
+    for s in range(8):
+        assert len(q.qlora_status_string(s)) > 0
+
+
+def test_workspace_bytes(L):
+    assert q.qlora_workspace_bytes(q.QLORA_OP_FWD, 4096, 4096, 4096, 16) >= 256 + 4096 * 16 * 2
+    assert q.qlora_workspace_bytes(q.QLORA_OP_BWD, 4096, 4096, 4096, 16) >= 256 + 2 * 4096 * 16 * 2
+    assert q.qlora_workspace_bytes(q.QLORA_OP_FWD, 64, 256, 256, 7) == 0      # r % 8 != 0
+    assert q.qlora_workspace_bytes(q.QLORA_OP_FWD, 64, 100, 256, 8) == 0      # in % 64 != 0
+    assert q.qlora_workspace_bytes(q.QLORA_OP_FWD, 0, 256, 256, 8) == 0       # M = 0
+    assert q.qlora_workspace_bytes(9, 64, 256, 256, 8) == 0                   # unknown op
+
+
+FAKE = ctypes.c_void_p(0x10000)   # never dereferenced: every case below fails before device access
+
+
+def test_quantize_rejects_before_launch(L):
+    assert L.qlora_quantize_nf4(None, 64, 64, FAKE, FAKE, FAKE, None) == 1
+    assert L.qlora_quantize_nf4(FAKE, 3, 7, FAKE, FAKE, FAKE, None) == 2
+    assert L.qlora_quantize_nf4(FAKE, 0, 64, FAKE, FAKE, FAKE, None) == 2
+
+
+def test_linear_rejects_before_launch(L):
+    w = q._Weight(0x10000, 0x10000, 0x10000, 256, 256)
+    wp = ctypes.byref(w)
+    fwd, bwd = L.qlora_linear_fwd, L.qlora_linear_bwd
+    assert fwd(wp, None, 64, FAKE, FAKE, 8, FAKE, None, FAKE, 1 << 30, None) == 1        # X NULL
+    assert fwd(wp, FAKE, 64, FAKE, FAKE, 12, FAKE, None, FAKE, 1 << 30, None) == 2       # r % 8
+    assert fwd(wp, FAKE, 0, FAKE, FAKE, 8, FAKE, None, FAKE, 1 << 30, None) == 2         # M = 0
+    assert fwd(wp, FAKE, 64, FAKE, FAKE, 8, FAKE, None, FAKE, 16, None) == 4             # ws too small
+    assert fwd(wp, FAKE, 64, FAKE, FAKE, 8, FAKE, None, None, 1 << 30, None) == 4        # ws NULL
+    w2 = q._Weight(0x10000, 0x10000, 0x10000, 256, 100)                               # out % 64
+    assert fwd(ctypes.byref(w2), FAKE, 64, FAKE, FAKE, 8, FAKE, None, FAKE, 1 << 30, None) == 2
+    assert bwd(wp, FAKE, None, FAKE, 64, FAKE, FAKE, 8, None, None, FAKE, FAKE, 1 << 30, None) == 1
+    assert bwd(wp, FAKE, None, FAKE, 64, FAKE, FAKE, 264, None, FAKE, FAKE, FAKE, 1 << 30, None) == 2
+    assert bwd(wp, FAKE, None, FAKE, 64, FAKE, FAKE, 8, None, FAKE, FAKE, FAKE, 8, None) == 4
+    w0 = q._Weight(0, 0x10000, 0x10000, 256, 256)                                      # codes NULL
+    assert fwd(ctypes.byref(w0), FAKE, 64, FAKE, FAKE, 8, FAKE, None, FAKE, 1 << 30, None) == 1
+
+
+def test_dequant_merge_reject_before_launch(L):
+    w = q._Weight(0x10000, 0x10000, 0x10000, 256, 256)
+    assert L.qlora_dequantize(ctypes.byref(w), FAKE, 5, None) == 1                      # bad dtype
+    assert L.qlora_dequantize(None, FAKE, 0, None) == 1
+    assert L.qlora_merge(ctypes.byref(w), FAKE, FAKE, 4, FAKE, 0, None) == 2           # r < 8
+    assert L.qlora_merge(ctypes.byref(w), None, FAKE, 8, FAKE, 0, None) == 1
+
+
+def test_no_gpu_means_loud_error_not_fallback(L):
+    """With no usable sm_100 device the calls report an error instead of computing."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert L.qlora_quantize_nf4(FAKE, 64, 64, FAKE, FAKE, FAKE, None) in (5, 6)

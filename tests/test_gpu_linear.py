@@ -1,0 +1,132 @@
+"""GPU parity of the adapted linear layer (forward and backward) against the
+float64 oracle: relative Frobenius error <= 1e-2 and max-abs error <= 2e-2 of
+max |ref| on Y, V, dX, dA, dB; exact invariants where the method fixes them."""
+
+import numpy as np
+import pytest
+import torch
+
+import quantized_rank_fine_b200 as q
+import synth
+from oracle import linear
+from tests.helpers import assert_close, layer_on_gpu, oracle_weight, require_gpu, run_fwd_bwd
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def full_check(t, w, out):
+    Wq = oracle_weight(w)
+    Y, V = linear.forward(t["X"], t["A"], t["B"], Wq)
+    g = linear.backward(t["X"], t["A"], t["B"], Wq, t["dY"])
+    assert_close(out["Y"], Y, "Y")
+    assert_close(out["V"], V, "V")
+    assert_close(out["dX"], g["dX"], "dX")
+    assert_close(out["dA"], g["dA"], "dA")
+    assert_close(out["dB"], g["dB"], "dB")
+
+
+def test_linear_256_m64_r8_full():
+    """The small configuration: in = out = 256, M = 64, r = 8, every output."""
+    t, w = layer_on_gpu(256, 256, 64, 8)
+    full_check(t, w, run_fwd_bwd(t, w))
+
+
+@pytest.mark.parametrize("M,n_in,n_out,r", [
+    (1, 64, 64, 8), (7, 192, 320, 16), (300, 320, 192, 24), (257, 512, 768, 64),
+    (130, 256, 512, 72), (513, 128, 1024, 256), (64, 1024, 64, 8), (1000, 576, 704, 40),
+])
+def test_linear_ragged_shapes(M, n_in, n_out, r):
+    """Ragged M and N tiles, K not a multiple of the tile, several adapter K-steps."""
+    t, w = layer_on_gpu(n_in, n_out, M, r, tag="ragged")
+    full_check(t, w, run_fwd_bwd(t, w))
+
+
+def test_B_zero_invariants():
+    """B = 0: dA is exactly zero, and the forward output does not depend on A
+    at all (the adapter adds exact zeros to the accumulator)."""
+    t, w = layer_on_gpu(320, 448, 200, 16, zero_B=True)
+    out = run_fwd_bwd(t, w)
+    assert torch.count_nonzero(out["dA"]).item() == 0
+    t2 = dict(t)
+    t2["A"] = synth.normal("otherA", t["A"].shape, 0.5, torch.bfloat16, "cuda")
+    out2 = run_fwd_bwd(t2, w)
+    assert torch.equal(out["Y"], out2["Y"])
+    full_check(t, w, out)
+
+
+def test_frozen_weight_untouched_by_fwd_bwd():
+    t, w = layer_on_gpu(256, 320, 96, 16)
+    snap = [x.clone() for x in (w.codes, w.dq_codes, w.dq_scales)]
+    run_fwd_bwd(t, w)
+    assert all(torch.equal(a, b) for a, b in zip(snap, (w.codes, w.dq_codes, w.dq_scales)))
+
+
+def test_bwd_without_saved_V_and_without_dX():
+    """V = NULL recomputes X A inside the backward; dX = NULL skips the dX GEMM."""
+    t, w = layer_on_gpu(256, 384, 120, 16)
+    ws = q.Workspace()
+    Y, V = q.qlora_linear_fwd(w, t["X"], t["A"], t["B"], ws)
+    dX1, dA1, dB1 = q.qlora_linear_bwd(w, t["X"], V, t["dY"], t["A"], t["B"], ws)
+    dX2, dA2, dB2 = q.qlora_linear_bwd(w, t["X"], None, t["dY"], t["A"], t["B"], ws, need_dX=False)
+    torch.cuda.synchronize()
+    assert dX2 is None
+    assert torch.equal(dA1, dA2) and torch.equal(dB1, dB2)
+
+
+def sampled_check(t, w, out, rows):
+    Wq = oracle_weight(w)
+    Yr, Vr = linear.forward_rows(t["X"], t["A"], t["B"], Wq, rows)
+    assert_close(out["Y"][rows], Yr, "Y rows")
+    assert_close(out["V"][rows], Vr, "V rows")
+    assert_close(out["dX"][rows], linear.dX_rows(t["A"], t["B"], Wq, t["dY"], rows), "dX rows")
+    g = linear.adapter_grads(t["X"], t["A"], t["B"], t["dY"])
+    assert_close(out["dA"], g["dA"], "dA")
+    assert_close(out["dB"], g["dB"], "dB")
+
+
+def test_linear_attn4096_m4096_r16_sampled():
+    """Attention projection 4096 x 4096, r = 16, M = 4096: dA, dB in full, Y, V
+    and dX on 96 sampled token rows (first, last and random)."""
+    t, w = layer_on_gpu(4096, 4096, 4096, 16)
+    out = run_fwd_bwd(t, w)
+    rows = sorted(set([0, 4095] + list(np.random.default_rng(0).integers(0, 4096, 94))))
+    sampled_check(t, w, out, rows)
+
+
+@pytest.mark.parametrize("n_in,n_out", [(4096, 11008), (11008, 4096)])
+def test_linear_mlp_m8192_r64_sampled(n_in, n_out):
+    """MLP projections at M = 8192, r = 64 (the launch configuration the
+    benchmark times), sampled rows for Y, V, dX and full dA, dB."""
+    t, w = layer_on_gpu(n_in, n_out, 8192, 64)
+    out = run_fwd_bwd(t, w)
+    rows = sorted(set([0, 8191] + list(np.random.default_rng(1).integers(0, 8192, 62))))
+    sampled_check(t, w, out, rows)
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+@pytest.mark.parametrize("n_in,n_out", [(4096, 4096), (4096, 11008)])
+def test_linear_small_m_forward(M, n_in, n_out):
+    """Small-M forward (token counts 1, 4, 16), every output."""
+    t, w = layer_on_gpu(n_in, n_out, M, 16, tag="gemv")
+    ws = q.Workspace()
+    Y, V = q.qlora_linear_fwd(w, t["X"], t["A"], t["B"], ws)
+    torch.cuda.synchronize()
+    Yr, Vr = linear.forward(t["X"], t["A"], t["B"], oracle_weight(w))
+    assert_close(Y, Yr, "Y")
+    assert_close(V, Vr, "V")
+
+
+def test_linear_stack_layer_sample():
+    """Llama-7B-shaped stack, M = 2048, r = 16: one layer's seven projections
+    (q, k, v, o, gate, up, down), sampled rows for Y, V, dX, full dA, dB."""
+    shapes = [(4096, 4096)] * 4 + [(4096, 11008)] * 2 + [(11008, 4096)]
+    rows = sorted(set([0, 2047] + list(np.random.default_rng(2).integers(0, 2048, 30))))
+    for i, (n_in, n_out) in enumerate(shapes):
+        t, w = layer_on_gpu(n_in, n_out, 2048, 16, tag=f"stack{i}")
+        out = run_fwd_bwd(t, w)
+        sampled_check(t, w, out, rows)

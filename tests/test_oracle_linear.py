@@ -60,6 +60,8 @@ def test_backward_factored_equals_dense_form():
     d = linear.backward_dense(t["X"], t["A"], t["B"], t["dY"])
     assert linear.rel_fro(g["dA"], d["dA"]) < 1e-12
     assert linear.rel_fro(g["dB"], d["dB"]) < 1e-12
+    a = linear.adapter_grads(t["X"], t["A"], t["B"], t["dY"])
+    assert np.array_equal(a["dA"], g["dA"]) and np.array_equal(a["dB"], g["dB"])
 
 
 def test_backward_finite_differences():
