@@ -1,0 +1,524 @@
+#!/usr/bin/env python
+"""Benchmark of the QLoRA adapted linear layer (libqlora, B200).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one forward + backward pass of the adapted linear layer(s) of the
+workload over one batch of M tokens: dequantisation of the frozen NF4 weight
+inside the GEMMs, V = X A, Y, U = dY B^T, dX, dA, dB.  Quantisation and merge
+are one-time operations of the method ("How it works" steps 1 and 5) and are
+timed separately under "rows", with the small-M forward.
+
+Timing: W untimed warm-up steps, then exactly K steps between a barrier +
+synchronize on both sides, CUDA events on the launching stream, max over ranks.
+Inputs rotate over several independent sets whose combined size exceeds the L2
+cache, so every step reads its operands from HBM.  One JSON line on rank 0.
+
+With --gpus N > 1 (launched by torch.distributed.run) every rank runs an
+independent replica on its own GPU (the layer's data-parallel split has no
+exchange in the forward; weak scaling), and the value is all ranks' tokens over
+the slowest rank's time.
+
+--impl reference times the float64 CPU oracle (the reference arm) on a bounded
+sample of the same workload on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOADS = {
+    # Llama-7B attention projection (the headline configuration)
+    "attn4096_m4096_r16": dict(shapes=[(4096, 4096)], M=4096, r=16),
+    # Llama-7B MLP projections, one gate/up and one down per step
+    "mlp4096x11008_m8192_r64": dict(shapes=[(4096, 11008), (11008, 4096)], M=8192, r=64),
+    # the smallest configuration (launch-bound)
+    "linear256_m64_r8": dict(shapes=[(256, 256)], M=64, r=8),
+}
+DEFAULT_WORKLOAD = "attn4096_m4096_r16"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-rows", action="store_true", help="skip the per-kernel row measurements")
+    p.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def flops_fwd_bwd(n_in, n_out, M, r):
+    """Algorithmic flops of one forward + backward: 4 M in out + 6 M r (in + out)."""
+    return 4 * M * n_in * n_out + 6 * M * r * (n_in + n_out)
+
+
+def flops_fwd_gemm(n_in, n_out, M, r):
+    """The fused forward GEMM: X W (2 M in out) plus V B (2 M r out)."""
+    return 2 * M * n_out * (n_in + r)
+
+
+def src_hash(*names):
+    h = hashlib.sha1()
+    for n in names:
+        with open(os.path.join(ROOT, "quantized_rank_fine_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms while running."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_init(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    """Largest value of x over all ranks (identity with one rank)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ our arm
+
+def build_sets(wl, nsets, seed_base):
+    import torch
+    import quantized_rank_fine_b200 as q
+    import synth
+    M, r = wl["M"], wl["r"]
+    sets = []
+    for s in range(nsets):
+        layers = []
+        for li, (n_in, n_out) in enumerate(wl["shapes"]):
+            t = synth.layer_inputs(n_in, n_out, M, r, device="cuda", seed=seed_base + s, tag=f"bench{li}:")
+            w = q.qlora_quantize_nf4(t["W0"])
+            del t["W0"]
+            out = {
+                "Y": torch.empty((M, n_out), dtype=torch.bfloat16, device="cuda"),
+                "V": torch.empty((M, r), dtype=torch.bfloat16, device="cuda"),
+                "dX": torch.empty((M, n_in), dtype=torch.bfloat16, device="cuda"),
+                "dA": torch.empty((n_in, r), dtype=torch.float32, device="cuda"),
+                "dB": torch.empty((r, n_out), dtype=torch.float32, device="cuda"),
+            }
+            layers.append((w, t, out))
+        sets.append(layers)
+    torch.cuda.synchronize()
+    return sets
+
+
+def set_bytes(wl):
+    M, r = wl["M"], wl["r"]
+    tot = 0
+    for n_in, n_out in wl["shapes"]:
+        n = n_in * n_out
+        tot += n // 2 + n // 64 + 2 * M * (n_in + n_out) * 2 + 2 * r * (n_in + n_out) + 4 * r * (n_in + n_out)
+    return tot
+
+
+def run_step(layers, ws):
+    import quantized_rank_fine_b200 as q
+    for w, t, o in layers:
+        q.qlora_linear_fwd(w, t["X"], t["A"], t["B"], ws, Y=o["Y"], V=o["V"])
+        q.qlora_linear_bwd(w, t["X"], o["V"], t["dY"], t["A"], t["B"], ws, dX=o["dX"], dA=o["dA"], dB=o["dB"])
+
+
+def time_rows(wl, pk):
+    """Per-kernel measurements of the other rows of the path (one GPU)."""
+    import torch
+    import quantized_rank_fine_b200 as q
+    import synth
+    rows = {}
+    n_in, n_out = wl["shapes"][0]
+    n = n_in * n_out
+    reps = max(3, math.ceil(3 * L2_BYTES / (4 * n)))
+    W0s = [synth.normal(f"rowsW{i}", (n_in, n_out), 0.02, device="cuda") for i in range(reps)]
+    ws_ = [q.qlora_quantize_nf4(W) for W in W0s]
+    torch.cuda.synchronize()
+
+    def timed(fn, which, iters):
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize()
+        tm = q.KernelTimer(which, iters)
+        for i in range(iters):
+            fn(i)
+        torch.cuda.synchronize()
+        ts = tm.times_ms()
+        tm.disarm()
+        return statistics.median(ts)
+
+    hbm = pk["hbm_gbs"]
+    iters = 30
+    t = timed(lambda i: q.qlora_quantize_nf4(W0s[i % reps], out=ws_[i % reps]), q.KERNEL_QUANTIZE, iters)
+    b = n * (4 + 0.5 + 1 / 64) + 4 * math.ceil(n / 64 / 256)
+    rows["quantize"] = {"ms": t, "gbs": b / t / 1e6, "frac_hbm": b / t / 1e6 / hbm, "bytes_per_weight": 4.516}
+    outs = [torch.empty((n_in, n_out), dtype=torch.bfloat16, device="cuda") for _ in range(reps)]
+    t = timed(lambda i: q.qlora_dequantize(ws_[i % reps], torch.bfloat16, out=outs[i % reps]), q.KERNEL_DEQUANTIZE, iters)
+    b = n * (0.5 + 1 / 64 + 2) + 4 * math.ceil(n / 64 / 256)
+    rows["dequantize_bf16"] = {"ms": t, "gbs": b / t / 1e6, "frac_hbm": b / t / 1e6 / hbm}
+    r = wl["r"]
+    A = synth.normal("rowsA", (n_in, r), 1 / math.sqrt(n_in), torch.bfloat16, "cuda")
+    B = synth.normal("rowsB", (r, n_out), 0.01, torch.bfloat16, "cuda")
+    outs32 = [torch.empty((n_in, n_out), dtype=torch.float32, device="cuda") for _ in range(reps)]
+    t = timed(lambda i: q.qlora_merge(ws_[i % reps], A, B, torch.float32, out=outs32[i % reps]), q.KERNEL_MERGE, iters)
+    b = n * (0.5 + 1 / 64 + 4) + 2 * r * (n_in + n_out)
+    rows["merge_f32"] = {"ms": t, "gbs": b / t / 1e6, "frac_hbm": b / t / 1e6 / hbm}
+    del outs, outs32, W0s
+    torch.cuda.synchronize()
+    return rows
+
+
+def arm_ours(args, world, rank, local):
+    import torch
+    import quantized_rank_fine_b200 as q
+
+    wl = WORKLOADS[args.workload]
+    pk, pk_src = peaks()
+    M, r = wl["M"], wl["r"]
+    nsets = max(2, math.ceil(3 * L2_BYTES / set_bytes(wl)))
+    sets = build_sets(wl, nsets, seed_base=100 * rank)
+    ws = q.Workspace()
+    nl = len(wl["shapes"])
+
+    for i in range(args.warmup):
+        run_step(sets[i % nsets], ws)
+    torch.cuda.synchronize()
+    if ws.status() != 0:
+        raise RuntimeError("a kernel wait timed out during warm-up")
+
+    timer = q.KernelTimer(q.KERNEL_FWD_GEMM, args.steps * nl)
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    smi_id = vis.split(",")[local] if vis and len(vis.split(",")) > local else str(local)
+    clocks = ClockSampler(smi_id)
+    launches0 = q.qlora_launch_count()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    ev0.record(stream)
+    for i in range(args.steps):
+        run_step(sets[i % nsets], ws)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    launches = q.qlora_launch_count() - launches0
+    ms_local = ev0.elapsed_time(ev1)
+    gemm_ms = timer.times_ms()
+    timer.disarm()
+    if ws.status() != 0:
+        raise RuntimeError("a kernel wait timed out in the timed region")
+    ms = max_over_ranks(ms_local, world)
+
+    tokens = M * args.steps * world
+    value = tokens / (ms / 1e3)
+    step_flops = sum(flops_fwd_bwd(a, b, M, r) for a, b in wl["shapes"])
+    gemm_flops = [flops_fwd_gemm(a, b, M, r) for a, b in wl["shapes"]] * args.steps
+    achieved = sum(gemm_flops) / (sum(gemm_ms) / 1e3) / 1e12
+    timed_s = ms / 1e3
+    peak = pk["bf16_tflops"] if timed_s < 2.0 else pk["bf16_tflops_sustained"]
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tp):
+        with open(tp) as f:
+            tr = json.load(f)
+        e = tr.get(args.workload, {}).get("fwd_gemm")
+        if e and e.get("src") == src_hash("gemm.cu"):
+            traffic = e["bytes_per_launch"]
+
+    line = {
+        "metric": "QLoRA linear fwd+bwd tokens/s",
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; W0 ~ N(0,0.02) fp32 quantised on device, X/dY ~ N(0,1) bf16)",
+        "config": {"workload": args.workload, "M": M, "shapes": wl["shapes"], "r": r,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": f"{nsets} rotating input sets of {set_bytes(wl) / 2**20:.0f} MiB each (> L2 per cycle)"},
+        "tflops": step_flops * args.steps * world / (ms / 1e3) / 1e12,
+        "roofline": {"kernel": "nf4_gemm_kernel<fwd> (fused dequant GEMM, tcgen05)", "bound": "tensor",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{pk_src} {'burst' if timed_s < 2.0 else 'sustained'} bf16",
+                     "flops_per_launch": gemm_flops[0] if nl == 1 else gemm_flops[:nl],
+                     "mean_launch_ms": statistics.mean(gemm_ms), "traffic": traffic},
+        "gpu_launches": launches,
+        "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"],
+                   "samples": clk["samples"]},
+    }
+
+    # end to end through the public API with host buffers
+    line["e2e"] = e2e(args, sets, ws, wl, world)
+
+    if world == 1 and not args.no_rows:
+        line["rows"] = time_rows(wl, pk)
+    if world == 1 and rank == 0 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(args.workload, budget_s=20.0)
+    return line
+
+
+def e2e(args, sets, ws, wl, world):
+    """Same metric, each step copying X and dY from pinned host memory and the
+    adapter gradients dA, dB back to pinned host memory, on one stream."""
+    import torch
+    M = wl["M"]
+    nsets = len(sets)
+    host = []
+    for layers in sets:
+        hl = []
+        for w, t, o in layers:
+            hl.append({"X": t["X"].cpu().pin_memory(), "dY": t["dY"].cpu().pin_memory(),
+                       "dA": torch.empty(o["dA"].shape, dtype=torch.float32).pin_memory(),
+                       "dB": torch.empty(o["dB"].shape, dtype=torch.float32).pin_memory()})
+        host.append(hl)
+    h2d = sum(h["X"].numel() * 2 + h["dY"].numel() * 2 for h in host[0])
+    d2h = sum(h["dA"].numel() * 4 + h["dB"].numel() * 4 for h in host[0])
+    steps = max(10, args.steps // 4)
+
+    def step(i):
+        layers, hl = sets[i % nsets], host[i % nsets]
+        for (w, t, o), h in zip(layers, hl):
+            t["X"].copy_(h["X"], non_blocking=True)
+            t["dY"].copy_(h["dY"], non_blocking=True)
+        run_step(layers, ws)
+        for (w, t, o), h in zip(layers, hl):
+            h["dA"].copy_(o["dA"], non_blocking=True)
+            h["dB"].copy_(o["dB"], non_blocking=True)
+
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(s)
+    for i in range(steps):
+        step(i)
+    e1.record(s)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    return {"value": M * steps * world / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+# ------------------------------------------------------------------ the oracle (CPU baseline / reference arm)
+
+def oracle_cores():
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count() or 1
+    try:
+        from threadpoolctl import threadpool_info, threadpool_limits
+        threadpool_limits(n)
+        used = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        used = n
+    return n, used
+
+
+def oracle_inputs(workload, rows_frac, tokens):
+    """Oracle inputs of a bounded sample: the first rows_frac of each weight's
+    input rows (whole double-quant groups) and `tokens` tokens, quantised by the
+    oracle itself."""
+    import synth
+    from oracle import nf4
+    wl = WORKLOADS[workload]
+    r = wl["r"]
+    layers = []
+    for li, (n_in, n_out) in enumerate(wl["shapes"]):
+        rows_per_group = max(1, (64 * 256) // n_out)
+        n_rows = max(rows_per_group, int(n_in * rows_frac) // rows_per_group * rows_per_group)
+        t = synth.layer_inputs(n_rows, n_out, tokens, r, tag=f"oracle{li}:")
+        codes, dqc, dqs = nf4.quantize_nf4(t["W0"].numpy())
+        layers.append((t, (codes, dqc, dqs), n_rows, n_out, n_in))
+    return layers
+
+
+def oracle_step(layers):
+    """One oracle forward + backward over the sample (dequantisation included)."""
+    from oracle import linear, nf4
+    for t, (codes, dqc, dqs), n_rows, n_out, _ in layers:
+        Wq = nf4.dequantize_bf16(codes, dqc, dqs, n_rows, n_out)
+        linear.forward(t["X"], t["A"], t["B"], Wq)
+        linear.backward(t["X"], t["A"], t["B"], Wq, t["dY"])
+
+
+def oracle_sample_time(workload, budget_s):
+    """Pick a sample that costs about budget_s per step; returns (layers, seconds
+    per step, fraction of the full step's work)."""
+    wl = WORKLOADS[workload]
+    M = wl["M"]
+    tokens = min(M, 256)
+    frac = 1.0 / 16
+    while True:
+        layers = oracle_inputs(workload, frac, tokens)
+        t0 = time.perf_counter()
+        oracle_step(layers)
+        dt = time.perf_counter() - t0
+        if dt * 2 > budget_s or frac >= 1.0:
+            break
+        frac = min(1.0, frac * 2)
+    row_frac = sum(l[2] for l in layers) / sum(l[4] for l in layers)
+    return layers, dt, row_frac, tokens
+
+
+def cpu_baseline(workload, budget_s=20.0):
+    cores, used = oracle_cores()
+    layers, dt, row_frac, tokens = oracle_sample_time(workload, budget_s / 4)
+    reps = max(1, int(budget_s / max(dt, 1e-3) / 2))
+    ts = []
+    for _ in range(min(reps, 5)):
+        t0 = time.perf_counter()
+        oracle_step(layers)
+        ts.append(time.perf_counter() - t0)
+    dt = statistics.median(ts)
+    value = tokens * row_frac / dt   # tokens/s of the full layer (work scales with the weight rows)
+    return {"value": value, "unit": "tokens/s", "cores": used, "kind": "oracle",
+            "sample": f"float64 oracle fwd+bwd incl. dequantisation, {tokens} tokens x {row_frac:.4f} of each "
+                      f"weight's input rows, median of {len(ts)} runs, scaled to the full layer"}
+
+
+def arm_reference(args, world, rank):
+    """The reference arm: the float64 oracle on the host cores, K timed steps."""
+    if rank != 0:
+        return None
+    wl = WORKLOADS[args.workload]
+    budget = max(0.05, 150.0 / max(1, args.steps + args.warmup))
+    layers, _, row_frac, tokens = oracle_sample_time(args.workload, budget)
+    for _ in range(args.warmup):
+        oracle_step(layers)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(layers)
+    dt = time.perf_counter() - t0
+    cores, used = oracle_cores()
+    value = tokens * row_frac * args.steps / dt
+    sample = (f"float64 oracle fwd+bwd incl. dequantisation, per step {tokens} tokens x {row_frac:.4f} of each "
+              f"weight's input rows, scaled to the full layer")
+    return {
+        "impl": "reference", "metric": "QLoRA linear fwd+bwd tokens/s", "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "M": wl["M"], "shapes": wl["shapes"], "r": wl["r"]},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": used, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_init(args)
+    if args.impl == "reference":
+        line = arm_reference(args, world, rank)
+    else:
+        line = arm_ours(args, world, rank, local)
+    if rank == 0 and line is not None:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

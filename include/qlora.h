@@ -187,6 +187,28 @@ QLORA_API void qlora_nf4_codebook(float out[16]);
 /* Adapter parameters of one layer: r (in + out) ("How it works", adapter size). */
 QLORA_API int64_t qlora_adapter_params(int64_t in, int64_t out, int r);
 
+/* ---------------------------------------------------------------- measurement */
+
+/* Kernels that qlora_time_kernel() can bracket with events. */
+typedef enum qlora_kernel {
+  QLORA_KERNEL_QUANTIZE = 1,   /* NF4 + double-quant encoder (qlora_quantize_nf4) */
+  QLORA_KERNEL_DEQUANTIZE = 2, /* dense dequantisation (qlora_dequantize) */
+  QLORA_KERNEL_MERGE = 3,      /* adapter merge (qlora_merge) */
+  QLORA_KERNEL_FWD_GEMM = 4,   /* fused dequant GEMM of the forward */
+  QLORA_KERNEL_DX_GEMM = 5,    /* fused dequant GEMM of dX */
+  QLORA_KERNEL_RANK_R = 6      /* the rank-r kernels: V, U, dA, dB (and their split sums) */
+} qlora_kernel;
+
+/* Arm launch timing for benchmarks: the next n launches of kernel `which` are
+ * each bracketed by cudaEventRecord(starts[i]) / cudaEventRecord(stops[i]) on the
+ * launching stream (starts/stops: [host] arrays of cudaEvent_t owned by the
+ * caller).  n = 0 disarms.  Process-wide state; not for concurrent callers.
+ * Returns QLORA_ERR_INVALID_ARG for an unknown kernel or NULL arrays with n > 0. */
+QLORA_API qlora_status qlora_time_kernel(int which, void* const* starts, void* const* stops, int n);
+
+/* Number of kernel launches libqlora has issued in this process. */
+QLORA_API uint64_t qlora_launch_count(void);
+
 /* Human-readable name of a status code (static string). */
 QLORA_API const char* qlora_status_string(qlora_status s);
 

@@ -34,8 +34,11 @@ STATUS_NAMES = {
 EXPORTS = (
     "qlora_quantize_nf4", "qlora_dequantize", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_merge",
     "qlora_workspace_bytes", "qlora_ws_init", "qlora_ws_status", "qlora_nf4_codebook",
-    "qlora_adapter_params", "qlora_status_string",
+    "qlora_adapter_params", "qlora_status_string", "qlora_time_kernel", "qlora_launch_count",
 )
+
+# Kernel ids of qlora_time_kernel.
+KERNEL_QUANTIZE, KERNEL_DEQUANTIZE, KERNEL_MERGE, KERNEL_FWD_GEMM, KERNEL_DX_GEMM, KERNEL_RANK_R = 1, 2, 3, 4, 5, 6
 
 
 class QLoRAError(RuntimeError):
@@ -73,6 +76,8 @@ def lib() -> ctypes.CDLL:
             "qlora_nf4_codebook": (None, [ctypes.POINTER(ctypes.c_float)]),
             "qlora_adapter_params": (i64, [i64, i64, i32]),
             "qlora_status_string": (ctypes.c_char_p, [i32]),
+            "qlora_time_kernel": (i32, [i32, ctypes.POINTER(vp), ctypes.POINTER(vp), i32]),
+            "qlora_launch_count": (ctypes.c_uint64, []),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -127,6 +132,32 @@ def qlora_adapter_params(n_in: int, n_out: int, r: int) -> int:
 
 def qlora_status_string(status: int) -> str:
     return lib().qlora_status_string(status).decode()
+
+
+def qlora_launch_count() -> int:
+    return lib().qlora_launch_count()
+
+
+class KernelTimer:
+    """Bracket the next n launches of one kernel kind with CUDA events recorded
+    by the library on the launching stream (qlora_time_kernel)."""
+
+    def __init__(self, which: int, n: int):
+        self.starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        self.stops = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in self.starts + self.stops:
+            e.record()          # materialise the cudaEvent_t handles
+        self._s = (ctypes.c_void_p * n)(*[e.cuda_event for e in self.starts])
+        self._e = (ctypes.c_void_p * n)(*[e.cuda_event for e in self.stops])
+        _check(lib().qlora_time_kernel(which, self._s, self._e, n), "qlora_time_kernel")
+        self.n = n
+
+    def disarm(self):
+        lib().qlora_time_kernel(KERNEL_QUANTIZE, None, None, 0)
+
+    def times_ms(self, count: int | None = None) -> list:
+        count = self.n if count is None else count
+        return [self.starts[i].elapsed_time(self.stops[i]) for i in range(count)]
 
 
 def qlora_workspace_bytes(op: int, M: int, n_in: int, n_out: int, r: int) -> int:

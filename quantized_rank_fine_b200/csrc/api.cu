@@ -3,6 +3,8 @@
 #include <cuda_runtime.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "../../include/qlora.h"
 #include "common.cuh"
 #include "kernels.h"
@@ -111,9 +113,45 @@ WsLayout ws_layout(int op, int64_t M, int64_t in, int64_t out, int r) {
   return L;
 }
 
+std::atomic<uint64_t> g_launches{0};
+
+struct TimingHook {
+  int which = 0;
+  void* const* starts = nullptr;
+  void* const* stops = nullptr;
+  int n = 0, i = 0;
+} g_hook;
+
 }  // namespace
 
+namespace qlora {
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+void timing_before(int which, cudaStream_t stream) {
+  if (g_hook.which == which && g_hook.i < g_hook.n)
+    cudaEventRecord(static_cast<cudaEvent_t>(g_hook.starts[g_hook.i]), stream);
+}
+void timing_after(int which, cudaStream_t stream) {
+  if (g_hook.which == which && g_hook.i < g_hook.n) {
+    cudaEventRecord(static_cast<cudaEvent_t>(g_hook.stops[g_hook.i]), stream);
+    ++g_hook.i;
+  }
+}
+}  // namespace qlora
+
 extern "C" {
+
+qlora_status qlora_time_kernel(int which, void* const* starts, void* const* stops, int n) {
+  if (n < 0 || which < QLORA_KERNEL_QUANTIZE || which > QLORA_KERNEL_RANK_R) return QLORA_ERR_INVALID_ARG;
+  if (n > 0 && (!starts || !stops)) return QLORA_ERR_INVALID_ARG;
+  g_hook.which = n > 0 ? which : 0;
+  g_hook.starts = starts;
+  g_hook.stops = stops;
+  g_hook.n = n;
+  g_hook.i = 0;
+  return QLORA_OK;
+}
+
+uint64_t qlora_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 const char* qlora_status_string(qlora_status s) {
   switch (s) {

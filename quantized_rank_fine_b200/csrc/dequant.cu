@@ -145,10 +145,13 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* dq_codes,
   const int64_t n16 = n / 16;
   if (n16 == 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>((n16 + kDqThreads - 1) / kDqThreads);
+  timing_before(QLORA_KERNEL_DEQUANTIZE, stream);
   if (bf16)
     dequantize_kernel<true><<<grid, kDqThreads, 0, stream>>>(codes, dq_codes, dq_scales, n16, out);
   else
     dequantize_kernel<false><<<grid, kDqThreads, 0, stream>>>(codes, dq_codes, dq_scales, n16, out);
+  timing_after(QLORA_KERNEL_DEQUANTIZE, stream);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -159,10 +162,13 @@ cudaError_t launch_merge(const uint8_t* codes, const uint8_t* dq_codes, const fl
             static_cast<unsigned>((n_in + kMgRows - 1) / kMgRows));
   const auto* a = reinterpret_cast<const __nv_bfloat16*>(A);
   const auto* b = reinterpret_cast<const __nv_bfloat16*>(B);
+  timing_before(QLORA_KERNEL_MERGE, stream);
   if (bf16)
     merge_kernel<true><<<grid, 256, 0, stream>>>(codes, dq_codes, dq_scales, a, b, r, n_in, n_out, out);
   else
     merge_kernel<false><<<grid, 256, 0, stream>>>(codes, dq_codes, dq_scales, a, b, r, n_in, n_out, out);
+  timing_after(QLORA_KERNEL_MERGE, stream);
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -331,7 +331,11 @@ cudaError_t launch_gemm(const CUtensorMap& act, const CUtensorMap& ea, const CUt
     attr_set[dev] = true;
   }
   dim3 grid(static_cast<unsigned>((a.N + kBN - 1) / kBN), static_cast<unsigned>((a.M + kBM - 1) / kBM));
+  const int which = kDX ? QLORA_KERNEL_DX_GEMM : QLORA_KERNEL_FWD_GEMM;
+  timing_before(which, stream);
   nf4_gemm_kernel<kDX><<<grid, kThreads, kSmemBytes, stream>>>(act, ea, eb, a);
+  timing_after(which, stream);
+  count_launch();
   return cudaGetLastError();
 }
 

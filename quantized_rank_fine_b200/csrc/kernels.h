@@ -12,6 +12,12 @@ namespace qlora {
 
 constexpr int kMaxSplits = 16;   // most K/M splits of the rank-r kernels
 
+// Bookkeeping of the measurement helpers (defined in api.cu): every kernel
+// launch is counted; an armed timing hook brackets launches of one kernel kind.
+void count_launch();
+void timing_before(int which, cudaStream_t stream);
+void timing_after(int which, cudaStream_t stream);
+
 struct WeightView {
   const uint8_t* codes;
   const uint8_t* dq_codes;

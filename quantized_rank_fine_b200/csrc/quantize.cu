@@ -158,8 +158,11 @@ cudaError_t launch_quantize_nf4(const float* W0, int64_t n, uint8_t* codes, uint
   const int64_t nblocks = n / kBlock;
   const int64_t ngroups = (nblocks + kGroup - 1) / kGroup;
   if (ngroups == 0) return cudaSuccess;
+  timing_before(QLORA_KERNEL_QUANTIZE, stream);
   quantize_nf4_kernel<<<static_cast<unsigned>(ngroups), kQThreads, 0, stream>>>(
       W0, nblocks, codes, dq_codes, dq_scales);
+  timing_after(QLORA_KERNEL_QUANTIZE, stream);
+  count_launch();
   return cudaGetLastError();
 }
 

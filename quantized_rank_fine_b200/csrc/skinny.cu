@@ -238,16 +238,22 @@ cudaError_t run_skinny(bool a_trans, bool b_trans, const Operand& a, const Opera
   kps = (kps + kTile - 1) / kTile * kTile;
   SkinnyArgs p{a, b, 0, kps, k_total, out_rows, r, part, out, out_kind, splits};
   dim3 grid(static_cast<unsigned>(mt), splits, rt);
+  timing_before(QLORA_KERNEL_RANK_R, stream);
   if (!a_trans && b_trans) skinny_mma_kernel<false, true><<<grid, kSkThreads, 0, stream>>>(p);
   else if (!a_trans && !b_trans) skinny_mma_kernel<false, false><<<grid, kSkThreads, 0, stream>>>(p);
   else if (a_trans && b_trans) skinny_mma_kernel<true, true><<<grid, kSkThreads, 0, stream>>>(p);
   else skinny_mma_kernel<true, false><<<grid, kSkThreads, 0, stream>>>(p);
+  count_launch();
   cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess || splits == 1) return e;
-  const int64_t n = out_rows * r;
-  const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, 4 * 148));
-  reduce_splits_kernel<<<blocks, 256, 0, stream>>>(part, splits, out_rows, r, out, out_kind);
-  return cudaGetLastError();
+  if (e == cudaSuccess && splits > 1) {
+    const int64_t n = out_rows * r;
+    const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, 4 * 148));
+    reduce_splits_kernel<<<blocks, 256, 0, stream>>>(part, splits, out_rows, r, out, out_kind);
+    count_launch();
+    e = cudaGetLastError();
+  }
+  timing_after(QLORA_KERNEL_RANK_R, stream);
+  return e;
 }
 
 }  // namespace
