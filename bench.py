@@ -255,9 +255,58 @@ def time_rows(wl, pk):
     t = timed(lambda i: q.qlora_merge(ws_[i % reps], A, B, torch.float32, out=outs32[i % reps]), q.KERNEL_MERGE, iters)
     b = n * (0.5 + 1 / 64 + 4) + 2 * r * (n_in + n_out)
     rows["merge_f32"] = {"ms": t, "gbs": b / t / 1e6, "frac_hbm": b / t / 1e6 / hbm}
-    del outs, outs32, W0s
+    del outs, outs32, W0s, ws_
     torch.cuda.synchronize()
+    rows["gemv"] = time_gemv(pk)
     return rows
+
+
+def time_gemv(pk):
+    """Small-M forward (M = 1, 4, 16) on the 4096 x 4096 and 4096 x 11008 shapes,
+    r = 16: the dequant-GEMV kernel's HBM bandwidth.  Algorithmic bytes: codes,
+    absmax codes and scales, A and B, X, V and Y."""
+    import torch
+    import quantized_rank_fine_b200 as q
+    import synth
+    out = {}
+    r = 16
+    for n_in, n_out in ((4096, 4096), (4096, 11008)):
+        wbytes = n_in * n_out * (0.5 + 1 / 64)
+        reps = max(3, math.ceil(3 * L2_BYTES / wbytes))
+        wts = [q.qlora_quantize_nf4(synth.normal(f"gemvW{i}", (n_in, n_out), 0.02, device="cuda")) for i in range(reps)]
+        A = synth.normal("gemvA", (n_in, r), 1 / math.sqrt(n_in), torch.bfloat16, "cuda")
+        B = synth.normal("gemvB", (r, n_out), 0.01, torch.bfloat16, "cuda")
+        for M in (1, 4, 16):
+            X = synth.normal(f"gemvX{M}", (M, n_in), 1.0, torch.bfloat16, "cuda")
+            Y = torch.empty((M, n_out), dtype=torch.bfloat16, device="cuda")
+            V = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+            ws = q.Workspace()
+            for i in range(3):
+                q.qlora_linear_fwd(wts[i % reps], X, A, B, ws, Y=Y, V=V)
+            torch.cuda.synchronize()
+            # the calls (V = X A, then the GEMV) captured in one CUDA graph so the
+            # device never waits for the host between launches
+            iters = 60
+            tm = q.KernelTimer(q.KERNEL_GEMV, iters)
+            graph = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                with torch.cuda.graph(graph, stream=side, capture_error_mode="relaxed"):
+                    for i in range(iters):
+                        q.qlora_linear_fwd(wts[i % reps], X, A, B, ws, Y=Y, V=V)
+            torch.cuda.current_stream().wait_stream(side)
+            tm.disarm()
+            graph.replay()
+            torch.cuda.synchronize()
+            t = statistics.median(tm.times_ms())
+            del graph
+            b = n_in * n_out * (0.5 + 1 / 64) + 4 * math.ceil(n_in * n_out / 16384) + 2 * r * (n_in + n_out) \
+                + 2 * M * (n_in + n_out) + 2 * M * r
+            out[f"{n_in}x{n_out}_m{M}"] = {"us": t * 1e3, "gbs": b / t / 1e6, "frac_hbm": b / t / 1e6 / pk["hbm_gbs"]}
+        del wts
+        torch.cuda.synchronize()
+    return out
 
 
 def arm_ours(args, world, rank, local):

@@ -125,6 +125,8 @@ QLORA_API qlora_status qlora_dequantize(const qlora_nf4_weight* w, void* W_out, 
  * Forward of the adapted layer ("How it works" steps 2-3; "LoRA & QLoRA"
  * Mathematical Formulation h = W0 x + B(A x)):
  *   V = bf16(X A)  (fp32 accumulation),   Y = bf16(X bf16(w') + V B)  (fp32 accumulation).
+ * For M <= 16 a dequant-GEMV computes the base term as sum_k bf16(x_k a'_k) bf16(l_k)
+ * (the block absmax folded into the activation; the same sum in exact arithmetic).
  *   w      [host] descriptor of [device] tensors.
  *   X      [device] bf16 (M, in).
  *   A      [device] bf16 (in, r).          B [device] bf16 (r, out).
@@ -173,7 +175,9 @@ QLORA_API qlora_status qlora_merge(const qlora_nf4_weight* w, const uint16_t* A,
  * (0 for an unknown op or invalid sizes).  Host only, no device access. */
 QLORA_API size_t qlora_workspace_bytes(int op, int64_t M, int64_t in, int64_t out, int r);
 
-/* Zero the workspace's status words (once, before the workspace's first use). */
+/* Zero the whole workspace (once, before its first use).  The calls keep the
+ * workspace's bookkeeping words at zero between calls; calls that share one
+ * workspace must be ordered on one stream. */
 QLORA_API qlora_status qlora_ws_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronise `stream`, then report QLORA_ERR_TIMEOUT if a bounded wait in a
@@ -196,13 +200,15 @@ typedef enum qlora_kernel {
   QLORA_KERNEL_MERGE = 3,      /* adapter merge (qlora_merge) */
   QLORA_KERNEL_FWD_GEMM = 4,   /* fused dequant GEMM of the forward */
   QLORA_KERNEL_DX_GEMM = 5,    /* fused dequant GEMM of dX */
-  QLORA_KERNEL_RANK_R = 6      /* the rank-r kernels: V, U, dA, dB (and their split sums) */
+  QLORA_KERNEL_RANK_R = 6,     /* the rank-r kernels: V, U, dA, dB (and their split sums) */
+  QLORA_KERNEL_GEMV = 7        /* small-M forward (M <= 16) */
 } qlora_kernel;
 
 /* Arm launch timing for benchmarks: the next n launches of kernel `which` are
  * each bracketed by cudaEventRecord(starts[i]) / cudaEventRecord(stops[i]) on the
  * launching stream (starts/stops: [host] arrays of cudaEvent_t owned by the
- * caller).  n = 0 disarms.  Process-wide state; not for concurrent callers.
+ * caller), as external event records so that they also time launches captured
+ * in a CUDA graph.  n = 0 disarms.  Process-wide state; not for concurrent callers.
  * Returns QLORA_ERR_INVALID_ARG for an unknown kernel or NULL arrays with n > 0. */
 QLORA_API qlora_status qlora_time_kernel(int which, void* const* starts, void* const* stops, int n);
 

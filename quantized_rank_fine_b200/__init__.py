@@ -39,6 +39,7 @@ EXPORTS = (
 
 # Kernel ids of qlora_time_kernel.
 KERNEL_QUANTIZE, KERNEL_DEQUANTIZE, KERNEL_MERGE, KERNEL_FWD_GEMM, KERNEL_DX_GEMM, KERNEL_RANK_R = 1, 2, 3, 4, 5, 6
+KERNEL_GEMV = 7
 
 
 class QLoRAError(RuntimeError):

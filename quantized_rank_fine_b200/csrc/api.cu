@@ -88,19 +88,30 @@ WeightView view(const qlora_nf4_weight* w) { return WeightView{w->codes, w->dq_c
 
 // Workspace layout (byte offsets), shared by the size query and the calls.
 struct WsLayout {
-  size_t v_off, u_off, part_off, total;
+  size_t v_off, u_off, part_off, gemv_off, total;
 };
+
+constexpr int64_t kGemvMaxM = 16;     // token counts served by the dequant-GEMV
+constexpr int64_t kTicketWords = 4096;  // split-K tickets of the GEMV: one per 64-column panel
+// Every layout reserves the tickets right after the status words, so no call
+// ever writes that region except the GEMV, which leaves it zero.
+constexpr size_t kTicketOff = 256;
+constexpr size_t kFixedBytes = kTicketOff + kTicketWords * 4;
 
 WsLayout ws_layout(int op, int64_t M, int64_t in, int64_t out, int r) {
   WsLayout L{};
   const size_t mr = align256(static_cast<size_t>(M) * r * 2);
-  size_t off = kStatusBytes;
+  size_t off = kFixedBytes;
   L.v_off = off;
   off += mr;
   size_t parts = 0;
   if (op == QLORA_OP_FWD) {
     L.u_off = 0;
     parts = qlora::skinny_partial_floats(M, r, in);
+    if (M <= kGemvMaxM && out / 64 <= kTicketWords) {
+      L.gemv_off = off;
+      off += align256(qlora::gemv_workspace_bytes(M, in, out));
+    }
   } else {
     L.u_off = off;
     off += mr;
@@ -126,13 +137,21 @@ struct TimingHook {
 
 namespace qlora {
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+// Record `e` on `stream`; inside a stream capture as an external event node, so
+// that it is recorded at every replay of the graph.
+static void record_event(void* e, cudaStream_t stream) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(static_cast<cudaEvent_t>(e), stream, cudaEventRecordExternal);
+  else
+    cudaEventRecord(static_cast<cudaEvent_t>(e), stream);
+}
 void timing_before(int which, cudaStream_t stream) {
-  if (g_hook.which == which && g_hook.i < g_hook.n)
-    cudaEventRecord(static_cast<cudaEvent_t>(g_hook.starts[g_hook.i]), stream);
+  if (g_hook.which == which && g_hook.i < g_hook.n) record_event(g_hook.starts[g_hook.i], stream);
 }
 void timing_after(int which, cudaStream_t stream) {
   if (g_hook.which == which && g_hook.i < g_hook.n) {
-    cudaEventRecord(static_cast<cudaEvent_t>(g_hook.stops[g_hook.i]), stream);
+    record_event(g_hook.stops[g_hook.i], stream);
     ++g_hook.i;
   }
 }
@@ -141,7 +160,7 @@ void timing_after(int which, cudaStream_t stream) {
 extern "C" {
 
 qlora_status qlora_time_kernel(int which, void* const* starts, void* const* stops, int n) {
-  if (n < 0 || which < QLORA_KERNEL_QUANTIZE || which > QLORA_KERNEL_RANK_R) return QLORA_ERR_INVALID_ARG;
+  if (n < 0 || which < QLORA_KERNEL_QUANTIZE || which > QLORA_KERNEL_GEMV) return QLORA_ERR_INVALID_ARG;
   if (n > 0 && (!starts || !stops)) return QLORA_ERR_INVALID_ARG;
   g_hook.which = n > 0 ? which : 0;
   g_hook.starts = starts;
@@ -183,7 +202,7 @@ qlora_status qlora_ws_init(void* ws, size_t ws_bytes, void* stream) {
   if (!ws || ws_bytes < kStatusBytes) return QLORA_ERR_WORKSPACE;
   QLORA_TRY(check_device());
   QLORA_TRY(check_ptr(ws));
-  QLORA_CUDA(cudaMemsetAsync(ws, 0, kStatusBytes, static_cast<cudaStream_t>(stream)));
+  QLORA_CUDA(cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)));
   return QLORA_OK;
 }
 
@@ -264,8 +283,14 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int6
   uint16_t* V = V_save ? V_save : reinterpret_cast<uint16_t*>(base + L.v_off);
   float* part = reinterpret_cast<float*>(base + L.part_off);
   const WeightView wv = view(w);
-  QLORA_CUDA(qlora::launch_xa(X, A, M, w->in, r, V, part, s));
-  QLORA_CUDA(qlora::launch_fwd_gemm(wv, X, V, B, M, r, Y, status, s));
+  uint32_t* tickets = reinterpret_cast<uint32_t*>(base + kTicketOff);
+  QLORA_CUDA(qlora::launch_xa(X, A, M, w->in, r, V, part, tickets, status, s));
+  if (M <= kGemvMaxM && w->out / 64 <= kTicketWords) {
+    float* gpart = reinterpret_cast<float*>(base + L.gemv_off);
+    QLORA_CUDA(qlora::launch_gemv(wv, X, V, B, M, r, Y, gpart, tickets, s));
+  } else {
+    QLORA_CUDA(qlora::launch_fwd_gemm(wv, X, V, B, M, r, Y, status, s));
+  }
   return QLORA_OK;
 }
 
@@ -295,14 +320,15 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16_t* X, cons
   uint16_t* U = reinterpret_cast<uint16_t*>(base + L.u_off);
   float* part = reinterpret_cast<float*>(base + L.part_off);
   const WeightView wv = view(w);
+  uint32_t* tickets = reinterpret_cast<uint32_t*>(base + kTicketOff);
   if (!V) {
     uint16_t* Vw = reinterpret_cast<uint16_t*>(base + L.v_off);
-    QLORA_CUDA(qlora::launch_xa(X, A, M, w->in, r, Vw, part, s));
+    QLORA_CUDA(qlora::launch_xa(X, A, M, w->in, r, Vw, part, tickets, status, s));
     V = Vw;
   }
-  QLORA_CUDA(qlora::launch_dybt(dY, B, M, w->out, r, U, part, s));
-  QLORA_CUDA(qlora::launch_vtdy(V, dY, M, w->out, r, dB, part, s));
-  QLORA_CUDA(qlora::launch_xtu(X, U, M, w->in, r, dA, part, s));
+  QLORA_CUDA(qlora::launch_dybt(dY, B, M, w->out, r, U, part, tickets, status, s));
+  QLORA_CUDA(qlora::launch_vtdy(V, dY, M, w->out, r, dB, part, tickets, status, s));
+  QLORA_CUDA(qlora::launch_xtu(X, U, M, w->in, r, dA, part, tickets, status, s));
   if (dX) QLORA_CUDA(qlora::launch_dx_gemm(wv, dY, U, A, M, r, dX, status, s));
   return QLORA_OK;
 }

@@ -12,13 +12,16 @@
 // SM.  Two UMMA M=128 x N=256 accumulators fill the 512 TMEM columns; both use
 // the same dequantised weight tile, so each weight is dequantised M/256 times.
 // Warp roles (320 threads):
-//   warp 0     TMA producer: activation tile (256 x 64 bf16, 128B swizzle) and,
-//              for the adapter K-steps, the V/U tile and the B/A tile.
+//   warp 0     TMA producer: per K-step the activation tile (256 x 64 bf16,
+//              128B swizzle) and the packed codes of the weight tile (8 KB); for
+//              the adapter K-steps the V/U tile and the B/A tile instead.
 //   warp 1     TMEM allocation + the single thread that issues tcgen05.mma.
 //   warps 2-9  dequant producers (one thread per 64-weight block per K-step):
-//              raw codes from global memory -> per-block 16-entry bf16 table ->
+//              codes from shared memory -> per-block 16-entry bf16 table ->
 //              byte-permute lookup -> 16-byte stores in the UMMA canonical
 //              layout; then the epilogue (TMEM -> registers -> bf16 -> global).
+// Barriers per stage: `loaded` (TMA bytes), `ready` (8 dequant warps, after the
+// weight tile is written) and `free` (tcgen05.commit once the MMAs have read it).
 // The weight tile is written MN-major for the forward (N contiguous in W) and
 // K-major for dX (K contiguous in W), so the dequant never transposes.
 #include "common.cuh"
@@ -38,7 +41,8 @@ constexpr int kThreads = 320;
 constexpr int kDeqWarps = 8;
 constexpr uint32_t kABytes = kBM * kBK * 2;     // 32 KB
 constexpr uint32_t kBBytes = kBN * kBK * 2;     // 32 KB
-constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr uint32_t kCBytes = kBN * kBK / 2;     // 8 KB of packed codes
+constexpr uint32_t kStageBytes = kABytes + kBBytes + kCBytes;
 constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 + 256;
 constexpr uint32_t kTmemCols = 512;
 
@@ -93,13 +97,14 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 template <bool kDX>
 __global__ void __launch_bounds__(kThreads, 1)
 nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_ext_a,
-                const __grid_constant__ CUtensorMap tm_ext_b, const GemmArgs p) {
+                const __grid_constant__ CUtensorMap tm_ext_b, const __grid_constant__ CUtensorMap tm_codes,
+                const GemmArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 1);
-  const uint32_t full0 = smem_addr(bars), empty0 = smem_addr(bars + kStages);
-  const uint32_t tmem_full = smem_addr(bars + 2 * kStages);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 1);
+  const uint32_t loaded0 = smem_addr(bars), ready0 = smem_addr(bars + kStages);
+  const uint32_t free0 = smem_addr(bars + 2 * kStages), tmem_full = smem_addr(bars + 3 * kStages);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kBN;
@@ -110,8 +115,9 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(full0 + 8 * s, 1 + kDeqWarps);
-      mbar_init(empty0 + 8 * s, 1);
+      mbar_init(loaded0 + 8 * s, 1);
+      mbar_init(ready0 + 8 * s, kDeqWarps);
+      mbar_init(free0 + 8 * s, 1);
     }
     mbar_init(tmem_full, 1);
     fence_mbar_init();
@@ -124,6 +130,7 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
     tma_prefetch_desc(&tm_act);
     tma_prefetch_desc(&tm_ext_a);
     tma_prefetch_desc(&tm_ext_b);
+    tma_prefetch_desc(&tm_codes);
   }
   tc_fence_before();
   __syncthreads();
@@ -136,22 +143,26 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
       for (int kb = 0; kb < nkb; ++kb) {
         const int s = kb % kStages;
         const uint32_t ph = (kb / kStages) & 1;
-        if (!mbar_wait(empty0 + 8 * s, ph ^ 1, p.status, kFlagTimeoutProducer)) break;
+        if (!mbar_wait(free0 + 8 * s, ph ^ 1, p.status, kFlagTimeoutProducer)) break;
         const uint32_t a_dst = smem_addr(smem + s * kStageBytes);
         const uint32_t b_dst = a_dst + kABytes;
+        const uint32_t c_dst = b_dst + kBBytes;
+        const uint32_t bar = loaded0 + 8 * s;
         if (kb < nkb_w) {
-          mbar_arrive_expect_tx(full0 + 8 * s, kABytes);
-          tma_load_2d(a_dst, &tm_act, full0 + 8 * s, kb * kBK, static_cast<int32_t>(m0));
+          mbar_arrive_expect_tx(bar, kABytes + kCBytes);
+          tma_load_2d(a_dst, &tm_act, bar, kb * kBK, static_cast<int32_t>(m0));
+          if (!kDX) tma_load_2d(c_dst, &tm_codes, bar, static_cast<int32_t>(n0 / 2), kb * kBK);
+          else tma_load_2d(c_dst, &tm_codes, bar, kb * (kBK / 2), static_cast<int32_t>(n0));
         } else {
           const int j = kb - nkb_w;
-          mbar_arrive_expect_tx(full0 + 8 * s, kABytes + kBBytes);
-          tma_load_2d(a_dst, &tm_ext_a, full0 + 8 * s, j * kBK, static_cast<int32_t>(m0));
+          mbar_arrive_expect_tx(bar, kABytes + kBBytes);
+          tma_load_2d(a_dst, &tm_ext_a, bar, j * kBK, static_cast<int32_t>(m0));
           if (!kDX) {
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-              tma_load_2d(b_dst + i * 8192, &tm_ext_b, full0 + 8 * s, static_cast<int32_t>(n0 + 64 * i), j * kBK);
+              tma_load_2d(b_dst + i * 8192, &tm_ext_b, bar, static_cast<int32_t>(n0 + 64 * i), j * kBK);
           } else {
-            tma_load_2d(b_dst, &tm_ext_b, full0 + 8 * s, j * kBK, static_cast<int32_t>(n0));
+            tma_load_2d(b_dst, &tm_ext_b, bar, j * kBK, static_cast<int32_t>(n0));
           }
         }
       }
@@ -160,11 +171,11 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, 256, false, !kDX);
-      bool ok = true;
-      for (int kb = 0; kb < nkb && ok; ++kb) {
+      for (int kb = 0; kb < nkb; ++kb) {
         const int s = kb % kStages;
         const uint32_t ph = (kb / kStages) & 1;
-        if (!mbar_wait(full0 + 8 * s, ph, p.status, kFlagTimeoutMma)) { ok = false; break; }
+        if (!mbar_wait(ready0 + 8 * s, ph, p.status, kFlagTimeoutMma)) break;
+        if (!mbar_wait(loaded0 + 8 * s, ph, p.status, kFlagTimeoutMma)) break;
         tc_fence_after();
         int nk16 = 4;
         if (kb >= nkb_w) nk16 = min(4, (p.r - (kb - nkb_w) * kBK + 15) / 16);
@@ -179,7 +190,7 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
             umma_bf16(tmem_base + h * 256, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
         }
-        umma_commit(empty0 + 8 * s);
+        umma_commit(free0 + 8 * s);
       }
       umma_commit(tmem_full);
     }
@@ -190,52 +201,67 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
     const int64_t blocks_per_row = p.w_out / kBlock;
     int64_t blk;                                    // block index at kb = 0
     bool valid;
-    uint32_t row_off;                               // byte offset of this thread's 8 chunks
+    uint32_t row_off;                               // byte offset of this thread's 8 chunks (weight tile)
+    uint32_t code_off0, code_off1;                  // byte offsets of its two 16-byte code chunks
     int swz;
     if (!kDX) {
-      const int kr = t >> 2, j = t & 3;             // k row in tile, 64-wide n block
+      // Quarter-warps (8 lanes) take 8 consecutive k rows of one 64-wide n block,
+      // so their 16-byte stores fall in 8 distinct bank groups.
+      const int kr = (t & 7) + ((t >> 5) << 3), j = (t >> 3) & 3;
       valid = (n0 + 64 * j) < p.N;
       blk = static_cast<int64_t>(kr) * blocks_per_row + (n0 >> 6) + j;
       row_off = j * 8192 + (kr >> 3) * 1024 + (kr & 7) * 128;
       swz = kr & 7;
+      // codes tile: 64 rows of 128 bytes, 128-byte swizzle
+      code_off0 = kr * 128 + (((2 * j) ^ (kr & 7)) << 4);
+      code_off1 = kr * 128 + (((2 * j + 1) ^ (kr & 7)) << 4);
     } else {
       const int nr = t;
       valid = (n0 + nr) < p.N;
       blk = (n0 + nr) * blocks_per_row;
       row_off = nr * 128;
       swz = nr & 7;
+      // codes tile: 256 rows of 32 bytes, 32-byte swizzle
+      const int x = (nr >> 2) & 1;
+      code_off0 = nr * 32 + ((0 ^ x) << 4);
+      code_off1 = nr * 32 + ((1 ^ x) << 4);
     }
     // K-step kb moves the block index by 64 rows (forward) or 1 block (dX).
     const int64_t blk_step = kDX ? 1 : 64 * blocks_per_row;
 
-    uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0;
-    uint8_t dqc = 0;
-    float dqs = 0.0f;
+    // absmax codes and scales, two K-steps ahead
+    uint8_t dqc0 = 0, dqc1 = 0;
+    float dqs0 = 0.0f, dqs1 = 0.0f;
     if (valid && nkb_w > 0) {
-      const uint4* src = reinterpret_cast<const uint4*>(p.codes + blk * 32);
-      c0 = __ldg(src);
-      c1 = __ldg(src + 1);
-      dqc = __ldg(p.dq_codes + blk);
-      dqs = __ldg(p.dq_scales + blk / kGroup);
+      dqc0 = __ldg(p.dq_codes + blk);
+      dqs0 = __ldg(p.dq_scales + blk / kGroup);
+    }
+    if (valid && nkb_w > 1) {
+      dqc1 = __ldg(p.dq_codes + blk + blk_step);
+      dqs1 = __ldg(p.dq_scales + (blk + blk_step) / kGroup);
     }
     for (int kb = 0; kb < nkb; ++kb) {
       const int s = kb % kStages;
       const uint32_t ph = (kb / kStages) & 1;
       // every lane waits; the warp leaves the loop together if the wait gave up
-      const bool got = mbar_wait(empty0 + 8 * s, ph ^ 1, p.status, kFlagTimeoutProducer);
+      const bool got = mbar_wait(loaded0 + 8 * s, ph, p.status, kFlagTimeoutProducer);
       if (!__all_sync(0xffffffffu, got)) break;
       if (kb < nkb_w) {
-        const uint32_t dst = smem_addr(smem + s * kStageBytes + kABytes) + row_off;
-        const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        const BlockLut lut = make_lut(valid ? absmax_deq(dqc, dqs) : 0.0f);
-        // prefetch the next K-step's block
-        if (valid && kb + 1 < nkb_w) {
-          const int64_t nb = blk + (kb + 1) * blk_step;
-          const uint4* src = reinterpret_cast<const uint4*>(p.codes + nb * 32);
-          c0 = __ldg(src);
-          c1 = __ldg(src + 1);
-          dqc = __ldg(p.dq_codes + nb);
-          dqs = __ldg(p.dq_scales + nb / kGroup);
+        const uint32_t stage = smem_addr(smem + s * kStageBytes);
+        const uint32_t dst = stage + kABytes + row_off;
+        const uint32_t csrc = stage + kABytes + kBBytes;
+        uint32_t w[8];
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(csrc + code_off0));
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7]) : "r"(csrc + code_off1));
+        const BlockLut lut = make_lut(valid ? absmax_deq(dqc0, dqs0) : 0.0f);
+        dqc0 = dqc1;
+        dqs0 = dqs1;
+        if (valid && kb + 2 < nkb_w) {
+          const int64_t nb = blk + (kb + 2) * blk_step;
+          dqc1 = __ldg(p.dq_codes + nb);
+          dqs1 = __ldg(p.dq_scales + nb / kGroup);
         }
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
@@ -247,7 +273,7 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
         fence_proxy_async_smem();
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(full0 + 8 * s);
+      if (lane == 0) mbar_arrive(ready0 + 8 * s);
     }
 
     // ------------------------------------------------------------ epilogue
@@ -303,24 +329,30 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-// Row-major bf16 matrix (rows x cols) -> 2-D tensor map with a (box_cols x box_rows)
-// box and 128-byte swizzle; box_cols * 2 must be <= 128.
-bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_cols, int box_rows) {
+// Row-major matrix (rows x cols elements of `esize` bytes) -> 2-D tensor map with
+// a (box_cols x box_rows) box; box_cols * esize must not exceed the swizzle span.
+bool make_map_t(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_cols, int box_rows,
+                CUtensorMapDataType dtype, int esize, CUtensorMapSwizzle swizzle) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols * 2)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols * esize)};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
-  CUresult rc = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult rc = enc(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return rc == CUDA_SUCCESS;
 }
 
+// bf16 matrix, 128-byte swizzle (box_cols <= 64).
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_cols, int box_rows) {
+  return make_map_t(m, base, rows, cols, box_cols, box_rows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 template <bool kDX>
-cudaError_t launch_gemm(const CUtensorMap& act, const CUtensorMap& ea, const CUtensorMap& eb, const GemmArgs& a,
-                        cudaStream_t stream) {
+cudaError_t launch_gemm(const CUtensorMap& act, const CUtensorMap& ea, const CUtensorMap& eb, const CUtensorMap& cm,
+                        const GemmArgs& a, cudaStream_t stream) {
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -333,7 +365,7 @@ cudaError_t launch_gemm(const CUtensorMap& act, const CUtensorMap& ea, const CUt
   dim3 grid(static_cast<unsigned>((a.N + kBN - 1) / kBN), static_cast<unsigned>((a.M + kBM - 1) / kBM));
   const int which = kDX ? QLORA_KERNEL_DX_GEMM : QLORA_KERNEL_FWD_GEMM;
   timing_before(which, stream);
-  nf4_gemm_kernel<kDX><<<grid, kThreads, kSmemBytes, stream>>>(act, ea, eb, a);
+  nf4_gemm_kernel<kDX><<<grid, kThreads, kSmemBytes, stream>>>(act, ea, eb, cm, a);
   timing_after(which, stream);
   count_launch();
   return cudaGetLastError();
@@ -344,23 +376,27 @@ cudaError_t launch_gemm(const CUtensorMap& act, const CUtensorMap& ea, const CUt
 // Y = X deq(W) + V B.
 cudaError_t launch_fwd_gemm(const WeightView& w, const uint16_t* X, const uint16_t* V, const uint16_t* B,
                             int64_t M, int r, uint16_t* Y, uint32_t* status, cudaStream_t stream) {
-  CUtensorMap act, ea, eb;
+  CUtensorMap act, ea, eb, cm;
+  // codes as a (in x out/2) byte matrix: 64 rows x 128 bytes per K-step, 128-byte swizzle
   if (!make_map(&act, X, M, w.in, 64, 256) || !make_map(&ea, V, M, r, 64, 256) ||
-      !make_map(&eb, B, r, w.out, 64, 64))
+      !make_map(&eb, B, r, w.out, 64, 64) ||
+      !make_map_t(&cm, w.codes, w.in, w.out / 2, 128, 64, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   GemmArgs a{w.codes, w.dq_codes, w.dq_scales, w.out, M, w.out, w.in, r, Y, status};
-  return launch_gemm<false>(act, ea, eb, a, stream);
+  return launch_gemm<false>(act, ea, eb, cm, a, stream);
 }
 
 // dX = dY deq(W)^T + U A^T.
 cudaError_t launch_dx_gemm(const WeightView& w, const uint16_t* dY, const uint16_t* U, const uint16_t* A,
                            int64_t M, int r, uint16_t* dX, uint32_t* status, cudaStream_t stream) {
-  CUtensorMap act, ea, eb;
+  CUtensorMap act, ea, eb, cm;
+  // codes as a (in x out/2) byte matrix: 256 rows x 32 bytes per K-step, 32-byte swizzle
   if (!make_map(&act, dY, M, w.out, 64, 256) || !make_map(&ea, U, M, r, 64, 256) ||
-      !make_map(&eb, A, w.in, r, 64, 256))
+      !make_map(&eb, A, w.in, r, 64, 256) ||
+      !make_map_t(&cm, w.codes, w.in, w.out / 2, 32, 256, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, CU_TENSOR_MAP_SWIZZLE_32B))
     return cudaErrorInvalidValue;
   GemmArgs a{w.codes, w.dq_codes, w.dq_scales, w.out, M, w.in, w.out, r, dX, status};
-  return launch_gemm<true>(act, ea, eb, a, stream);
+  return launch_gemm<true>(act, ea, eb, cm, a, stream);
 }
 
 }  // namespace qlora

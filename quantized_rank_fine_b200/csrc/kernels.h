@@ -33,16 +33,25 @@ cudaError_t launch_merge(const uint8_t* codes, const uint8_t* dq_codes, const fl
                          const uint16_t* A, const uint16_t* B, int r, int64_t n_in, int64_t n_out,
                          bool bf16, void* out, cudaStream_t stream);
 
-// Rank-r products; `part` is fp32 scratch of skinny_partial_floats(...) floats.
+// Rank-r products (tcgen05); `part` is fp32 scratch of skinny_partial_floats(...)
+// floats, `tickets` the workspace's ticket words (zero between launches, left at
+// zero), `status` the workspace status word.
 size_t skinny_partial_floats(int64_t out_rows, int r, int64_t k_total);
 cudaError_t launch_xa(const uint16_t* X, const uint16_t* A, int64_t M, int64_t n_in, int r, uint16_t* V,
-                      float* part, cudaStream_t stream);
+                      float* part, uint32_t* tickets, uint32_t* status, cudaStream_t stream);
 cudaError_t launch_dybt(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t n_out, int r,
-                        uint16_t* U, float* part, cudaStream_t stream);
+                        uint16_t* U, float* part, uint32_t* tickets, uint32_t* status, cudaStream_t stream);
 cudaError_t launch_xtu(const uint16_t* X, const uint16_t* U, int64_t M, int64_t n_in, int r, float* dA,
-                       float* part, cudaStream_t stream);
+                       float* part, uint32_t* tickets, uint32_t* status, cudaStream_t stream);
 cudaError_t launch_vtdy(const uint16_t* V, const uint16_t* dY, int64_t M, int64_t n_out, int r,
-                        float* dB, float* part, cudaStream_t stream);
+                        float* dB, float* part, uint32_t* tickets, uint32_t* status, cudaStream_t stream);
+
+// Small-M forward (M <= 16): base + adapter, split-K with a last-CTA finalize.
+// `part` holds gemv_workspace_bytes(...) bytes; `tickets` (N / 64 words) start
+// and end at 0.
+size_t gemv_workspace_bytes(int64_t M, int64_t K, int64_t N);
+cudaError_t launch_gemv(const WeightView& w, const uint16_t* X, const uint16_t* V, const uint16_t* B, int64_t M,
+                        int r, uint16_t* Y, float* part, uint32_t* tickets, cudaStream_t stream);
 
 // Fused dequant GEMMs (tcgen05); `status` is the workspace status word.
 cudaError_t launch_fwd_gemm(const WeightView& w, const uint16_t* X, const uint16_t* V, const uint16_t* B,

@@ -1,300 +1,335 @@
-// Rank-r side products of the adapted layer.
+// Rank-r side products of the adapted layer on the tcgen05 tensor cores.
 //
 //   V  = X A        (M x r)   forward intermediate ("How it works" step 2, (X A) B)
 //   U  = dY B^T     (M x r)   backward intermediate
 //   dA = X^T U      (in x r)  ("How it works" step 4, dA = dW B^T with dW = X^T dY)
-//   dB = V^T dY     (r x out) (dB = A^T dW)
+//   dB = V^T dY     (r x out) (dB = A^T dW), computed as dB^T = dY^T V and stored transposed
 //
-// Each is a contraction with one side only r (<= 64 per pass) wide, so the
-// kernels are bound by reading the big operand (X or dY) once from HBM; the
-// reduction dimension (in/out for V/U, the M tokens for dA/dB) is split across
-// CTAs so that even small M fills the 148 SMs, with fp32 partial sums written to
-// the workspace and a second kernel adding the splits in a fixed order
-// (deterministic results).  Tiles are 64 x 64 bf16 staged by cp.async into
-// 128-byte-swizzled shared memory and consumed with ldmatrix + mma.sync
-// m16n8k16 (bf16 in, fp32 accumulate).
+// Each is D (rows x r) = sum_k Aop(rows, k) Bop(r, k) with r <= 64 per pass, bound
+// by streaming the big operand (X or dY) from HBM once.  A CTA owns 128 output
+// rows and one slice of the reduction: TMA brings 128 x 64 (Aop) and 64 x 64
+// (Bop) bf16 tiles into a 4-stage shared-memory ring (128-byte swizzle, K- or
+// MN-major as the operand sits in memory; two CTAs per SM), one thread issues
+// tcgen05.mma into a 128 x r fp32 TMEM accumulator, and four warps move the
+// result out.  The reduction is split across CTAs so that the whole grid is
+// resident at once (two per SM);
+// each split writes an fp32 partial tile to the workspace and the last CTA of a
+// tile (an atomic ticket in the workspace, left at zero afterwards) adds them in
+// split order, so the sums are deterministic and need no second launch.
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
+
+#include <cudaTypedefs.h>
 
 namespace qlora {
 
 namespace {
 
-constexpr int kSkThreads = 128;    // 4 warps, 16 output rows each
-constexpr int kTile = 64;          // rows/cols of a staged tile
-constexpr int kTileBytes = kTile * kTile * 2;
+using namespace sm100;
 
-// One operand of the contraction as it sits in global memory: element
-// (row, col) at base[row * ld + col]; rows >= nrows or cols >= ncols read as 0.
-// The reduction index k runs along rows when k_on_rows, else along columns.
-struct Operand {
-  const uint16_t* base;
-  int64_t ld;
-  int64_t nrows, ncols;
-  bool k_on_rows;
-  int64_t fixed0;   // origin of the non-k dimension for this CTA
-};
+constexpr int kSkThreads = 192;    // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 epilogue
+constexpr int kSkStages = 4;       // 96 KB ring: two CTAs per SM
+constexpr int kRowsT = 128;        // output rows per CTA (UMMA M)
+constexpr int kKT = 64;            // reduction step
+constexpr int kColsT = 64;         // output columns per CTA
+constexpr uint32_t kATile = kRowsT * kKT * 2;    // 16 KB
+constexpr uint32_t kBTile = kColsT * kKT * 2;    // 8 KB
+constexpr uint32_t kSkStage = kATile + kBTile;
+constexpr uint32_t kSkSmem = kSkStages * kSkStage + 1024 + 256;
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ int swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-  const int n = valid ? 16 : 0;
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(n));
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
-
-// Stage the 64x64 tile of `op` whose k-origin is k0 into swizzled smem.
-__device__ __forceinline__ void load_tile(const Operand& op, int64_t k0, uint8_t* smem) {
-  const int64_t r0 = op.k_on_rows ? k0 : op.fixed0;
-  const int64_t c0 = op.k_on_rows ? op.fixed0 : k0;
-  const uint32_t s = smem_u32(smem);
-#pragma unroll
-  for (int i = 0; i < (kTile * 8) / kSkThreads; ++i) {
-    const int e = threadIdx.x + i * kSkThreads;
-    const int row = e >> 3, chunk = e & 7;
-    const int64_t gr = r0 + row, gc = c0 + chunk * 8;
-    const bool valid = (gr < op.nrows) && (gc < op.ncols);
-    const uint16_t* src = valid ? op.base + gr * op.ld + gc : op.base;
-    cp_async16(s + swz(row, chunk), src, valid);
-  }
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(addr));
-}
-
-__device__ __forceinline__ void mma_bf16(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};\n"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// C (64 x RC) += Aop (64 x K) * Bop (K x RC) over this CTA's k-range.
-//   Aop stored [m][k] (a_trans = false) or [k][m] (a_trans = true).
-//   Bop stored [n][k] (b_trans = false) or [k][n] (b_trans = true).
-// Output: fp32 partial at part[(split * out_rows + row) * out_ld + col], or,
-// with a single split, the final value (bf16 or fp32, optionally transposed).
-struct SkinnyArgs {
-  Operand a, b;
-  int64_t k_begin, k_per_split, k_total;
-  int64_t out_rows;       // rows of C (M, or in/out for the weight gradients)
-  int r;                  // columns of C
-  float* part;            // fp32 partials [splits][out_rows][r] (splits > 1)
-  void* out;              // final output when splits == 1
-  int out_kind;           // 0 = bf16 [row][r], 1 = fp32 [row][r], 2 = fp32 transposed [r][row]
+struct SkArgs {
+  int64_t rows;          // output rows
+  int r;                 // output columns
+  int64_t k_total;       // reduction length
+  int64_t k_per_split;   // multiple of 64
   int splits;
+  float* part;           // fp32 partials [splits][rows][r] (splits > 1)
+  uint32_t* tickets;     // one per (row tile, column chunk), zero between launches
+  void* out;
+  int out_kind;          // 0 = bf16 [row][r], 1 = fp32 [row][r], 2 = fp32 transposed [r][row]
+  uint32_t* status;
 };
 
-template <bool kATrans, bool kBTrans>
-__global__ void __launch_bounds__(kSkThreads)
-skinny_mma_kernel(SkinnyArgs p) {
-  __shared__ __align__(128) uint8_t smem[2][2][kTileBytes];
+__device__ __forceinline__ void store_pair(const SkArgs& p, int64_t row, int col, float v0, float v1) {
+  if (p.out_kind == 0) {
+    *reinterpret_cast<uint32_t*>(reinterpret_cast<uint16_t*>(p.out) + row * p.r + col) = pack_bf16x2(v0, v1);
+  } else if (p.out_kind == 1) {
+    *reinterpret_cast<float2*>(reinterpret_cast<float*>(p.out) + row * p.r + col) = make_float2(v0, v1);
+  } else {
+    float* d = reinterpret_cast<float*>(p.out);
+    d[static_cast<int64_t>(col) * p.rows + row] = v0;
+    d[static_cast<int64_t>(col + 1) * p.rows + row] = v1;
+  }
+}
+
+// A_MN: Aop stored with the row index contiguous (MN-major), else k contiguous.
+// B_MN: Bop stored with the column index contiguous (MN-major), else k contiguous.
+template <bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(kSkThreads, 2)
+skinny_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                 const SkArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSkStages * kSkStage);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kSkStages + 1);
+  __shared__ int last;
+  const uint32_t full0 = smem_addr(bars), free0 = smem_addr(bars + kSkStages);
+  const uint32_t tmem_full = smem_addr(bars + 2 * kSkStages);
+
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kRowsT;
   const int split = blockIdx.y;
-  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kTile;
-  const int j0 = blockIdx.z * kTile;
+  const int col0 = blockIdx.z * kColsT;
+  const int cols = min(kColsT, p.r - col0);
+  const int n_mma = (cols + 15) / 16 * 16;
+  const int64_t kbeg = split * p.k_per_split;
+  const int64_t kend = min(p.k_total, kbeg + p.k_per_split);
+  const int nkb = kend > kbeg ? static_cast<int>((kend - kbeg + kKT - 1) / kKT) : 0;
 
-  Operand A = p.a, B = p.b;
-  A.fixed0 = m0;
-  B.fixed0 = j0;
-  const int64_t kb = p.k_begin + split * p.k_per_split;
-  const int64_t ke = min(p.k_total, kb + p.k_per_split);
-  const int nk = ke > kb ? static_cast<int>((ke - kb + kTile - 1) / kTile) : 0;
-
-  float acc[8][4];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
-  const int ntile = min(8, (p.r - j0 + 7) / 8);   // n8 tiles that hold real columns
-
-  if (nk > 0) {
-    load_tile(A, kb, smem[0][0]);
-    load_tile(B, kb, smem[0][1]);
-    cp_async_commit();
-  }
-  for (int t = 0; t < nk; ++t) {
-    const int cur = t & 1;
-    if (t + 1 < nk) {
-      load_tile(A, kb + (t + 1) * kTile, smem[cur ^ 1][0]);
-      load_tile(B, kb + (t + 1) * kTile, smem[cur ^ 1][1]);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kSkStages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(free0 + 8 * s, 1);
     }
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-    const uint32_t sa = smem_u32(smem[cur][0]);
-    const uint32_t sb = smem_u32(smem[cur][1]);
-#pragma unroll
-    for (int ks = 0; ks < kTile; ks += 16) {
-      uint32_t af[4];
-      const int mi = warp * 16;
-      if (!kATrans) {
-        const int row = mi + (lane & 15), chunk = (ks >> 3) + (lane >> 4);
-        ldsm_x4(sa + swz(row, chunk), af[0], af[1], af[2], af[3]);
-      } else {
-        const int q = lane >> 3;
-        const int row = ks + (lane & 7) + ((q >> 1) << 3), chunk = (mi >> 3) + (q & 1);
-        ldsm_x4_t(sa + swz(row, chunk), af[0], af[1], af[2], af[3]);
-      }
-#pragma unroll
-      for (int np = 0; np < 4; ++np) {          // pairs of n8 tiles
-        if (2 * np >= ntile) break;
-        uint32_t b0, b1, b2, b3;
-        const int q = lane >> 3;
-        if (!kBTrans) {
-          // matrices: (n 0-7, k 0-7), (n 0-7, k 8-15), (n 8-15, k 0-7), (n 8-15, k 8-15)
-          const int row = np * 16 + (lane & 7) + ((q >> 1) << 3), chunk = (ks >> 3) + (q & 1);
-          ldsm_x4(sb + swz(row, chunk), b0, b1, b2, b3);
+    mbar_init(tmem_full, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), 64);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % kSkStages;
+        const uint32_t ph = (kb / kSkStages) & 1;
+        if (!mbar_wait(free0 + 8 * s, ph ^ 1, p.status, kFlagTimeoutProducer)) break;
+        const uint32_t a_dst = smem_addr(smem + s * kSkStage), b_dst = a_dst + kATile;
+        const uint32_t bar = full0 + 8 * s;
+        const int32_t k0 = static_cast<int32_t>(kbeg + kb * kKT);
+        mbar_arrive_expect_tx(bar, kSkStage);
+        if (!A_MN) {
+          tma_load_2d(a_dst, &tm_a, bar, k0, static_cast<int32_t>(row0));
         } else {
-          // matrices: (k 0-7, n 0-7), (k 8-15, n 0-7), (k 0-7, n 8-15), (k 8-15, n 8-15)
-          const int row = ks + (lane & 7) + ((q & 1) << 3), chunk = np * 2 + (q >> 1);
-          ldsm_x4_t(sb + swz(row, chunk), b0, b1, b2, b3);
+          tma_load_2d(a_dst, &tm_a, bar, static_cast<int32_t>(row0), k0);
+          tma_load_2d(a_dst + 8192, &tm_a, bar, static_cast<int32_t>(row0 + 64), k0);
         }
-        mma_bf16(acc[2 * np], af, b0, b1);
-        if (2 * np + 1 < ntile) mma_bf16(acc[2 * np + 1], af, b2, b3);
+        if (!B_MN) tma_load_2d(b_dst, &tm_b, bar, k0, col0);
+        else tma_load_2d(b_dst, &tm_b, bar, col0, k0);
       }
     }
-    __syncthreads();
-  }
-
-  // Epilogue: c0,c1 -> (row g, cols 2t, 2t+1); c2,c3 -> (row g+8, same cols).
-  const int g = lane >> 2, tq = lane & 3;
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, n_mma, A_MN, B_MN);
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % kSkStages;
+        const uint32_t ph = (kb / kSkStages) & 1;
+        if (!mbar_wait(full0 + 8 * s, ph, p.status, kFlagTimeoutMma)) break;
+        tc_fence_after();
+        const uint32_t a_base = smem_addr(smem + s * kSkStage), b_base = a_base + kATile;
 #pragma unroll
-  for (int nt = 0; nt < 8; ++nt) {
-    if (nt >= ntile) break;
-    const int col = j0 + nt * 8 + 2 * tq;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int64_t row = m0 + warp * 16 + g + 8 * h;
-      if (row >= p.out_rows) continue;
-      const float v0 = acc[nt][2 * h], v1 = acc[nt][2 * h + 1];
-      if (p.splits > 1) {
-        float* d = p.part + (static_cast<int64_t>(split) * p.out_rows + row) * p.r + col;
-        *reinterpret_cast<float2*>(d) = make_float2(v0, v1);
-      } else if (p.out_kind == 0) {
-        uint16_t* d = reinterpret_cast<uint16_t*>(p.out) + row * p.r + col;
-        *reinterpret_cast<uint32_t*>(d) = pack_bf16x2(v0, v1);
-      } else if (p.out_kind == 1) {
-        float* d = reinterpret_cast<float*>(p.out) + row * p.r + col;
-        *reinterpret_cast<float2*>(d) = make_float2(v0, v1);
+        for (int kk = 0; kk < kKT / 16; ++kk) {
+          const uint64_t ad = A_MN ? smem_desc_sw128(a_base + kk * 2048, 8192, 1024)
+                                   : smem_desc_sw128(a_base + kk * 32, 16, 1024);
+          const uint64_t bd = B_MN ? smem_desc_sw128(b_base + kk * 2048, 8192, 1024)
+                                   : smem_desc_sw128(b_base + kk * 32, 16, 1024);
+          umma_bf16(tmem_base, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+        }
+        umma_commit(free0 + 8 * s);
+      }
+      umma_commit(tmem_full);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2-5)
+    const bool ok =
+        __all_sync(0xffffffffu, nkb == 0 || mbar_wait(tmem_full, 0, p.status, kFlagTimeoutEpilogue));
+    tc_fence_after();
+    const int quarter = warp & 3;                  // TMEM lanes 32*quarter .. +31
+    const int64_t row = row0 + quarter * 32 + lane;
+    const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+    float* dst_part = p.part + (static_cast<int64_t>(split) * p.rows + row) * p.r + col0;
+#pragma unroll 1
+    for (int c = 0; c < n_mma; c += 16) {
+      uint32_t v[16];
+      if (ok && nkb > 0) {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+            "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+              "=r"(v[15])
+            : "r"(taddr + c));
+        tmem_ld_wait();
       } else {
-        float* d = reinterpret_cast<float*>(p.out);
-        d[static_cast<int64_t>(col) * p.out_rows + row] = v0;
-        d[static_cast<int64_t>(col + 1) * p.out_rows + row] = v1;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = 0u;   // an empty slice contributes zeros
+      }
+      if (row < p.rows) {
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
+          if (c + i >= cols) break;
+          const float v0 = __uint_as_float(v[i]), v1 = __uint_as_float(v[i + 1]);
+          if (p.splits == 1) store_pair(p, row, col0 + c + i, v0, v1);
+          else *reinterpret_cast<float2*>(dst_part + c + i) = make_float2(v0, v1);
+        }
       }
     }
   }
-}
 
-// Sum the split partials in split order and write the final layout.
-__global__ void reduce_splits_kernel(const float* __restrict__ part, int splits, int64_t rows, int r,
-                                     void* __restrict__ out, int out_kind) {
-  const int64_t n = rows * r;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    float s = 0.0f;
-    for (int k = 0; k < splits; ++k) s += part[k * n + i];
-    if (out_kind == 0) {
-      reinterpret_cast<__nv_bfloat16*>(out)[i] = __float2bfloat16_rn(s);
-    } else if (out_kind == 1) {
-      reinterpret_cast<float*>(out)[i] = s;
-    } else {
-      const int64_t row = i / r, col = i % r;
-      reinterpret_cast<float*>(out)[col * rows + row] = s;
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 64);
+  }
+  if (p.splits == 1) return;
+
+  // ------------------------------------------------------------ split reduction
+  __threadfence();
+  __syncthreads();
+  const int tile = blockIdx.x + gridDim.x * blockIdx.z;
+  if (threadIdx.x == 0) last = (atomicAdd(p.tickets + tile, 1u) == static_cast<uint32_t>(p.splits - 1));
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  const int pairs = cols / 2;
+  for (int e = threadIdx.x; e < kRowsT * pairs; e += kSkThreads) {
+    const int rr = e / pairs, cc = 2 * (e - rr * pairs);
+    const int64_t row = row0 + rr;
+    if (row >= p.rows) continue;
+    float v0 = 0.0f, v1 = 0.0f;
+    for (int sp = 0; sp < p.splits; ++sp) {
+      const float2 x =
+          __ldcg(reinterpret_cast<const float2*>(p.part + (static_cast<int64_t>(sp) * p.rows + row) * p.r + col0 + cc));
+      v0 += x.x;
+      v1 += x.y;
     }
+    store_pair(p, row, col0 + cc, v0, v1);
   }
+  if (threadIdx.x == 0) p.tickets[tile] = 0u;
 }
 
-constexpr int kTargetCtas = 2 * 148;
+// ---------------------------------------------------------------- host side
 
-int choose_splits(int64_t base_ctas, int64_t k_total) {
-  const int64_t ktiles = (k_total + kTile - 1) / kTile;
-  int64_t s = (kTargetCtas + base_ctas - 1) / base_ctas;
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// bf16 row-major (rows x cols) -> tensor map with a (box_cols x box_rows) box, 128B swizzle.
+bool bf16_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_cols, int box_rows) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols * 2)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr int kResident = 2 * 148;   // CTAs that fit on the GPU at once
+
+struct Plan {
+  int splits;
+  int64_t kps;
+  dim3 grid;
+};
+
+Plan plan(int64_t rows, int r, int64_t k_total) {
+  const int64_t rt = (rows + kRowsT - 1) / kRowsT;
+  const int ct = (r + kColsT - 1) / kColsT;
+  const int64_t ktiles = (k_total + kKT - 1) / kKT;
+  // as many reduction slices as keep the whole grid resident (one wave), each
+  // slice at least two K-steps long
+  int64_t s = kResident / (rt * ct);
   s = std::min<int64_t>(s, std::max<int64_t>(1, ktiles / 2));
-  s = std::min<int64_t>(s, kMaxSplits);
-  return static_cast<int>(std::max<int64_t>(1, s));
+  s = std::max<int64_t>(1, std::min<int64_t>(s, kMaxSplits));
+  const int64_t kps = (ktiles + s - 1) / s * kKT;
+  s = (k_total + kps - 1) / kps;
+  return Plan{static_cast<int>(s), kps, dim3(static_cast<unsigned>(rt), static_cast<unsigned>(s), ct)};
 }
 
-cudaError_t run_skinny(bool a_trans, bool b_trans, const Operand& a, const Operand& b,
-                       int64_t k_total, int64_t out_rows, int r, void* out, int out_kind,
-                       float* part, cudaStream_t stream) {
-  const int64_t mt = (out_rows + kTile - 1) / kTile;
-  const int rt = (r + kTile - 1) / kTile;
-  const int splits = choose_splits(mt * rt, k_total);
-  int64_t kps = (k_total + splits - 1) / splits;
-  kps = (kps + kTile - 1) / kTile * kTile;
-  SkinnyArgs p{a, b, 0, kps, k_total, out_rows, r, part, out, out_kind, splits};
-  dim3 grid(static_cast<unsigned>(mt), splits, rt);
-  timing_before(QLORA_KERNEL_RANK_R, stream);
-  if (!a_trans && b_trans) skinny_mma_kernel<false, true><<<grid, kSkThreads, 0, stream>>>(p);
-  else if (!a_trans && !b_trans) skinny_mma_kernel<false, false><<<grid, kSkThreads, 0, stream>>>(p);
-  else if (a_trans && b_trans) skinny_mma_kernel<true, true><<<grid, kSkThreads, 0, stream>>>(p);
-  else skinny_mma_kernel<true, false><<<grid, kSkThreads, 0, stream>>>(p);
-  count_launch();
-  cudaError_t e = cudaGetLastError();
-  if (e == cudaSuccess && splits > 1) {
-    const int64_t n = out_rows * r;
-    const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, 4 * 148));
-    reduce_splits_kernel<<<blocks, 256, 0, stream>>>(part, splits, out_rows, r, out, out_kind);
-    count_launch();
-    e = cudaGetLastError();
+template <bool A_MN, bool B_MN>
+cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows, int r, int64_t k_total, void* out,
+                int out_kind, float* part, uint32_t* tickets, uint32_t* status, cudaStream_t stream) {
+  static bool set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(skinny_tc_kernel<A_MN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kSkSmem));
+    if (e != cudaSuccess) return e;
+    set[dev] = true;
   }
+  const Plan pl = plan(rows, r, k_total);
+  SkArgs a{rows, r, k_total, pl.kps, pl.splits, part, tickets, out, out_kind, status};
+  timing_before(QLORA_KERNEL_RANK_R, stream);
+  skinny_tc_kernel<A_MN, B_MN><<<pl.grid, kSkThreads, kSkSmem, stream>>>(ta, tb, a);
   timing_after(QLORA_KERNEL_RANK_R, stream);
-  return e;
+  count_launch();
+  return cudaGetLastError();
 }
 
 }  // namespace
 
 size_t skinny_partial_floats(int64_t out_rows, int r, int64_t k_total) {
-  const int64_t mt = (out_rows + kTile - 1) / kTile;
-  const int rt = (r + kTile - 1) / kTile;
-  const int splits = choose_splits(mt * rt, k_total);
-  return splits > 1 ? static_cast<size_t>(splits) * out_rows * r : 0;
+  const Plan pl = plan(out_rows, r, k_total);
+  return pl.splits > 1 ? static_cast<size_t>(pl.splits) * out_rows * r : 0;
 }
 
-// V = X A: X (M, in) row-major [m][k]; A (in, r) row-major [k][j].
-cudaError_t launch_xa(const uint16_t* X, const uint16_t* A, int64_t M, int64_t n_in, int r,
-                      uint16_t* V, float* part, cudaStream_t stream) {
-  Operand a{X, n_in, M, n_in, false, 0};
-  Operand b{A, r, n_in, r, true, 0};
-  return run_skinny(false, true, a, b, n_in, M, r, V, 0, part, stream);
+// V = X A: Aop = X (M x in, k contiguous); Bop[j][k] = A[k][j] (j contiguous).
+cudaError_t launch_xa(const uint16_t* X, const uint16_t* A, int64_t M, int64_t n_in, int r, uint16_t* V,
+                      float* part, uint32_t* tickets, uint32_t* status, cudaStream_t stream) {
+  CUtensorMap ta, tb;
+  if (!bf16_map(&ta, X, M, n_in, 64, 128) || !bf16_map(&tb, A, n_in, r, 64, 64)) return cudaErrorInvalidValue;
+  return run<false, true>(ta, tb, M, r, n_in, V, 0, part, tickets, status, stream);
 }
 
-// U = dY B^T: dY (M, out) [m][k]; B (r, out) row-major = [j][k].
-cudaError_t launch_dybt(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t n_out, int r,
-                        uint16_t* U, float* part, cudaStream_t stream) {
-  Operand a{dY, n_out, M, n_out, false, 0};
-  Operand b{B, n_out, r, n_out, false, 0};
-  return run_skinny(false, false, a, b, n_out, M, r, U, 0, part, stream);
+// U = dY B^T: Aop = dY (M x out, k contiguous); Bop = B (r x out, k contiguous).
+cudaError_t launch_dybt(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t n_out, int r, uint16_t* U,
+                        float* part, uint32_t* tickets, uint32_t* status, cudaStream_t stream) {
+  CUtensorMap ta, tb;
+  if (!bf16_map(&ta, dY, M, n_out, 64, 128) || !bf16_map(&tb, B, r, n_out, 64, 64)) return cudaErrorInvalidValue;
+  return run<false, false>(ta, tb, M, r, n_out, U, 0, part, tickets, status, stream);
 }
 
-// dA = X^T U (in, r): A-operand X stored [k = token][m = in]; U stored [k][j].
-cudaError_t launch_xtu(const uint16_t* X, const uint16_t* U, int64_t M, int64_t n_in, int r,
-                       float* dA, float* part, cudaStream_t stream) {
-  Operand a{X, n_in, M, n_in, true, 0};
-  Operand b{U, r, M, r, true, 0};
-  return run_skinny(true, true, a, b, M, n_in, r, dA, 1, part, stream);
+// dA = X^T U: Aop[i][m] = X[m][i] (i contiguous); Bop[j][m] = U[m][j] (j contiguous).
+cudaError_t launch_xtu(const uint16_t* X, const uint16_t* U, int64_t M, int64_t n_in, int r, float* dA,
+                       float* part, uint32_t* tickets, uint32_t* status, cudaStream_t stream) {
+  CUtensorMap ta, tb;
+  if (!bf16_map(&ta, X, M, n_in, 64, 64) || !bf16_map(&tb, U, M, r, 64, 64)) return cudaErrorInvalidValue;
+  return run<true, true>(ta, tb, n_in, r, M, dA, 1, part, tickets, status, stream);
 }
 
-// dB = V^T dY (r, out), computed as dB^T = dY^T V (out, r) and stored transposed.
-cudaError_t launch_vtdy(const uint16_t* V, const uint16_t* dY, int64_t M, int64_t n_out, int r,
-                        float* dB, float* part, cudaStream_t stream) {
-  Operand a{dY, n_out, M, n_out, true, 0};
-  Operand b{V, r, M, r, true, 0};
-  return run_skinny(true, true, a, b, M, n_out, r, dB, 2, part, stream);
+// dB^T = dY^T V: Aop[o][m] = dY[m][o] (o contiguous); Bop[j][m] = V[m][j]; stored as dB (r x out).
+cudaError_t launch_vtdy(const uint16_t* V, const uint16_t* dY, int64_t M, int64_t n_out, int r, float* dB,
+                        float* part, uint32_t* tickets, uint32_t* status, cudaStream_t stream) {
+  CUtensorMap ta, tb;
+  if (!bf16_map(&ta, dY, M, n_out, 64, 64) || !bf16_map(&tb, V, M, r, 64, 64)) return cudaErrorInvalidValue;
+  return run<true, true>(ta, tb, n_out, r, M, dB, 2, part, tickets, status, stream);
 }
 
 }  // namespace qlora
