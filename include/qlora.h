@@ -142,6 +142,29 @@ QLORA_API qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16_
                               uint16_t* V_save, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * The forward above for callers that cannot allocate device memory (no paper
+ * counterpart: the pages describe the method, not how a library hands out
+ * scratch space).  Some callers have no device allocator to give a workspace
+ * with: a host program using only this C ABI, a plugin inside a runtime that
+ * owns all device memory, or a path where a cudaMalloc and its possible device
+ * synchronisation is not acceptable.  This entry point takes the same arguments
+ * minus the workspace and uses a fixed array of QLORA_STATIC_WS_BYTES inside the
+ * library's own device memory instead (held by every GPU that loads the library
+ * until the process exits); it allocates nothing.
+ *   Returns QLORA_ERR_WORKSPACE, launching nothing, when the sizes need more than
+ *   QLORA_STATIC_WS_BYTES (qlora_workspace_bytes(QLORA_OP_FWD, ...) larger).
+ *   The first call on each device looks up the array's device address; make that
+ *   first call before any stream capture.  Every call shares the one array and
+ *   zeroes its bookkeeping words first; calls whose work overlaps on the GPU
+ *   (other streams, other threads) race and must not be issued.  A wait that
+ *   times out inside a kernel is not reported by this entry point.
+ */
+#define QLORA_STATIC_WS_BYTES (16u << 20)
+QLORA_API qlora_status qlora_linear_fwd_static_ws(const qlora_nf4_weight* w, const uint16_t* X, int64_t M,
+                                                  const uint16_t* A, const uint16_t* B, int r, uint16_t* Y,
+                                                  uint16_t* V_save, void* stream);
+
+/*
  * Backward of the adapted layer ("How it works" step 4; "The code, line by line":
  * dA = dW B^T, dB = A^T dW, here in the factored form that never forms dW):
  *   U  = bf16(dY B^T)

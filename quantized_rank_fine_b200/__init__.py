@@ -35,6 +35,7 @@ EXPORTS = (
     "qlora_quantize_nf4", "qlora_dequantize", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_merge",
     "qlora_workspace_bytes", "qlora_ws_init", "qlora_ws_status", "qlora_nf4_codebook",
     "qlora_adapter_params", "qlora_status_string", "qlora_time_kernel", "qlora_launch_count",
+    "qlora_linear_fwd_static_ws",
 )
 
 # Kernel ids of qlora_time_kernel.
@@ -79,6 +80,7 @@ def lib() -> ctypes.CDLL:
             "qlora_status_string": (ctypes.c_char_p, [i32]),
             "qlora_time_kernel": (i32, [i32, ctypes.POINTER(vp), ctypes.POINTER(vp), i32]),
             "qlora_launch_count": (ctypes.c_uint64, []),
+            "qlora_linear_fwd_static_ws": (i32, [wp, vp, i64, vp, vp, i32, vp, vp, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)

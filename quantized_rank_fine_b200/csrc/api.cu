@@ -92,11 +92,11 @@ struct WsLayout {
 };
 
 constexpr int64_t kGemvMaxM = 16;     // token counts served by the dequant-GEMV
-constexpr int64_t kTicketWords = 4096;  // split-K tickets of the GEMV: one per 64-column panel
+constexpr int64_t kTicketWords = static_cast<int64_t>(qlora::kWsTicketWords);
 // Every layout reserves the tickets right after the status words, so no call
-// ever writes that region except the GEMV, which leaves it zero.
-constexpr size_t kTicketOff = 256;
-constexpr size_t kFixedBytes = kTicketOff + kTicketWords * 4;
+// ever writes that region except the split-K kernels, which leave it zero.
+constexpr size_t kTicketOff = qlora::kWsStatusBytes;
+constexpr size_t kFixedBytes = qlora::kWsFixedBytes;
 
 WsLayout ws_layout(int op, int64_t M, int64_t in, int64_t out, int r) {
   WsLayout L{};

@@ -12,6 +12,12 @@ namespace qlora {
 
 constexpr int kMaxSplits = 16;   // most K/M splits of the rank-r kernels
 
+// Workspace prefix shared by every call: the status word(s) and the split-K
+// tickets (kept at zero between launches).
+constexpr size_t kWsStatusBytes = 256;
+constexpr size_t kWsTicketWords = 4096;
+constexpr size_t kWsFixedBytes = kWsStatusBytes + kWsTicketWords * 4;
+
 // Bookkeeping of the measurement helpers (defined in api.cu): every kernel
 // launch is counted; an armed timing hook brackets launches of one kernel kind.
 void count_launch();

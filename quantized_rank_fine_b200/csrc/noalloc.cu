@@ -1,0 +1,70 @@
+// Forward of the adapted layer for callers that cannot allocate device memory.
+//
+// qlora_linear_fwd needs a caller-provided workspace.  Some callers have no way
+// to provide one: a host program linked against this library through its C ABI
+// that has no device allocator of its own, a plugin or custom operator inside a
+// runtime that owns all device memory and exposes no scratch allocator, or a
+// latency-critical path where a cudaMalloc (which may synchronise the device)
+// is not acceptable once the program is running.  For them this file keeps a
+// fixed-size scratch array in the library's own device memory and runs the
+// same forward with it.
+//
+// The array is a file-scope __device__ variable: every GPU that loads the
+// library holds its kStaticWsBytes until the process exits.  In host code the
+// array's name is only a host-side stand-in, so its device address is looked up
+// with cudaGetSymbolAddress, once per device, on the first call made with that
+// device current; that first call should come before any stream capture.  All
+// calls share the array and it keeps the previous call's contents, so each call
+// first zeroes the part that must start at zero (status word and split-K
+// tickets).  Two calls whose work overlaps on the GPU (different streams, or
+// different host threads) race on the array.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "../../include/qlora.h"
+#include "kernels.h"
+
+namespace {
+
+constexpr size_t kStaticWsBytes = QLORA_STATIC_WS_BYTES;
+
+static __device__ __align__(256) unsigned char g_static_ws[kStaticWsBytes];
+
+std::mutex g_setup_mutex;
+void* g_static_ws_addr[64] = {};
+
+// Device address of g_static_ws on the current device (looked up once).
+qlora_status static_ws_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return QLORA_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  if (!g_static_ws_addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_static_ws) != cudaSuccess || !ptr) {
+      cudaGetLastError();
+      return QLORA_ERR_CUDA;
+    }
+    g_static_ws_addr[dev] = ptr;
+  }
+  *out = g_static_ws_addr[dev];
+  return QLORA_OK;
+}
+
+}  // namespace
+
+extern "C" qlora_status qlora_linear_fwd_static_ws(const qlora_nf4_weight* w, const uint16_t* X, int64_t M,
+                                                   const uint16_t* A, const uint16_t* B, int r, uint16_t* Y,
+                                                   uint16_t* V_save, void* stream) {
+  if (!w) return QLORA_ERR_INVALID_ARG;
+  const size_t need = qlora_workspace_bytes(QLORA_OP_FWD, M, w->in, w->out, r);
+  if (need == 0) return QLORA_ERR_SHAPE;
+  if (need > kStaticWsBytes) return QLORA_ERR_WORKSPACE;   // larger than the fixed array
+  void* ws = nullptr;
+  const qlora_status st = static_ws_address(&ws);
+  if (st != QLORA_OK) return st;
+  if (cudaMemsetAsync(ws, 0, qlora::kWsFixedBytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  return qlora_linear_fwd(w, X, M, A, B, r, Y, V_save, ws, kStaticWsBytes, stream);
+}
