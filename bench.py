@@ -228,16 +228,7 @@ def time_rows(wl, pk):
     torch.cuda.synchronize()
 
     def timed(fn, which, iters):
-        for i in range(3):
-            fn(i)
-        torch.cuda.synchronize()
-        tm = q.KernelTimer(which, iters)
-        for i in range(iters):
-            fn(i)
-        torch.cuda.synchronize()
-        ts = tm.times_ms()
-        tm.disarm()
-        return statistics.median(ts)
+        return graph_timed(fn, which, iters)
 
     hbm = pk["hbm_gbs"]
     iters = 30
@@ -261,6 +252,33 @@ def time_rows(wl, pk):
     return rows
 
 
+def graph_timed(fn, which, iters):
+    """Median duration (ms) of kernel `which` over `iters` calls of fn(i), the
+    calls captured in one CUDA graph and replayed, so that the device never
+    waits for the host between launches (short kernels would otherwise be timed
+    together with the host's launch overhead)."""
+    import torch
+    import quantized_rank_fine_b200 as q
+    for i in range(3):
+        fn(i)
+    torch.cuda.synchronize()
+    tm = q.KernelTimer(which, iters)
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side, capture_error_mode="relaxed"):
+            for i in range(iters):
+                fn(i)
+    torch.cuda.current_stream().wait_stream(side)
+    tm.disarm()
+    graph.replay()
+    torch.cuda.synchronize()
+    t = statistics.median(tm.times_ms())
+    del graph
+    return t
+
+
 def time_gemv(pk):
     """Small-M forward (M = 1, 4, 16) on the 4096 x 4096 and 4096 x 11008 shapes,
     r = 16: the dequant-GEMV kernel's HBM bandwidth.  Algorithmic bytes: codes,
@@ -281,26 +299,7 @@ def time_gemv(pk):
             Y = torch.empty((M, n_out), dtype=torch.bfloat16, device="cuda")
             V = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
             ws = q.Workspace()
-            for i in range(3):
-                q.qlora_linear_fwd(wts[i % reps], X, A, B, ws, Y=Y, V=V)
-            torch.cuda.synchronize()
-            # the calls (V = X A, then the GEMV) captured in one CUDA graph so the
-            # device never waits for the host between launches
-            iters = 60
-            tm = q.KernelTimer(q.KERNEL_GEMV, iters)
-            graph = torch.cuda.CUDAGraph()
-            side = torch.cuda.Stream()
-            side.wait_stream(torch.cuda.current_stream())
-            with torch.cuda.stream(side):
-                with torch.cuda.graph(graph, stream=side, capture_error_mode="relaxed"):
-                    for i in range(iters):
-                        q.qlora_linear_fwd(wts[i % reps], X, A, B, ws, Y=Y, V=V)
-            torch.cuda.current_stream().wait_stream(side)
-            tm.disarm()
-            graph.replay()
-            torch.cuda.synchronize()
-            t = statistics.median(tm.times_ms())
-            del graph
+            t = graph_timed(lambda i: q.qlora_linear_fwd(wts[i % reps], X, A, B, ws, Y=Y, V=V), q.KERNEL_GEMV, 60)
             b = n_in * n_out * (0.5 + 1 / 64) + 4 * math.ceil(n_in * n_out / 16384) + 2 * r * (n_in + n_out) \
                 + 2 * M * (n_in + n_out) + 2 * M * r
             out[f"{n_in}x{n_out}_m{M}"] = {"us": t * 1e3, "gbs": b / t / 1e6, "frac_hbm": b / t / 1e6 / pk["hbm_gbs"]}

@@ -12,8 +12,10 @@
 //     8-wide B operand.  A lane (g, t) loads one 32-bit word (8 codes) from each
 //     of the rows k0+2t, k0+2t+1, k0+2t+8, k0+2t+9 of its panel; byte j of the
 //     words fills tile j (output columns 8g+2j, 8g+2j+1).  A 256-entry table in
-//     shared memory maps a code byte to the bf16 pair of its two levels, and one
-//     byte-permute pairs two rows into an A register.
+//     shared memory maps a code byte to the bf16 pair of its two levels (one copy
+//     per lane, so lookups never conflict), and one byte-permute pairs two rows
+//     into an A register.  Each warp issues the code loads of up to 8 of its
+//     steps before the shared-memory set-up, and keeps 8 steps in flight after.
 //   * The block scale is folded into the activations: sum_k x_k (a'_k l_k) =
 //     sum_k (x_k a'_k) l_k.  Per CTA, x'[m][k] = bf16(x[m][k] * a'(k, panel)) is
 //     computed once into shared memory (M/64 multiplies per weight instead of
@@ -31,6 +33,8 @@ namespace {
 constexpr int kGvThreads = 256;
 constexpr int kGvWarps = 8;
 constexpr int kPanel = 64;
+constexpr int kDepth = 8;                       // code-load steps in flight per warp
+constexpr int kLutBytes = 256 * 32 * 4;         // 32 copies of the 256-entry table
 
 struct GemvArgs {
   const uint8_t* codes;
@@ -62,9 +66,9 @@ template <int MT>   // token tiles of 8: 1 (M <= 8) or 2 (M <= 16)
 __global__ void __launch_bounds__(kGvThreads)
 nf4_gemv_kernel(const GemvArgs p) {
   extern __shared__ __align__(16) uint8_t smem[];
-  uint32_t* lut = reinterpret_cast<uint32_t*>(smem);                   // 256 words
-  float* ascale = reinterpret_cast<float*>(smem + 1024);               // Kc floats
-  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + 1024 + 4 * p.Kc);  // [MT*8][Kc] bf16
+  uint32_t* lut = reinterpret_cast<uint32_t*>(smem);                   // [256][32]: entry b, copy lane
+  float* ascale = reinterpret_cast<float*>(smem + kLutBytes);          // Kc floats
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + kLutBytes + 4 * p.Kc);  // [MT*8][Kc] bf16
   float* red = reinterpret_cast<float*>(xs);                           // [8][MT*8][64] after the loop
   __shared__ int last;
 
@@ -76,8 +80,32 @@ nf4_gemv_kernel(const GemvArgs p) {
   const int64_t blocks_per_row = p.N / kPanel;
   constexpr int TM = MT * 8;
 
-  // level pairs of every code byte
-  lut[tid] = pack_bf16x2(nf4_level(tid & 15), nf4_level(tid >> 4));
+  const int nsteps = rows / 16;
+  const uint8_t* cbase = p.codes + (k_begin * p.N + static_cast<int64_t>(panel) * kPanel) / 2 + 4 * g;
+  const int64_t row_bytes = p.N / 2;
+  const int r0 = 2 * t, r1 = 2 * t + 1, r2 = 2 * t + 8, r3 = 2 * t + 9;
+  // this warp's steps are warp, warp + 8, ...; the codes of the first kDepth of
+  // them are requested before anything else
+  uint32_t wq[kDepth][4];
+#pragma unroll
+  for (int i = 0; i < kDepth; ++i) {
+    const int st = warp + i * kGvWarps;
+    if (st < nsteps) {
+      const uint8_t* c = cbase + static_cast<int64_t>(st * 16) * row_bytes;
+      wq[i][0] = __ldcs(reinterpret_cast<const unsigned int*>(c + r0 * row_bytes));
+      wq[i][1] = __ldcs(reinterpret_cast<const unsigned int*>(c + r1 * row_bytes));
+      wq[i][2] = __ldcs(reinterpret_cast<const unsigned int*>(c + r2 * row_bytes));
+      wq[i][3] = __ldcs(reinterpret_cast<const unsigned int*>(c + r3 * row_bytes));
+    }
+  }
+
+  // level pairs of every code byte, one copy per lane
+  {
+    const uint32_t v = pack_bf16x2(nf4_level(tid & 15), nf4_level(tid >> 4));
+    uint4* dst = reinterpret_cast<uint4*>(lut + tid * 32);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dst[i] = make_uint4(v, v, v, v);
+  }
   // absmax' of this panel's block in each row of the range
   for (int kk = tid; kk < rows; kk += kGvThreads) {
     const int64_t b = (k_begin + kk) * blocks_per_row + panel;
@@ -104,29 +132,22 @@ nf4_gemv_kernel(const GemvArgs p) {
 #pragma unroll
       for (int c = 0; c < 4; ++c) acc[a][j][c] = 0.0f;
 
-  const int nsteps = rows / 16;
-  const uint8_t* cbase = p.codes + (k_begin * p.N + static_cast<int64_t>(panel) * kPanel) / 2 + 4 * g;
-  const int64_t row_bytes = p.N / 2;
-  const int r0 = 2 * t, r1 = 2 * t + 1, r2 = 2 * t + 8, r3 = 2 * t + 9;
-
-  int st = warp;
-  uint32_t w0 = 0, w1 = 0, w2 = 0, w3 = 0;
-  if (st < nsteps) {
-    const uint8_t* c = cbase + static_cast<int64_t>(st * 16) * row_bytes;
-    w0 = __ldcs(reinterpret_cast<const unsigned int*>(c + r0 * row_bytes));
-    w1 = __ldcs(reinterpret_cast<const unsigned int*>(c + r1 * row_bytes));
-    w2 = __ldcs(reinterpret_cast<const unsigned int*>(c + r2 * row_bytes));
-    w3 = __ldcs(reinterpret_cast<const unsigned int*>(c + r3 * row_bytes));
-  }
-  for (; st < nsteps; st += kGvWarps) {
-    const uint32_t c0 = w0, c1 = w1, c2 = w2, c3 = w3;
+  const uint32_t* mylut = lut + lane;
+#pragma unroll 1
+  for (int base = 0; base * kGvWarps + warp < nsteps; base += kDepth) {
+#pragma unroll
+   for (int i = 0; i < kDepth; ++i) {
+    const int st = warp + (base + i) * kGvWarps;
+    if (st >= nsteps) break;
+    const uint32_t c0 = wq[i][0], c1 = wq[i][1], c2 = wq[i][2], c3 = wq[i][3];
     const int kk0 = st * 16;
-    if (st + kGvWarps < nsteps) {
-      const uint8_t* c = cbase + static_cast<int64_t>((st + kGvWarps) * 16) * row_bytes;
-      w0 = __ldcs(reinterpret_cast<const unsigned int*>(c + r0 * row_bytes));
-      w1 = __ldcs(reinterpret_cast<const unsigned int*>(c + r1 * row_bytes));
-      w2 = __ldcs(reinterpret_cast<const unsigned int*>(c + r2 * row_bytes));
-      w3 = __ldcs(reinterpret_cast<const unsigned int*>(c + r3 * row_bytes));
+    const int nst = st + kDepth * kGvWarps;      // refill this slot kDepth steps ahead
+    if (nst < nsteps) {
+      const uint8_t* c = cbase + static_cast<int64_t>(nst * 16) * row_bytes;
+      wq[i][0] = __ldcs(reinterpret_cast<const unsigned int*>(c + r0 * row_bytes));
+      wq[i][1] = __ldcs(reinterpret_cast<const unsigned int*>(c + r1 * row_bytes));
+      wq[i][2] = __ldcs(reinterpret_cast<const unsigned int*>(c + r2 * row_bytes));
+      wq[i][3] = __ldcs(reinterpret_cast<const unsigned int*>(c + r3 * row_bytes));
     }
     uint32_t bx[MT][2];
 #pragma unroll
@@ -138,10 +159,10 @@ nf4_gemv_kernel(const GemvArgs p) {
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const uint32_t la = lut[(c0 >> (8 * j)) & 0xFFu];
-      const uint32_t lb = lut[(c1 >> (8 * j)) & 0xFFu];
-      const uint32_t lc = lut[(c2 >> (8 * j)) & 0xFFu];
-      const uint32_t ld = lut[(c3 >> (8 * j)) & 0xFFu];
+      const uint32_t la = mylut[((c0 >> (8 * j)) & 0xFFu) * 32];
+      const uint32_t lb = mylut[((c1 >> (8 * j)) & 0xFFu) * 32];
+      const uint32_t lc = mylut[((c2 >> (8 * j)) & 0xFFu) * 32];
+      const uint32_t ld = mylut[((c3 >> (8 * j)) & 0xFFu) * 32];
       const uint32_t a0 = __byte_perm(la, lb, 0x5410);   // even column, rows 2t, 2t+1
       const uint32_t a1 = __byte_perm(la, lb, 0x7632);   // odd column
       const uint32_t a2 = __byte_perm(lc, ld, 0x5410);   // even column, rows 2t+8, 2t+9
@@ -149,6 +170,7 @@ nf4_gemv_kernel(const GemvArgs p) {
 #pragma unroll
       for (int a = 0; a < MT; ++a) mma_bf16_16816(acc[a][j], a0, a1, a2, a3, bx[a][0], bx[a][1]);
     }
+   }
   }
   __syncthreads();   // x' no longer read; its space becomes the reduction buffer
 
@@ -213,7 +235,7 @@ void gemv_plan(int64_t K, int64_t N, int& S, int& Kc) {
 size_t gemv_smem_bytes(int Kc, int MT) {
   const size_t xs = static_cast<size_t>(MT) * 8 * Kc * 2;
   const size_t red = static_cast<size_t>(kGvWarps) * MT * 8 * kPanel * 4;
-  return 1024 + 4 * static_cast<size_t>(Kc) + std::max(xs, red);
+  return kLutBytes + 4 * static_cast<size_t>(Kc) + std::max(xs, red);
 }
 
 }  // namespace

@@ -7,13 +7,16 @@
 //   per group of 256 consecutive blocks:  s = fl32(max a / 448),
 //     dq_code = E4M3_RNE_satfinite(fl32(a / s))   (0 when s = 0).
 //
-// Layout: one CTA per group (16,384 weights = 64 KB of fp32), 8 warps, each warp
-// owning 32 consecutive blocks handled 8 at a time: lane l serves a quarter (16
-// consecutive weights) of block l/4, so the block absmax needs only a 2-step
-// shuffle and each lane stores its 16 codes as one 8-byte word (a warp writes
-// 256 contiguous bytes).  All 64 weights of a lane's four iterations are loaded
-// before any is used.  HBM traffic per weight: 4 B read + 0.5 B codes + 1/64 B dq
-// code + 4/16384 B scale.
+// Layout: a persistent grid, one 512-thread CTA per SM, walks the groups (16,384
+// weights = 64 KB of fp32 each).  A bulk asynchronous copy streams each group
+// into one of three 64 KB shared-memory buffers, two groups ahead of the one
+// being encoded, so HBM is read continuously with no thread involvement.  Warp w
+// owns blocks 16w .. 16w+15 of a group, 8 at a time; lane l serves a quarter (16
+// consecutive weights) of block l/4, reading its four 16-byte chunks in a
+// rotated order so that the 8 lanes of each quarter-warp hit 8 different bank
+// groups.  The block absmax needs a 2-step shuffle and each lane stores its 16
+// codes as one 8-byte word (a warp writes 256 contiguous bytes).  HBM traffic
+// per weight: 4 B read + 0.5 B codes + 1/64 B dq code + 4/16384 B scale.
 //
 // Division.  x must be the correctly rounded quotient.  The fast path multiplies
 // by the correctly rounded reciprocal of a (|q - x| <= 3 * 2^-24 for |x| <= 1)
@@ -33,12 +36,16 @@
 // all 16 with IEEE division and a direct count over the 15 thresholds.
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace qlora {
 
 namespace {
 
-constexpr int kQThreads = 256;
+constexpr int kQThreads = 512;
+constexpr int kQWarps = kQThreads / 32;
+constexpr int kQBuf = 3;                              // groups in flight
+constexpr uint32_t kGroupBytes = kGroup * kBlock * 4; // 64 KB of fp32
 constexpr int kCells = 65;
 constexpr float kRoundBase = 12582912.0f;            // 1.5 * 2^23: integers land in the low bits
 
@@ -68,14 +75,23 @@ __device__ __forceinline__ uint32_t pack4(uint32_t a, uint32_t b, uint32_t c, ui
   return a | (b << 4) | (c << 8) | (d << 12);
 }
 
-__global__ void __launch_bounds__(kQThreads, 3)
-quantize_nf4_kernel(const float* __restrict__ W0, int64_t nblocks, uint8_t* __restrict__ codes,
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+__global__ void __launch_bounds__(kQThreads, 1)
+quantize_nf4_kernel(const float* __restrict__ W0, int64_t nblocks, int64_t ngroups, uint8_t* __restrict__ codes,
                     uint8_t* __restrict__ dq_codes, float* __restrict__ dq_scales) {
+  extern __shared__ __align__(128) uint8_t qsmem[];
   __shared__ uint32_t lut[kCells];
   __shared__ float amax[kGroup];
-  __shared__ float red[kQThreads / 32];
+  __shared__ float red[8];
+  __shared__ __align__(8) uint64_t bars[kQBuf];
 
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t buf0 = sm100::smem_addr(qsmem), bar0 = sm100::smem_addr(bars);
   if (tid < kCells) {
     const float lo = -1.0f + (tid - 0.5f) * (1.0f / 32.0f);
     const float hi = lo + (1.0f / 32.0f);
@@ -89,84 +105,121 @@ quantize_nf4_kernel(const float* __restrict__ W0, int64_t nblocks, uint8_t* __re
     }
     lut[tid] = (__float_as_uint(thr) & ~0xFu) | base;
   }
-
-  const int64_t g = blockIdx.x;
-  const int64_t blk0 = g * kGroup;
-  const int nblk = static_cast<int>(nblocks - blk0 < kGroup ? nblocks - blk0 : kGroup);
-  const int warp = tid >> 5, lane = tid & 31;
-  const int quarter = lane & 3;           // which 16 weights of the block
-  __syncthreads();                         // cell table ready
-
-#pragma unroll 1
-  for (int half = 0; half < 2; ++half) {
-    float4 v[2][4];
-#pragma unroll
-    for (int it = 0; it < 2; ++it) {
-      const int lb = warp * 32 + (2 * half + it) * 8 + (lane >> 2);
-      const float4* src = reinterpret_cast<const float4*>(W0 + (blk0 + lb) * kBlock + quarter * 16);
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        v[it][i] = (lb < nblk) ? __ldcs(src + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+  if (tid == 0) {
+    for (int b = 0; b < kQBuf; ++b) sm100::mbar_init(bar0 + 8 * b, 1);
+    sm100::fence_mbar_init();
+    for (int b = 0; b < kQBuf; ++b) {
+      const int64_t g = blockIdx.x + static_cast<int64_t>(b) * gridDim.x;
+      if (g >= ngroups) break;
+      const int64_t nb = min(static_cast<int64_t>(kGroup), nblocks - g * kGroup);
+      const uint32_t bytes = static_cast<uint32_t>(nb * kBlock * 4);
+      sm100::mbar_arrive_expect_tx(bar0 + 8 * b, bytes);
+      bulk_load(buf0 + b * kGroupBytes, W0 + g * kGroup * kBlock, bytes, bar0 + 8 * b);
     }
+  }
+  __syncthreads();
+
+  const int quarter = lane & 3;            // which 16 weights of its block
+  const int bsub = lane >> 2;              // block among the 8 of an iteration
+  // rotated chunk order: the 8 lanes of a quarter-warp read 8 different 16-byte bank groups
+  const int rot = (quarter >> 1) + 2 * (bsub & 1);
+  int64_t i = 0, failed_at = -1;
+  for (int64_t g = blockIdx.x; g < ngroups; g += gridDim.x, ++i) {
+    const int b = static_cast<int>(i % kQBuf);
+    const uint32_t ph = static_cast<uint32_t>((i / kQBuf) & 1);
+    const bool got = sm100::mbar_wait(bar0 + 8 * b, ph, nullptr, 0);
+    if (!__syncthreads_and(got)) {
+      failed_at = i;
+      break;
+    }
+    const int64_t blk0 = g * kGroup;
+    const int nblk = static_cast<int>(nblocks - blk0 < kGroup ? nblocks - blk0 : kGroup);
+    const float* gs = reinterpret_cast<const float*>(qsmem + b * kGroupBytes);
+
 #pragma unroll
     for (int it = 0; it < 2; ++it) {
-      const int lb = warp * 32 + (2 * half + it) * 8 + (lane >> 2);
+      const int lb = warp * 16 + it * 8 + bsub;
+      float4 v[4];
+      int ci[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        ci[c] = (c + rot) & 3;
+        v[c] = (lb < nblk) ? *reinterpret_cast<const float4*>(gs + lb * kBlock + quarter * 16 + 4 * ci[c])
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
       float m = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        m = fmaxf(m, fmaxf(fmaxf(fabsf(v[it][i].x), fabsf(v[it][i].y)), fmaxf(fabsf(v[it][i].z), fabsf(v[it][i].w))));
+      for (int c = 0; c < 4; ++c)
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(v[c].x), fabsf(v[c].y)), fmaxf(fabsf(v[c].z), fabsf(v[c].w))));
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
       if (lb < nblk) {
         float rcp = (m > 0.0f) ? __frcp_rn(m) : 0.0f;
         bool near = !(rcp <= 3.0e38f);     // a subnormal absmax: exact path only
         if (near) rcp = 0.0f;
-        uint32_t c[16];
+        uint32_t c4[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          c[4 * i + 0] = fast_code(__fmul_rn(v[it][i].x, rcp), lut, near);
-          c[4 * i + 1] = fast_code(__fmul_rn(v[it][i].y, rcp), lut, near);
-          c[4 * i + 2] = fast_code(__fmul_rn(v[it][i].z, rcp), lut, near);
-          c[4 * i + 3] = fast_code(__fmul_rn(v[it][i].w, rcp), lut, near);
-        }
+        for (int c = 0; c < 4; ++c)
+          c4[c] = pack4(fast_code(__fmul_rn(v[c].x, rcp), lut, near), fast_code(__fmul_rn(v[c].y, rcp), lut, near),
+                        fast_code(__fmul_rn(v[c].z, rcp), lut, near), fast_code(__fmul_rn(v[c].w, rcp), lut, near));
         if (near) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            c[4 * i + 0] = exact_code(v[it][i].x, m);
-            c[4 * i + 1] = exact_code(v[it][i].y, m);
-            c[4 * i + 2] = exact_code(v[it][i].z, m);
-            c[4 * i + 3] = exact_code(v[it][i].w, m);
-          }
+          for (int c = 0; c < 4; ++c)
+            c4[c] = pack4(exact_code(v[c].x, m), exact_code(v[c].y, m), exact_code(v[c].z, m), exact_code(v[c].w, m));
         }
-        const uint32_t lo = pack4(c[0], c[1], c[2], c[3]) | (pack4(c[4], c[5], c[6], c[7]) << 16);
-        const uint32_t hi = pack4(c[8], c[9], c[10], c[11]) | (pack4(c[12], c[13], c[14], c[15]) << 16);
-        *reinterpret_cast<uint2*>(codes + (blk0 + lb) * (kBlock / 2) + quarter * 8) = make_uint2(lo, hi);
+        uint64_t word = 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) word |= static_cast<uint64_t>(c4[c]) << (16 * ci[c]);
+        *reinterpret_cast<uint2*>(codes + (blk0 + lb) * (kBlock / 2) + quarter * 8) =
+            make_uint2(static_cast<uint32_t>(word), static_cast<uint32_t>(word >> 32));
         if (quarter == 0) amax[lb] = m;
       }
     }
-  }
-  __syncthreads();
-
-  // Group maximum of the block absmax values.
-  float gm = (tid < nblk) ? amax[tid] : 0.0f;
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
-  if (lane == 0) red[warp] = gm;
-  __syncthreads();
-  gm = red[0];
-#pragma unroll
-  for (int w = 1; w < kQThreads / 32; ++w) gm = fmaxf(gm, red[w]);
-
-  const float s = __fdiv_rn(gm, 448.0f);
-  if (tid < nblk) {
-    uint8_t c = 0;
-    if (s > 0.0f) {
-      const float y = __fdiv_rn(amax[tid], s);
-      c = static_cast<uint8_t>(__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3));
+    __syncthreads();   // buffer b fully read; absmax of the group in shared memory
+    if (tid == 0) {
+      const int64_t gn = g + static_cast<int64_t>(kQBuf) * gridDim.x;
+      if (gn < ngroups) {
+        const int64_t nb = min(static_cast<int64_t>(kGroup), nblocks - gn * kGroup);
+        const uint32_t bytes = static_cast<uint32_t>(nb * kBlock * 4);
+        sm100::mbar_arrive_expect_tx(bar0 + 8 * b, bytes);
+        bulk_load(buf0 + b * kGroupBytes, W0 + gn * kGroup * kBlock, bytes, bar0 + 8 * b);
+      }
     }
-    dq_codes[blk0 + tid] = c;
+
+    // Group maximum of the block absmax values (threads 0..255).
+    if (tid < kGroup) {
+      float gm = (tid < nblk) ? amax[tid] : 0.0f;
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
+      if (lane == 0) red[warp] = gm;
+    }
+    __syncthreads();
+    if (tid < kGroup) {
+      float gm = red[0];
+#pragma unroll
+      for (int w = 1; w < 8; ++w) gm = fmaxf(gm, red[w]);
+      const float sc = __fdiv_rn(gm, 448.0f);
+      if (tid < nblk) {
+        uint8_t c = 0;
+        if (sc > 0.0f) {
+          const float y = __fdiv_rn(amax[tid], sc);
+          c = static_cast<uint8_t>(__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3));
+        }
+        dq_codes[blk0 + tid] = c;
+      }
+      if (tid == 0) dq_scales[g] = sc;
+    }
+    __syncthreads();   // amax and red reused by the next group
   }
-  if (tid == 0) dq_scales[g] = s;
+  // A wait that gave up leaves up to kQBuf copies in flight into this CTA's
+  // shared memory: wait for them (again bounded) before the CTA exits.
+  if (failed_at >= 0 && tid == 0) {
+    for (int64_t j = failed_at; j < failed_at + kQBuf; ++j) {
+      if (blockIdx.x + j * gridDim.x >= ngroups) break;
+      sm100::mbar_wait(bar0 + 8 * static_cast<int>(j % kQBuf), static_cast<uint32_t>((j / kQBuf) & 1), nullptr, 0);
+    }
+  }
+  __syncthreads();
 }
 
 }  // namespace
@@ -176,9 +229,21 @@ cudaError_t launch_quantize_nf4(const float* W0, int64_t n, uint8_t* codes, uint
   const int64_t nblocks = n / kBlock;
   const int64_t ngroups = (nblocks + kGroup - 1) / kGroup;
   if (ngroups == 0) return cudaSuccess;
+  static bool set[64] = {};
+  static int sms[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(quantize_nf4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kQBuf * kGroupBytes));
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    set[dev] = true;
+  }
+  const int64_t grid = std::min<int64_t>(ngroups, dev < 64 ? sms[dev] : 148);
   timing_before(QLORA_KERNEL_QUANTIZE, stream);
-  quantize_nf4_kernel<<<static_cast<unsigned>(ngroups), kQThreads, 0, stream>>>(
-      W0, nblocks, codes, dq_codes, dq_scales);
+  quantize_nf4_kernel<<<static_cast<unsigned>(grid), kQThreads, kQBuf * kGroupBytes, stream>>>(
+      W0, nblocks, ngroups, codes, dq_codes, dq_scales);
   timing_after(QLORA_KERNEL_QUANTIZE, stream);
   count_launch();
   return cudaGetLastError();
