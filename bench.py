@@ -358,14 +358,15 @@ def arm_ours(args, world, rank, local):
     achieved = sum(gemm_flops) / (sum(gemm_ms) / 1e3) / 1e12
     timed_s = ms / 1e3
     peak = pk["bf16_tflops"] if timed_s < 2.0 else pk["bf16_tflops_sustained"]
-    traffic = None
-    tp = os.path.join(ROOT, "profiles", "traffic.json")
+    traffic = None   # DRAM bytes per launch from the last ncu capture, if gemm.cu is unchanged since
+    tp = os.path.join(ROOT, "profiles", "traffic.txt")
     if os.path.exists(tp):
         with open(tp) as f:
-            tr = json.load(f)
-        e = tr.get(args.workload, {}).get("fwd_gemm")
-        if e and e.get("src") == src_hash("gemm.cu"):
-            traffic = e["bytes_per_launch"]
+            for line in f:
+                fields = line.split("#", 1)[0].split()
+                if len(fields) == 4 and fields[0] == args.workload and fields[1] == "fwd_gemm" \
+                        and fields[3] == src_hash("gemm.cu"):
+                    traffic = int(fields[2])
 
     line = {
         "metric": "QLoRA linear fwd+bwd tokens/s",
