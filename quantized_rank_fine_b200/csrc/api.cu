@@ -287,7 +287,7 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int6
   QLORA_CUDA(qlora::launch_xa(X, A, M, w->in, r, V, part, tickets, status, s));
   if (M <= kGemvMaxM && w->out / 64 <= kTicketWords) {
     float* gpart = reinterpret_cast<float*>(base + L.gemv_off);
-    QLORA_CUDA(qlora::launch_gemv(wv, X, V, B, M, r, Y, gpart, tickets, s));
+    QLORA_CUDA(qlora::launch_gemv(wv, X, V, B, M, r, Y, gpart, tickets, status, s));
   } else {
     QLORA_CUDA(qlora::launch_fwd_gemm(wv, X, V, B, M, r, Y, status, s));
   }

@@ -41,6 +41,18 @@ __host__ __device__ constexpr float nf4_threshold(int j) {
   return kThr[j];
 }
 
+// Copies of the two tables for run-time indices in device code: indexing the
+// constexpr arrays above with a run-time value makes every thread build its own
+// copy in local memory.
+static __constant__ float c_nf4_level[16] = {
+    nf4_level(0), nf4_level(1), nf4_level(2),  nf4_level(3),  nf4_level(4),  nf4_level(5),
+    nf4_level(6), nf4_level(7), nf4_level(8),  nf4_level(9),  nf4_level(10), nf4_level(11),
+    nf4_level(12), nf4_level(13), nf4_level(14), nf4_level(15)};
+static __constant__ float c_nf4_threshold[15] = {
+    nf4_threshold(0), nf4_threshold(1), nf4_threshold(2),  nf4_threshold(3),  nf4_threshold(4),
+    nf4_threshold(5), nf4_threshold(6), nf4_threshold(7),  nf4_threshold(8),  nf4_threshold(9),
+    nf4_threshold(10), nf4_threshold(11), nf4_threshold(12), nf4_threshold(13), nf4_threshold(14)};
+
 // ---------------------------------------------------------------- numerics
 
 // IEEE binary32 product with no contraction into an FMA.

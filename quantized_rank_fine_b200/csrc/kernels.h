@@ -57,7 +57,7 @@ cudaError_t launch_vtdy(const uint16_t* V, const uint16_t* dY, int64_t M, int64_
 // and end at 0.
 size_t gemv_workspace_bytes(int64_t M, int64_t K, int64_t N);
 cudaError_t launch_gemv(const WeightView& w, const uint16_t* X, const uint16_t* V, const uint16_t* B, int64_t M,
-                        int r, uint16_t* Y, float* part, uint32_t* tickets, cudaStream_t stream);
+                        int r, uint16_t* Y, float* part, uint32_t* tickets, uint32_t* status, cudaStream_t stream);
 
 // Fused dequant GEMMs (tcgen05); `status` is the workspace status word.
 cudaError_t launch_fwd_gemm(const WeightView& w, const uint16_t* X, const uint16_t* V, const uint16_t* B,
