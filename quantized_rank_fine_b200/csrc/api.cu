@@ -88,11 +88,9 @@ WeightView view(const qlora_nf4_weight* w) { return WeightView{w->codes, w->dq_c
 
 // Workspace layout (byte offsets), shared by the size query and the calls.
 struct WsLayout {
-  size_t v_off, u_off, part_off, gemv_off, total;
+  size_t v_off, u_off, part_off, total;
 };
 
-constexpr int64_t kGemvMaxM = 16;     // token counts served by the dequant-GEMV
-constexpr int64_t kTicketWords = static_cast<int64_t>(qlora::kWsTicketWords);
 // Every layout reserves the tickets right after the status words, so no call
 // ever writes that region except the split-K kernels, which leave it zero.
 constexpr size_t kTicketOff = qlora::kWsStatusBytes;
@@ -108,10 +106,6 @@ WsLayout ws_layout(int op, int64_t M, int64_t in, int64_t out, int r) {
   if (op == QLORA_OP_FWD) {
     L.u_off = 0;
     parts = qlora::skinny_partial_floats(M, r, in);
-    if (M <= kGemvMaxM && out / 64 <= kTicketWords) {
-      L.gemv_off = off;
-      off += align256(qlora::gemv_workspace_bytes(M, in, out));
-    }
   } else {
     L.u_off = off;
     off += mr;
@@ -284,11 +278,11 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int6
   float* part = reinterpret_cast<float*>(base + L.part_off);
   const WeightView wv = view(w);
   uint32_t* tickets = reinterpret_cast<uint32_t*>(base + kTicketOff);
-  QLORA_CUDA(qlora::launch_xa(X, A, M, w->in, r, V, part, tickets, status, s));
-  if (M <= kGemvMaxM && w->out / 64 <= kTicketWords) {
-    float* gpart = reinterpret_cast<float*>(base + L.gemv_off);
-    QLORA_CUDA(qlora::launch_gemv(wv, X, V, B, M, r, Y, gpart, tickets, status, s));
+  if (qlora::gemv_supported(M, w->in, w->out)) {
+    QLORA_CUDA(qlora::launch_xa_small(X, A, M, w->in, r, V, s));
+    QLORA_CUDA(qlora::launch_gemv(wv, X, V, B, M, r, Y, status, s));
   } else {
+    QLORA_CUDA(qlora::launch_xa(X, A, M, w->in, r, V, part, tickets, status, s));
     QLORA_CUDA(qlora::launch_fwd_gemm(wv, X, V, B, M, r, Y, status, s));
   }
   return QLORA_OK;

@@ -52,12 +52,17 @@ cudaError_t launch_xtu(const uint16_t* X, const uint16_t* U, int64_t M, int64_t 
 cudaError_t launch_vtdy(const uint16_t* V, const uint16_t* dY, int64_t M, int64_t n_out, int r,
                         float* dB, float* part, uint32_t* tickets, uint32_t* status, cudaStream_t stream);
 
-// Small-M forward (M <= 16): base + adapter, split-K with a last-CTA finalize.
-// `part` holds gemv_workspace_bytes(...) bytes; `tickets` (N / 64 words) start
-// and end at 0.
-size_t gemv_workspace_bytes(int64_t M, int64_t K, int64_t N);
+// Small-M forward (M <= kGemvMaxTokens): base + adapter in one kernel, the
+// K-splits of a column tile reduced inside a thread-block cluster; no workspace.
+// Launched as a programmatic dependent of the kernel before it (which writes V).
+constexpr int64_t kGemvMaxTokens = 16;
+bool gemv_supported(int64_t M, int64_t K, int64_t N);
+// V = X A for M <= kGemvMaxTokens on CUDA cores (K split over a cluster); lets
+// the small-M forward launched after it start early.
+cudaError_t launch_xa_small(const uint16_t* X, const uint16_t* A, int64_t M, int64_t K, int r, uint16_t* V,
+                            cudaStream_t stream);
 cudaError_t launch_gemv(const WeightView& w, const uint16_t* X, const uint16_t* V, const uint16_t* B, int64_t M,
-                        int r, uint16_t* Y, float* part, uint32_t* tickets, uint32_t* status, cudaStream_t stream);
+                        int r, uint16_t* Y, uint32_t* status, cudaStream_t stream);
 
 // Fused dequant GEMMs (tcgen05); `status` is the workspace status word.
 cudaError_t launch_fwd_gemm(const WeightView& w, const uint16_t* X, const uint16_t* V, const uint16_t* B,

@@ -87,6 +87,10 @@ skinny_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
   const int64_t kend = min(p.k_total, kbeg + p.k_per_split);
   const int nkb = kend > kbeg ? static_cast<int>((kend - kbeg + kKT - 1) / kKT) : 0;
 
+  // A kernel launched after this one as a programmatic dependent (the small-M
+  // forward) may start now; it waits for this grid to finish before it reads
+  // this grid's output.
+  grid_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSkStages; ++s) {
       mbar_init(full0 + 8 * s, 1);

@@ -121,6 +121,48 @@ def test_linear_small_m_forward(M, n_in, n_out):
     assert_close(V, Vr, "V")
 
 
+@pytest.mark.parametrize("M,n_in,n_out,r", [
+    (1, 64, 64, 8), (3, 192, 320, 16), (8, 128, 256, 8), (9, 1024, 704, 24),
+    (16, 8192, 512, 256), (13, 11008, 1088, 8), (2, 4096, 11072, 16), (5, 2048, 256, 72),
+    (12, 64, 192, 40),
+])
+def test_small_m_forward_shapes(M, n_in, n_out, r):
+    """Small-M forward on ragged shapes: a partial last column tile, one to
+    sixteen K-splits, both token-tile counts, the largest adapter rank."""
+    t, w = layer_on_gpu(n_in, n_out, M, r, tag="gemv-ragged")
+    ws = q.Workspace()
+    Y, V = q.qlora_linear_fwd(w, t["X"], t["A"], t["B"], ws)
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+    Yr, Vr = linear.forward(t["X"], t["A"], t["B"], oracle_weight(w))
+    assert_close(Y, Yr, "Y")
+    assert_close(V, Vr, "V")
+
+
+def test_small_m_forward_deterministic_and_graph():
+    """The small-M forward is deterministic (fixed reduction order), also when
+    captured in a CUDA graph together with the kernel that produces V."""
+    t, w = layer_on_gpu(4096, 4096, 4, 16, tag="gemv-graph")
+    ws = q.Workspace()
+    Y1, V1 = q.qlora_linear_fwd(w, t["X"], t["A"], t["B"], ws)
+    Y2, V2 = q.qlora_linear_fwd(w, t["X"], t["A"], t["B"], ws)
+    Yg = torch.empty_like(Y1)
+    Vg = torch.empty_like(V1)
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            q.qlora_linear_fwd(w, t["X"], t["A"], t["B"], ws, Y=Yg, V=Vg)
+    torch.cuda.current_stream().wait_stream(side)
+    Yg.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(Y1, Y2) and torch.equal(V1, V2)
+    assert torch.equal(Yg, Y1) and torch.equal(Vg, V1)
+    del graph
+
+
 def test_linear_stack_layer_sample():
     """Llama-7B-shaped stack, M = 2048, r = 16: one layer's seven projections
     (q, k, v, o, gate, up, down), sampled rows for Y, V, dX, full dA, dB."""
