@@ -281,13 +281,16 @@ def graph_timed(fn, which, iters):
 
 def time_gemv(pk):
     """Small-M forward (M = 1, 4, 16) on the 4096 x 4096 and 4096 x 11008 shapes,
-    r = 16: the dequant-GEMV kernel's HBM bandwidth.  Algorithmic bytes: codes,
-    absmax codes and scales, A and B, X, V and Y."""
+    r = 16, through qlora_linear_fwd: device time per call of a CUDA graph of
+    back-to-back calls (the X A kernel and the dequant-GEMV, which overlap through
+    programmatic dependent launch), weights rotated over sets larger than L2.
+    Algorithmic bytes: codes, absmax codes and scales, A and B, X, V and Y."""
     import torch
     import quantized_rank_fine_b200 as q
     import synth
     out = {}
     r = 16
+    iters = 60
     for n_in, n_out in ((4096, 4096), (4096, 11008)):
         wbytes = n_in * n_out * (0.5 + 1 / 64)
         reps = max(3, math.ceil(3 * L2_BYTES / wbytes))
@@ -299,10 +302,35 @@ def time_gemv(pk):
             Y = torch.empty((M, n_out), dtype=torch.bfloat16, device="cuda")
             V = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
             ws = q.Workspace()
-            t = graph_timed(lambda i: q.qlora_linear_fwd(wts[i % reps], X, A, B, ws, Y=Y, V=V), q.KERNEL_GEMV, 60)
+            for i in range(3):
+                q.qlora_linear_fwd(wts[i % reps], X, A, B, ws, Y=Y, V=V)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                with torch.cuda.graph(graph, stream=side):
+                    for i in range(iters):
+                        q.qlora_linear_fwd(wts[i % reps], X, A, B, ws, Y=Y, V=V)
+            torch.cuda.current_stream().wait_stream(side)
+            graph.replay()
+            torch.cuda.synchronize()
+            times = []
+            for _ in range(5):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                graph.replay()
+                e1.record()
+                torch.cuda.synchronize()
+                times.append(e0.elapsed_time(e1) / iters)
+            t = statistics.median(times)
+            del graph
+            if ws.status() != 0:
+                raise RuntimeError("a kernel wait timed out in the small-M forward")
             b = n_in * n_out * (0.5 + 1 / 64) + 4 * math.ceil(n_in * n_out / 16384) + 2 * r * (n_in + n_out) \
                 + 2 * M * (n_in + n_out) + 2 * M * r
-            out[f"{n_in}x{n_out}_m{M}"] = {"us": t * 1e3, "gbs": b / t / 1e6, "frac_hbm": b / t / 1e6 / pk["hbm_gbs"]}
+            out[f"{n_in}x{n_out}_m{M}"] = {"us_per_forward": t * 1e3, "gbs": b / t / 1e6,
+                                           "frac_hbm": b / t / 1e6 / pk["hbm_gbs"], "launches": 2}
         del wts
         torch.cuda.synchronize()
     return out

@@ -214,12 +214,18 @@ skinny_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
     const int rr = e / pairs, cc = 2 * (e - rr * pairs);
     const int64_t row = row0 + rr;
     if (row >= p.rows) continue;
+    // every split's partial is requested before any is added (one round trip)
+    float2 x[kMaxSplits];
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplits; ++sp)
+      x[sp] = sp < p.splits ? __ldcg(reinterpret_cast<const float2*>(
+                                  p.part + (static_cast<int64_t>(sp) * p.rows + row) * p.r + col0 + cc))
+                            : make_float2(0.0f, 0.0f);
     float v0 = 0.0f, v1 = 0.0f;
-    for (int sp = 0; sp < p.splits; ++sp) {
-      const float2 x =
-          __ldcg(reinterpret_cast<const float2*>(p.part + (static_cast<int64_t>(sp) * p.rows + row) * p.r + col0 + cc));
-      v0 += x.x;
-      v1 += x.y;
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplits; ++sp) {
+      v0 += x[sp].x;
+      v1 += x[sp].y;
     }
     store_pair(p, row, col0 + cc, v0, v1);
   }
