@@ -198,9 +198,10 @@ QLORA_API qlora_status qlora_merge(const qlora_nf4_weight* w, const uint16_t* A,
  * (0 for an unknown op or invalid sizes).  Host only, no device access. */
 QLORA_API size_t qlora_workspace_bytes(int op, int64_t M, int64_t in, int64_t out, int r);
 
-/* Zero the whole workspace (once, before its first use).  The calls keep the
- * workspace's bookkeeping words at zero between calls; calls that share one
- * workspace must be ordered on one stream. */
+/* Zero the whole workspace (once, before its first use).  Its first 256 bytes
+ * hold a status word that the kernels set when a bounded wait gives up and
+ * qlora_ws_status() clears; the rest is scratch (V, U) that every call rewrites.
+ * Calls that share one workspace must be ordered on one stream. */
 QLORA_API qlora_status qlora_ws_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronise `stream`, then report QLORA_ERR_TIMEOUT if a bounded wait in a

@@ -86,34 +86,28 @@ qlora_status check_weight(const qlora_nf4_weight* w) {
 
 WeightView view(const qlora_nf4_weight* w) { return WeightView{w->codes, w->dq_codes, w->dq_scales, w->in, w->out}; }
 
-// Workspace layout (byte offsets), shared by the size query and the calls.
+// Workspace layout (byte offsets), shared by the size query and the calls:
+// the status prefix, V (when the caller does not keep it) and U (backward).
 struct WsLayout {
-  size_t v_off, u_off, part_off, total;
+  size_t v_off, u_off, total;
 };
 
-// Every layout reserves the tickets right after the status words, so no call
-// ever writes that region except the split-K kernels, which leave it zero.
-constexpr size_t kTicketOff = qlora::kWsStatusBytes;
 constexpr size_t kFixedBytes = qlora::kWsFixedBytes;
 
 WsLayout ws_layout(int op, int64_t M, int64_t in, int64_t out, int r) {
+  (void)in;
+  (void)out;
   WsLayout L{};
   const size_t mr = align256(static_cast<size_t>(M) * r * 2);
   size_t off = kFixedBytes;
   L.v_off = off;
   off += mr;
-  size_t parts = 0;
   if (op == QLORA_OP_FWD) {
     L.u_off = 0;
-    parts = qlora::skinny_partial_floats(M, r, in);
   } else {
     L.u_off = off;
     off += mr;
-    parts = std::max({qlora::skinny_partial_floats(M, r, in), qlora::skinny_partial_floats(M, r, out),
-                      qlora::skinny_partial_floats(in, r, M), qlora::skinny_partial_floats(out, r, M)});
   }
-  L.part_off = off;
-  off += align256(parts * 4);
   L.total = off;
   return L;
 }
@@ -275,14 +269,12 @@ qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int6
   uint8_t* base = static_cast<uint8_t*>(ws);
   uint32_t* status = reinterpret_cast<uint32_t*>(base);
   uint16_t* V = V_save ? V_save : reinterpret_cast<uint16_t*>(base + L.v_off);
-  float* part = reinterpret_cast<float*>(base + L.part_off);
   const WeightView wv = view(w);
-  uint32_t* tickets = reinterpret_cast<uint32_t*>(base + kTicketOff);
   if (qlora::gemv_supported(M, w->in, w->out)) {
     QLORA_CUDA(qlora::launch_xa_small(X, A, M, w->in, r, V, s));
     QLORA_CUDA(qlora::launch_gemv(wv, X, V, B, M, r, Y, status, s));
   } else {
-    QLORA_CUDA(qlora::launch_xa(X, A, M, w->in, r, V, part, tickets, status, s));
+    QLORA_CUDA(qlora::launch_xa(X, A, M, w->in, r, V, status, s));
     QLORA_CUDA(qlora::launch_fwd_gemm(wv, X, V, B, M, r, Y, status, s));
   }
   return QLORA_OK;
@@ -312,17 +304,15 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16_t* X, cons
   uint8_t* base = static_cast<uint8_t*>(ws);
   uint32_t* status = reinterpret_cast<uint32_t*>(base);
   uint16_t* U = reinterpret_cast<uint16_t*>(base + L.u_off);
-  float* part = reinterpret_cast<float*>(base + L.part_off);
   const WeightView wv = view(w);
-  uint32_t* tickets = reinterpret_cast<uint32_t*>(base + kTicketOff);
   if (!V) {
     uint16_t* Vw = reinterpret_cast<uint16_t*>(base + L.v_off);
-    QLORA_CUDA(qlora::launch_xa(X, A, M, w->in, r, Vw, part, tickets, status, s));
+    QLORA_CUDA(qlora::launch_xa(X, A, M, w->in, r, Vw, status, s));
     V = Vw;
   }
-  QLORA_CUDA(qlora::launch_dybt(dY, B, M, w->out, r, U, part, tickets, status, s));
-  QLORA_CUDA(qlora::launch_vtdy(V, dY, M, w->out, r, dB, part, tickets, status, s));
-  QLORA_CUDA(qlora::launch_xtu(X, U, M, w->in, r, dA, part, tickets, status, s));
+  QLORA_CUDA(qlora::launch_dybt(dY, B, M, w->out, r, U, status, s));
+  QLORA_CUDA(qlora::launch_vtdy(V, dY, M, w->out, r, dB, status, s));
+  QLORA_CUDA(qlora::launch_xtu(X, U, M, w->in, r, dA, status, s));
   if (dX) QLORA_CUDA(qlora::launch_dx_gemm(wv, dY, U, A, M, r, dX, status, s));
   return QLORA_OK;
 }

@@ -12,11 +12,10 @@ namespace qlora {
 
 constexpr int kMaxSplits = 16;   // most K/M splits of the rank-r kernels
 
-// Workspace prefix shared by every call: the status word(s) and the split-K
-// tickets (kept at zero between launches).
+// Workspace prefix shared by every call: the status word(s), which must start
+// at zero (the only part of a workspace that needs initialising).
 constexpr size_t kWsStatusBytes = 256;
-constexpr size_t kWsTicketWords = 4096;
-constexpr size_t kWsFixedBytes = kWsStatusBytes + kWsTicketWords * 4;
+constexpr size_t kWsFixedBytes = kWsStatusBytes;
 
 // Bookkeeping of the measurement helpers (defined in api.cu): every kernel
 // launch is counted; an armed timing hook brackets launches of one kernel kind.
@@ -39,18 +38,16 @@ cudaError_t launch_merge(const uint8_t* codes, const uint8_t* dq_codes, const fl
                          const uint16_t* A, const uint16_t* B, int r, int64_t n_in, int64_t n_out,
                          bool bf16, void* out, cudaStream_t stream);
 
-// Rank-r products (tcgen05); `part` is fp32 scratch of skinny_partial_floats(...)
-// floats, `tickets` the workspace's ticket words (zero between launches, left at
-// zero), `status` the workspace status word.
-size_t skinny_partial_floats(int64_t out_rows, int r, int64_t k_total);
+// Rank-r products (tcgen05), split-K reduced inside a thread-block cluster;
+// `status` is the workspace status word.
 cudaError_t launch_xa(const uint16_t* X, const uint16_t* A, int64_t M, int64_t n_in, int r, uint16_t* V,
-                      float* part, uint32_t* tickets, uint32_t* status, cudaStream_t stream);
+                      uint32_t* status, cudaStream_t stream);
 cudaError_t launch_dybt(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t n_out, int r,
-                        uint16_t* U, float* part, uint32_t* tickets, uint32_t* status, cudaStream_t stream);
+                        uint16_t* U, uint32_t* status, cudaStream_t stream);
 cudaError_t launch_xtu(const uint16_t* X, const uint16_t* U, int64_t M, int64_t n_in, int r, float* dA,
-                       float* part, uint32_t* tickets, uint32_t* status, cudaStream_t stream);
+                       uint32_t* status, cudaStream_t stream);
 cudaError_t launch_vtdy(const uint16_t* V, const uint16_t* dY, int64_t M, int64_t n_out, int r,
-                        float* dB, float* part, uint32_t* tickets, uint32_t* status, cudaStream_t stream);
+                        float* dB, uint32_t* status, cudaStream_t stream);
 
 // Small-M forward (M <= kGemvMaxTokens): base + adapter in one kernel, the
 // K-splits of a column tile reduced inside a thread-block cluster; no workspace.

@@ -15,9 +15,9 @@
 // with cudaGetSymbolAddress, once per device, on the first call made with that
 // device current; that first call should come before any stream capture.  All
 // calls share the array and it keeps the previous call's contents, so each call
-// first zeroes the part that must start at zero (status word and split-K
-// tickets).  Two calls whose work overlaps on the GPU (different streams, or
-// different host threads) race on the array.
+// first zeroes the part that must start at zero (the status word).  Two calls
+// whose work overlaps on the GPU (different streams, or different host threads)
+// race on the array.
 #include <cuda_runtime.h>
 
 #include <mutex>

@@ -8,14 +8,14 @@
 // Each is D (rows x r) = sum_k Aop(rows, k) Bop(r, k) with r <= 64 per pass, bound
 // by streaming the big operand (X or dY) from HBM once.  A CTA owns 128 output
 // rows and one slice of the reduction: TMA brings 128 x 64 (Aop) and 64 x 64
-// (Bop) bf16 tiles into a 4-stage shared-memory ring (128-byte swizzle, K- or
+// (Bop) bf16 tiles into a 3-stage shared-memory ring (128-byte swizzle, K- or
 // MN-major as the operand sits in memory; two CTAs per SM), one thread issues
 // tcgen05.mma into a 128 x r fp32 TMEM accumulator, and four warps move the
 // result out.  The reduction is split across CTAs so that the whole grid is
-// resident at once (two per SM);
-// each split writes an fp32 partial tile to the workspace and the last CTA of a
-// tile (an atomic ticket in the workspace, left at zero afterwards) adds them in
-// split order, so the sums are deterministic and need no second launch.
+// resident at once; the splits of a row tile form one thread-block cluster.
+// Each split stores its TMEM rows straight into the shared memory of the CTA
+// that owns those rows (distributed shared memory); after one cluster barrier
+// the owners add the splits in order (deterministic, no workspace, no atomics).
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -29,23 +29,22 @@ namespace {
 using namespace sm100;
 
 constexpr int kSkThreads = 192;    // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 epilogue
-constexpr int kSkStages = 4;       // 96 KB ring: two CTAs per SM
+constexpr int kSkStages = 3;       // 72 KB ring + 36 KB receive buffer: two CTAs per SM
 constexpr int kRowsT = 128;        // output rows per CTA (UMMA M)
 constexpr int kKT = 64;            // reduction step
 constexpr int kColsT = 64;         // output columns per CTA
 constexpr uint32_t kATile = kRowsT * kKT * 2;    // 16 KB
 constexpr uint32_t kBTile = kColsT * kKT * 2;    // 8 KB
 constexpr uint32_t kSkStage = kATile + kBTile;
-constexpr uint32_t kSkSmem = kSkStages * kSkStage + 1024 + 256;
+constexpr int kRecvRows = kRowsT + kMaxSplits;   // S * ceil(128 / S) rows at most
+constexpr uint32_t kRecvBytes = kRecvRows * kColsT * 4;
+constexpr uint32_t kSkSmem = kSkStages * kSkStage + kRecvBytes + 1024 + 256;
 
 struct SkArgs {
   int64_t rows;          // output rows
   int r;                 // output columns
   int64_t k_total;       // reduction length
   int64_t k_per_split;   // multiple of 64
-  int splits;
-  float* part;           // fp32 partials [splits][rows][r] (splits > 1)
-  uint32_t* tickets;     // one per (row tile, column chunk), zero between launches
   void* out;
   int out_kind;          // 0 = bf16 [row][r], 1 = fp32 [row][r], 2 = fp32 transposed [r][row]
   uint32_t* status;
@@ -71,9 +70,9 @@ skinny_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
                  const SkArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSkStages * kSkStage);
+  float* recv = reinterpret_cast<float*>(smem + kSkStages * kSkStage);       // [S][cap][64]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSkStages * kSkStage + kRecvBytes);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kSkStages + 1);
-  __shared__ int last;
   const uint32_t full0 = smem_addr(bars), free0 = smem_addr(bars + kSkStages);
   const uint32_t tmem_full = smem_addr(bars + 2 * kSkStages);
 
@@ -86,11 +85,10 @@ skinny_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
   const int64_t kbeg = split * p.k_per_split;
   const int64_t kend = min(p.k_total, kbeg + p.k_per_split);
   const int nkb = kend > kbeg ? static_cast<int>((kend - kbeg + kKT - 1) / kKT) : 0;
+  // the splits of this row tile are the CTAs of the cluster (rank = split)
+  const int S = static_cast<int>(gridDim.y);
+  const int cap = (kRowsT + S - 1) / S;   // rows owned by each split
 
-  // A kernel launched after this one as a programmatic dependent (the small-M
-  // forward) may start now; it waits for this grid to finish before it reads
-  // this grid's output.
-  grid_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSkStages; ++s) {
       mbar_init(full0 + 8 * s, 1);
@@ -162,9 +160,15 @@ skinny_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
         __all_sync(0xffffffffu, nkb == 0 || mbar_wait(tmem_full, 0, p.status, kFlagTimeoutEpilogue));
     tc_fence_after();
     const int quarter = warp & 3;                  // TMEM lanes 32*quarter .. +31
-    const int64_t row = row0 + quarter * 32 + lane;
+    const int rl = quarter * 32 + lane;            // row within the tile
+    const int64_t row = row0 + rl;
     const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
-    float* dst_part = p.part + (static_cast<int64_t>(split) * p.rows + row) * p.r + col0;
+    // the owner of this row and this split's slot in the owner's receive buffer
+    const int owner = rl / cap;
+    const uint32_t dst =
+        S > 1 ? mapa_shared(smem_addr(recv) + static_cast<uint32_t>(((split * cap + rl - owner * cap) * kColsT) * 4),
+                            static_cast<uint32_t>(owner))
+              : 0u;
 #pragma unroll 1
     for (int c = 0; c < n_mma; c += 16) {
       uint32_t v[16];
@@ -181,14 +185,19 @@ skinny_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
 #pragma unroll
         for (int i = 0; i < 16; ++i) v[i] = 0u;   // an empty slice contributes zeros
       }
-      if (row < p.rows) {
+      if (S == 1) {
+        if (row < p.rows) {
 #pragma unroll
-        for (int i = 0; i < 16; i += 2) {
-          if (c + i >= cols) break;
-          const float v0 = __uint_as_float(v[i]), v1 = __uint_as_float(v[i + 1]);
-          if (p.splits == 1) store_pair(p, row, col0 + c + i, v0, v1);
-          else *reinterpret_cast<float2*>(dst_part + c + i) = make_float2(v0, v1);
+          for (int i = 0; i < 16; i += 2)
+            if (c + i < cols) store_pair(p, row, col0 + c + i, __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
         }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; i += 4)   // cols is a multiple of 8
+          if (c + i < cols)
+            st_shared_cluster_v4(dst + static_cast<uint32_t>((c + i) * 4),
+                                 make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                                             __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])));
       }
     }
   }
@@ -199,37 +208,24 @@ skinny_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
     tc_fence_after();
     tmem_dealloc(tmem_base, 64);
   }
-  if (p.splits == 1) return;
+  if (S == 1) return;
 
   // ------------------------------------------------------------ split reduction
-  __threadfence();
-  __syncthreads();
-  const int tile = blockIdx.x + gridDim.x * blockIdx.z;
-  if (threadIdx.x == 0) last = (atomicAdd(p.tickets + tile, 1u) == static_cast<uint32_t>(p.splits - 1));
-  __syncthreads();
-  if (!last) return;
-  __threadfence();
+  cluster_sync();   // every split's rows have landed in their owners' buffers
+  const int r_begin = split * cap, r_end = min(kRowsT, r_begin + cap);
   const int pairs = cols / 2;
-  for (int e = threadIdx.x; e < kRowsT * pairs; e += kSkThreads) {
-    const int rr = e / pairs, cc = 2 * (e - rr * pairs);
-    const int64_t row = row0 + rr;
+  for (int e = threadIdx.x; e < (r_end - r_begin) * pairs; e += kSkThreads) {
+    const int slot = e / pairs, cc = 2 * (e - slot * pairs);
+    const int64_t row = row0 + r_begin + slot;
     if (row >= p.rows) continue;
-    // every split's partial is requested before any is added (one round trip)
-    float2 x[kMaxSplits];
-#pragma unroll
-    for (int sp = 0; sp < kMaxSplits; ++sp)
-      x[sp] = sp < p.splits ? __ldcg(reinterpret_cast<const float2*>(
-                                  p.part + (static_cast<int64_t>(sp) * p.rows + row) * p.r + col0 + cc))
-                            : make_float2(0.0f, 0.0f);
     float v0 = 0.0f, v1 = 0.0f;
-#pragma unroll
-    for (int sp = 0; sp < kMaxSplits; ++sp) {
-      v0 += x[sp].x;
-      v1 += x[sp].y;
+    for (int sp = 0; sp < S; ++sp) {
+      const float2 x = *reinterpret_cast<const float2*>(recv + (sp * cap + slot) * kColsT + cc);
+      v0 += x.x;
+      v1 += x.y;
     }
     store_pair(p, row, col0 + cc, v0, v1);
   }
-  if (threadIdx.x == 0) p.tickets[tile] = 0u;
 }
 
 // ---------------------------------------------------------------- host side
@@ -284,62 +280,71 @@ Plan plan(int64_t rows, int r, int64_t k_total) {
 
 template <bool A_MN, bool B_MN>
 cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows, int r, int64_t k_total, void* out,
-                int out_kind, float* part, uint32_t* tickets, uint32_t* status, cudaStream_t stream) {
+                int out_kind, uint32_t* status, cudaStream_t stream) {
   static bool set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(skinny_tc_kernel<A_MN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(kSkSmem));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(skinny_tc_kernel<A_MN, B_MN>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
     set[dev] = true;
   }
   const Plan pl = plan(rows, r, k_total);
-  SkArgs a{rows, r, k_total, pl.kps, pl.splits, part, tickets, out, out_kind, status};
+  SkArgs a{rows, r, k_total, pl.kps, out, out_kind, status};
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = pl.grid;
+  cfg.blockDim = dim3(kSkThreads);
+  cfg.dynamicSmemBytes = kSkSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 1;
+  at[0].val.clusterDim.y = static_cast<unsigned>(pl.splits);
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
   timing_before(QLORA_KERNEL_RANK_R, stream);
-  skinny_tc_kernel<A_MN, B_MN><<<pl.grid, kSkThreads, kSkSmem, stream>>>(ta, tb, a);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, skinny_tc_kernel<A_MN, B_MN>, ta, tb, a);
   timing_after(QLORA_KERNEL_RANK_R, stream);
   count_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace
 
-size_t skinny_partial_floats(int64_t out_rows, int r, int64_t k_total) {
-  const Plan pl = plan(out_rows, r, k_total);
-  return pl.splits > 1 ? static_cast<size_t>(pl.splits) * out_rows * r : 0;
-}
-
 // V = X A: Aop = X (M x in, k contiguous); Bop[j][k] = A[k][j] (j contiguous).
 cudaError_t launch_xa(const uint16_t* X, const uint16_t* A, int64_t M, int64_t n_in, int r, uint16_t* V,
-                      float* part, uint32_t* tickets, uint32_t* status, cudaStream_t stream) {
+                      uint32_t* status, cudaStream_t stream) {
   CUtensorMap ta, tb;
   if (!bf16_map(&ta, X, M, n_in, 64, 128) || !bf16_map(&tb, A, n_in, r, 64, 64)) return cudaErrorInvalidValue;
-  return run<false, true>(ta, tb, M, r, n_in, V, 0, part, tickets, status, stream);
+  return run<false, true>(ta, tb, M, r, n_in, V, 0, status, stream);
 }
 
 // U = dY B^T: Aop = dY (M x out, k contiguous); Bop = B (r x out, k contiguous).
 cudaError_t launch_dybt(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t n_out, int r, uint16_t* U,
-                        float* part, uint32_t* tickets, uint32_t* status, cudaStream_t stream) {
+                        uint32_t* status, cudaStream_t stream) {
   CUtensorMap ta, tb;
   if (!bf16_map(&ta, dY, M, n_out, 64, 128) || !bf16_map(&tb, B, r, n_out, 64, 64)) return cudaErrorInvalidValue;
-  return run<false, false>(ta, tb, M, r, n_out, U, 0, part, tickets, status, stream);
+  return run<false, false>(ta, tb, M, r, n_out, U, 0, status, stream);
 }
 
 // dA = X^T U: Aop[i][m] = X[m][i] (i contiguous); Bop[j][m] = U[m][j] (j contiguous).
 cudaError_t launch_xtu(const uint16_t* X, const uint16_t* U, int64_t M, int64_t n_in, int r, float* dA,
-                       float* part, uint32_t* tickets, uint32_t* status, cudaStream_t stream) {
+                       uint32_t* status, cudaStream_t stream) {
   CUtensorMap ta, tb;
   if (!bf16_map(&ta, X, M, n_in, 64, 64) || !bf16_map(&tb, U, M, r, 64, 64)) return cudaErrorInvalidValue;
-  return run<true, true>(ta, tb, n_in, r, M, dA, 1, part, tickets, status, stream);
+  return run<true, true>(ta, tb, n_in, r, M, dA, 1, status, stream);
 }
 
 // dB^T = dY^T V: Aop[o][m] = dY[m][o] (o contiguous); Bop[j][m] = V[m][j]; stored as dB (r x out).
 cudaError_t launch_vtdy(const uint16_t* V, const uint16_t* dY, int64_t M, int64_t n_out, int r, float* dB,
-                        float* part, uint32_t* tickets, uint32_t* status, cudaStream_t stream) {
+                        uint32_t* status, cudaStream_t stream) {
   CUtensorMap ta, tb;
   if (!bf16_map(&ta, dY, M, n_out, 64, 64) || !bf16_map(&tb, V, M, r, 64, 64)) return cudaErrorInvalidValue;
-  return run<true, true>(ta, tb, n_out, r, M, dB, 2, part, tickets, status, stream);
+  return run<true, true>(ta, tb, n_out, r, M, dB, 2, status, stream);
 }
 
 }  // namespace qlora
