@@ -185,6 +185,53 @@ QLORA_API qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16_
                               void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Adam / AdamW on the adapters, fused into the backward ("QLoRA (low-rank adapters
+ * on a quantized model)", "The code, line by line": opt = Adam(A + B, lr=lr) is
+ * given dA and dB only; "LoRA fine-tuning on GPT-2" trains with AdamW).  The
+ * rule (Kingma & Ba with bias correction, weight decay decoupled as in AdamW):
+ *   theta <- theta (1 - lr wd);  m <- b1 m + (1 - b1) g;  v <- b2 v + (1 - b2) g^2;
+ *   theta <- theta - lr (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps)
+ * in fp32 for every element of A (g = dA) and of B (g = dB).
+ */
+typedef struct {
+  float lr;             /* >= 0 */
+  float beta1, beta2;   /* in [0, 1) */
+  float eps;            /* > 0 */
+  float weight_decay;   /* >= 0; 0 is plain Adam */
+  int64_t step;         /* t, 1-based: the bias corrections use b^t */
+} qlora_adam_hparams;
+
+/* The adapters' optimizer state, caller-owned fp32 device arrays, 16-byte aligned:
+ * master copies A32 (in, r) and B32 (r, out), and the first (m) and second (v)
+ * moments of each in the same layouts.  Updated in place. */
+typedef struct {
+  float* A32;
+  float* B32;
+  float* mA;
+  float* vA;
+  float* mB;
+  float* vB;
+} qlora_adam_state;
+
+/*
+ * One training step's backward with the optimizer step fused in: the gradients
+ * of qlora_linear_bwd (dX written if dX != NULL), and instead of writing dA and
+ * dB, one Adam step on (A32, mA, vA) with dA and on (B32, mB, vB) with dB, then
+ * A = bf16(A32) and B = bf16(B32) in place.  dA and dB never reach memory.  dX
+ * and U use the adapters as they were on entry (every read of A or B is ordered
+ * before their update).
+ *   X, V, dY, dX, ws, M, r: as for qlora_linear_bwd.
+ *   A, B  [device] bf16, read, then overwritten with the updated adapters.
+ *   st    [host] pointers to the optimizer state (device arrays, as above).
+ *   hp    [host] hyper-parameters; QLORA_ERR_INVALID_ARG if out of range.
+ */
+QLORA_API qlora_status qlora_linear_bwd_adam(const qlora_nf4_weight* w, const uint16_t* X, const uint16_t* V,
+                                             const uint16_t* dY, int64_t M, uint16_t* A, uint16_t* B, int r,
+                                             uint16_t* dX, const qlora_adam_state* st,
+                                             const qlora_adam_hparams* hp, void* ws, size_t ws_bytes,
+                                             void* stream);
+
+/*
  * Merge the adapters into a dense weight ("How it works" step 5):
  *   W_out = w' + A B   (fp32 accumulation; QLORA_F32 or QLORA_BF16 output, (in, out)).
  * Requires in % 64 == 0, out % 64 == 0, 8 <= r <= 256, r % 8 == 0.

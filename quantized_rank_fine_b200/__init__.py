@@ -35,7 +35,7 @@ EXPORTS = (
     "qlora_quantize_nf4", "qlora_dequantize", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_merge",
     "qlora_workspace_bytes", "qlora_ws_init", "qlora_ws_status", "qlora_nf4_codebook",
     "qlora_adapter_params", "qlora_status_string", "qlora_time_kernel", "qlora_launch_count",
-    "qlora_linear_fwd_static_ws",
+    "qlora_linear_fwd_static_ws", "qlora_linear_bwd_adam",
 )
 
 # Kernel ids of qlora_time_kernel.
@@ -52,6 +52,15 @@ class QLoRAError(RuntimeError):
 class _Weight(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("dq_codes", ctypes.c_void_p), ("dq_scales", ctypes.c_void_p),
                 ("in_", ctypes.c_int64), ("out", ctypes.c_int64)]
+
+
+class _AdamHparams(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float), ("step", ctypes.c_int64)]
+
+
+class _AdamState(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_void_p) for k in ("A32", "B32", "mA", "vA", "mB", "vB")]
 
 
 _lib = None
@@ -81,6 +90,8 @@ def lib() -> ctypes.CDLL:
             "qlora_time_kernel": (i32, [i32, ctypes.POINTER(vp), ctypes.POINTER(vp), i32]),
             "qlora_launch_count": (ctypes.c_uint64, []),
             "qlora_linear_fwd_static_ws": (i32, [wp, vp, i64, vp, vp, i32, vp, vp, vp]),
+            "qlora_linear_bwd_adam": (i32, [wp, vp, vp, vp, i64, vp, vp, i32, vp, ctypes.POINTER(_AdamState),
+                                            ctypes.POINTER(_AdamHparams), vp, sz, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -257,3 +268,33 @@ def qlora_linear_bwd(w: NF4Weight, X: torch.Tensor, V, dY: torch.Tensor, A: torc
                                   _ptr(dX) if need_dX else None, _ptr(dA), _ptr(dB), _ptr(buf), buf.numel(),
                                   _stream(stream)), "qlora_linear_bwd")
     return (dX if need_dX else None), dA, dB
+
+
+def adam_state(A: torch.Tensor, B: torch.Tensor) -> dict:
+    """Fresh optimizer state for one layer's adapters: fp32 master copies of A and
+    B and zero moments (device tensors, the layouts of A and B)."""
+    return {"A32": A.float().contiguous(), "B32": B.float().contiguous(),
+            "mA": torch.zeros(A.shape, dtype=torch.float32, device=A.device),
+            "vA": torch.zeros(A.shape, dtype=torch.float32, device=A.device),
+            "mB": torch.zeros(B.shape, dtype=torch.float32, device=B.device),
+            "vB": torch.zeros(B.shape, dtype=torch.float32, device=B.device)}
+
+
+def qlora_linear_bwd_adam(w: NF4Weight, X: torch.Tensor, V, dY: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
+                          state: dict, step: int, workspace: Workspace, lr: float = 1e-3, beta1: float = 0.9,
+                          beta2: float = 0.999, eps: float = 1e-8, weight_decay: float = 0.0,
+                          need_dX: bool = True, stream=None, dX=None):
+    """Backward with one fused Adam/AdamW step on the adapters: updates `state`
+    (fp32 A32, B32, mA, vA, mB, vB) and the bf16 A and B in place; returns dX or None."""
+    M, r = X.shape[0], A.shape[1]
+    if need_dX and dX is None:
+        dX = torch.empty((M, w.n_in), dtype=torch.bfloat16, device=X.device)
+    nb = qlora_workspace_bytes(QLORA_OP_BWD, M, w.n_in, w.n_out, r)
+    buf = workspace.get(nb, stream)
+    ws = w.c_struct()
+    st = _AdamState(*[_ptr(state[k]) for k in ("A32", "B32", "mA", "vA", "mB", "vB")])
+    hp = _AdamHparams(lr, beta1, beta2, eps, weight_decay, step)
+    _check(lib().qlora_linear_bwd_adam(ctypes.byref(ws), _ptr(X), _ptr(V), _ptr(dY), M, _ptr(A), _ptr(B), r,
+                                       _ptr(dX) if need_dX else None, ctypes.byref(st), ctypes.byref(hp),
+                                       _ptr(buf), buf.numel(), _stream(stream)), "qlora_linear_bwd_adam")
+    return dX if need_dX else None

@@ -1,6 +1,8 @@
 // The C ABI of libqlora: host-side argument checks, workspace layout, launches.
 // Declarations, argument meaning, layouts and error behaviour: include/qlora.h.
 #include <cuda_runtime.h>
+
+#include <cmath>
 #include <string.h>
 
 #include <atomic>
@@ -314,6 +316,72 @@ qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16_t* X, cons
   QLORA_CUDA(qlora::launch_vtdy(V, dY, M, w->out, r, dB, status, s));
   QLORA_CUDA(qlora::launch_xtu(X, U, M, w->in, r, dA, status, s));
   if (dX) QLORA_CUDA(qlora::launch_dx_gemm(wv, dY, U, A, M, r, dX, status, s));
+  return QLORA_OK;
+}
+
+qlora_status qlora_linear_bwd_adam(const qlora_nf4_weight* w, const uint16_t* X, const uint16_t* V,
+                                   const uint16_t* dY, int64_t M, uint16_t* A, uint16_t* B, int r, uint16_t* dX,
+                                   const qlora_adam_state* st, const qlora_adam_hparams* hp, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  if (!X || !dY || !A || !B || !st || !hp) return QLORA_ERR_INVALID_ARG;
+  if (!st->A32 || !st->B32 || !st->mA || !st->vA || !st->mB || !st->vB) return QLORA_ERR_INVALID_ARG;
+  if (!(hp->lr >= 0.0f) || !(hp->beta1 >= 0.0f && hp->beta1 < 1.0f) || !(hp->beta2 >= 0.0f && hp->beta2 < 1.0f) ||
+      !(hp->eps > 0.0f) || !(hp->weight_decay >= 0.0f) || hp->step < 1 || !std::isfinite(hp->lr))
+    return QLORA_ERR_INVALID_ARG;
+  QLORA_TRY(check_weight_shape(w));
+  if (!linear_shape_ok(M, w->in, w->out, r)) return QLORA_ERR_SHAPE;
+  if (!ws || ws_bytes < ws_layout(QLORA_OP_BWD, M, w->in, w->out, r).total) return QLORA_ERR_WORKSPACE;
+  QLORA_TRY(check_device());
+  QLORA_TRY(check_weight(w));
+  QLORA_TRY(check_ptr(X));
+  QLORA_TRY(check_ptr(V, false));
+  QLORA_TRY(check_ptr(dY));
+  QLORA_TRY(check_ptr(A));
+  QLORA_TRY(check_ptr(B));
+  QLORA_TRY(check_ptr(dX, false));
+  for (const float* q : {st->A32, st->B32, st->mA, st->vA, st->mB, st->vB}) QLORA_TRY(check_ptr(q));
+  const WsLayout L = ws_layout(QLORA_OP_BWD, M, w->in, w->out, r);
+  QLORA_TRY(check_ptr(ws));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint32_t* status = reinterpret_cast<uint32_t*>(base);
+  uint16_t* U = reinterpret_cast<uint16_t*>(base + L.u_off);
+  const WeightView wv = view(w);
+
+  // bias corrections and the constants of the rule, in double then rounded once
+  const double t = static_cast<double>(hp->step);
+  qlora::AdamParams pa{};
+  pa.lr = hp->lr;
+  pa.b1 = hp->beta1;
+  pa.b2 = hp->beta2;
+  pa.omb1 = static_cast<float>(1.0 - static_cast<double>(hp->beta1));
+  pa.omb2 = static_cast<float>(1.0 - static_cast<double>(hp->beta2));
+  pa.eps = hp->eps;
+  pa.decay = static_cast<float>(1.0 - static_cast<double>(hp->lr) * static_cast<double>(hp->weight_decay));
+  pa.bc1 = static_cast<float>(1.0 - std::pow(static_cast<double>(hp->beta1), t));
+  pa.bc2 = static_cast<float>(1.0 - std::pow(static_cast<double>(hp->beta2), t));
+  if (!(pa.bc1 > 0.0f) || !(pa.bc2 > 0.0f)) return QLORA_ERR_INVALID_ARG;
+  qlora::AdamParams pA = pa, pB = pa;
+  pA.theta = st->A32;
+  pA.m = st->mA;
+  pA.v = st->vA;
+  pA.p16 = A;
+  pB.theta = st->B32;
+  pB.m = st->mB;
+  pB.v = st->vB;
+  pB.p16 = B;
+
+  // Every read of A or B comes before its update: U and V read them first, the
+  // B step follows U, dX reads A before the A step.
+  if (!V) {
+    uint16_t* Vw = reinterpret_cast<uint16_t*>(base + L.v_off);
+    QLORA_CUDA(qlora::launch_xa(X, A, M, w->in, r, Vw, status, s));
+    V = Vw;
+  }
+  QLORA_CUDA(qlora::launch_dybt(dY, B, M, w->out, r, U, status, s));
+  QLORA_CUDA(qlora::launch_vtdy(V, dY, M, w->out, r, nullptr, status, s, &pB));
+  if (dX) QLORA_CUDA(qlora::launch_dx_gemm(wv, dY, U, A, M, r, dX, status, s));
+  QLORA_CUDA(qlora::launch_xtu(X, U, M, w->in, r, nullptr, status, s, &pA));
   return QLORA_OK;
 }
 

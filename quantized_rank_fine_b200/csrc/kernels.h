@@ -38,16 +38,28 @@ cudaError_t launch_merge(const uint8_t* codes, const uint8_t* dq_codes, const fl
                          const uint16_t* A, const uint16_t* B, int r, int64_t n_in, int64_t n_out,
                          bool bf16, void* out, cudaStream_t stream);
 
+// One Adam step fused into a gradient's final store (see qlora_linear_bwd_adam):
+// the element g of parameter index i updates theta[i], m[i], v[i] and p16[i].
+struct AdamParams {
+  float* theta;
+  float* m;
+  float* v;
+  uint16_t* p16;
+  float lr, b1, b2, omb1, omb2, eps, decay, bc1, bc2;   // omb = 1 - b, decay = 1 - lr wd, bc = 1 - b^t
+};
+
 // Rank-r products (tcgen05), split-K reduced inside a thread-block cluster;
-// `status` is the workspace status word.
+// `status` is the workspace status word.  dA and dB take an optional Adam step
+// (adam != nullptr): the gradient then updates the optimizer state instead of
+// being stored.
 cudaError_t launch_xa(const uint16_t* X, const uint16_t* A, int64_t M, int64_t n_in, int r, uint16_t* V,
                       uint32_t* status, cudaStream_t stream);
 cudaError_t launch_dybt(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t n_out, int r,
                         uint16_t* U, uint32_t* status, cudaStream_t stream);
 cudaError_t launch_xtu(const uint16_t* X, const uint16_t* U, int64_t M, int64_t n_in, int r, float* dA,
-                       uint32_t* status, cudaStream_t stream);
+                       uint32_t* status, cudaStream_t stream, const AdamParams* adam = nullptr);
 cudaError_t launch_vtdy(const uint16_t* V, const uint16_t* dY, int64_t M, int64_t n_out, int r,
-                        float* dB, uint32_t* status, cudaStream_t stream);
+                        float* dB, uint32_t* status, cudaStream_t stream, const AdamParams* adam = nullptr);
 
 // Small-M forward (M <= kGemvMaxTokens): base + adapter in one kernel, the
 // K-splits of a column tile reduced inside a thread-block cluster; no workspace.

@@ -48,9 +48,36 @@ struct SkArgs {
   void* out;
   int out_kind;          // 0 = bf16 [row][r], 1 = fp32 [row][r], 2 = fp32 transposed [r][row]
   uint32_t* status;
+  int adam;              // out_kind 1 or 2: apply the Adam step instead of storing
+  AdamParams ap;
 };
 
+// One Adam / AdamW step of parameter element i with gradient g (fp32, IEEE
+// division and square root; see qlora_linear_bwd_adam for the rule).
+__device__ __forceinline__ void adam_element(const AdamParams& a, int64_t i, float g) {
+  const float th = a.theta[i] * a.decay;
+  const float m = fmaf(a.b1, a.m[i], a.omb1 * g);
+  const float v = fmaf(a.b2, a.v[i], a.omb2 * (g * g));
+  const float den = sqrtf(__fdiv_rn(v, a.bc2)) + a.eps;
+  const float th1 = th - a.lr * __fdiv_rn(__fdiv_rn(m, a.bc1), den);
+  a.theta[i] = th1;
+  a.m[i] = m;
+  a.v[i] = v;
+  a.p16[i] = static_cast<uint16_t>(pack_bf16x2(th1, 0.0f));
+}
+
 __device__ __forceinline__ void store_pair(const SkArgs& p, int64_t row, int col, float v0, float v1) {
+  if (p.adam) {
+    // dA (in, r): element (row, col); dB (r, out) from dB^T: element (col, row)
+    if (p.out_kind == 1) {
+      adam_element(p.ap, row * p.r + col, v0);
+      adam_element(p.ap, row * p.r + col + 1, v1);
+    } else {
+      adam_element(p.ap, static_cast<int64_t>(col) * p.rows + row, v0);
+      adam_element(p.ap, static_cast<int64_t>(col + 1) * p.rows + row, v1);
+    }
+    return;
+  }
   if (p.out_kind == 0) {
     *reinterpret_cast<uint32_t*>(reinterpret_cast<uint16_t*>(p.out) + row * p.r + col) = pack_bf16x2(v0, v1);
   } else if (p.out_kind == 1) {
@@ -280,7 +307,7 @@ Plan plan(int64_t rows, int r, int64_t k_total) {
 
 template <bool A_MN, bool B_MN>
 cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows, int r, int64_t k_total, void* out,
-                int out_kind, uint32_t* status, cudaStream_t stream) {
+                int out_kind, uint32_t* status, cudaStream_t stream, const AdamParams* adam = nullptr) {
   static bool set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -293,7 +320,7 @@ cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows, int 
     set[dev] = true;
   }
   const Plan pl = plan(rows, r, k_total);
-  SkArgs a{rows, r, k_total, pl.kps, out, out_kind, status};
+  SkArgs a{rows, r, k_total, pl.kps, out, out_kind, status, adam ? 1 : 0, adam ? *adam : AdamParams{}};
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = pl.grid;
   cfg.blockDim = dim3(kSkThreads);
@@ -333,18 +360,18 @@ cudaError_t launch_dybt(const uint16_t* dY, const uint16_t* B, int64_t M, int64_
 
 // dA = X^T U: Aop[i][m] = X[m][i] (i contiguous); Bop[j][m] = U[m][j] (j contiguous).
 cudaError_t launch_xtu(const uint16_t* X, const uint16_t* U, int64_t M, int64_t n_in, int r, float* dA,
-                       uint32_t* status, cudaStream_t stream) {
+                       uint32_t* status, cudaStream_t stream, const AdamParams* adam) {
   CUtensorMap ta, tb;
   if (!bf16_map(&ta, X, M, n_in, 64, 64) || !bf16_map(&tb, U, M, r, 64, 64)) return cudaErrorInvalidValue;
-  return run<true, true>(ta, tb, n_in, r, M, dA, 1, status, stream);
+  return run<true, true>(ta, tb, n_in, r, M, dA, 1, status, stream, adam);
 }
 
 // dB^T = dY^T V: Aop[o][m] = dY[m][o] (o contiguous); Bop[j][m] = V[m][j]; stored as dB (r x out).
 cudaError_t launch_vtdy(const uint16_t* V, const uint16_t* dY, int64_t M, int64_t n_out, int r, float* dB,
-                        uint32_t* status, cudaStream_t stream) {
+                        uint32_t* status, cudaStream_t stream, const AdamParams* adam) {
   CUtensorMap ta, tb;
   if (!bf16_map(&ta, dY, M, n_out, 64, 64) || !bf16_map(&tb, V, M, r, 64, 64)) return cudaErrorInvalidValue;
-  return run<true, true>(ta, tb, n_out, r, M, dB, 2, status, stream);
+  return run<true, true>(ta, tb, n_out, r, M, dB, 2, status, stream, adam);
 }
 
 }  // namespace qlora

@@ -86,6 +86,32 @@ def test_linear_rejects_before_launch(L):
     assert fwd(ctypes.byref(w0), FAKE, 64, FAKE, FAKE, 8, FAKE, None, FAKE, 1 << 30, None) == 1
 
 
+def test_bwd_adam_rejects_before_launch(L):
+    """The fused backward + Adam step checks its state pointers and
+    hyper-parameters on the host, before any device access."""
+    w = q._Weight(0x10000, 0x10000, 0x10000, 256, 256)
+    wp = ctypes.byref(w)
+    st = q._AdamState(*([0x10000] * 6))
+    hp = q._AdamHparams(1e-3, 0.9, 0.999, 1e-8, 0.0, 1)
+    f = L.qlora_linear_bwd_adam
+
+    def call(st_, hp_, r=8, ws_bytes=1 << 30):
+        return f(wp, FAKE, None, FAKE, 64, FAKE, FAKE, r, None, st_, hp_, FAKE, ws_bytes, None)
+
+    assert call(None, ctypes.byref(hp)) == 1                                        # state NULL
+    assert call(ctypes.byref(st), None) == 1                                        # hparams NULL
+    st0 = q._AdamState(0x10000, 0x10000, 0, 0x10000, 0x10000, 0x10000)              # mA NULL
+    assert call(ctypes.byref(st0), ctypes.byref(hp)) == 1
+    for bad in (dict(step=0), dict(beta1=1.0), dict(beta2=-0.1), dict(eps=0.0), dict(lr=-1.0),
+                dict(weight_decay=-0.5), dict(lr=float("nan"))):
+        h = q._AdamHparams(1e-3, 0.9, 0.999, 1e-8, 0.0, 1)
+        for k, v in bad.items():
+            setattr(h, k, v)
+        assert call(ctypes.byref(st), ctypes.byref(h)) == 1, bad
+    assert call(ctypes.byref(st), ctypes.byref(hp), r=12) == 2                      # r % 8
+    assert call(ctypes.byref(st), ctypes.byref(hp), ws_bytes=8) == 4                # workspace too small
+
+
 def test_dequant_merge_reject_before_launch(L):
     w = q._Weight(0x10000, 0x10000, 0x10000, 256, 256)
     assert L.qlora_dequantize(ctypes.byref(w), FAKE, 5, None) == 1                      # bad dtype

@@ -71,7 +71,7 @@ def test_zero_gradient_zero_moments_leaves_adapters():
     np.testing.assert_allclose(t2, theta * (1 - 1e-4), rtol=1e-15)
 
 
-def test_step_is_bounded_by_lr_times_bias_ratio():
+def test_first_step_bounded_by_lr():
     """From zero state the first bias-corrected step of every element is at most lr
     and points against the gradient; a sign or bias-correction slip breaks this."""
     rng = np.random.default_rng(9)
