@@ -60,6 +60,10 @@ def parse():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-rows", action="store_true", help="skip the per-kernel row measurements")
+    p.add_argument("--rows", default="all",
+                   help="comma-separated subset of the rows: quantize, dequantize, merge, gemv, train_step")
+    p.add_argument("--rows-only", action="store_true",
+                   help="measure only the rows (no headline step); prints {'rows': ...}")
     p.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     return p.parse_args()
 
@@ -214,8 +218,28 @@ def run_step(layers, ws):
         q.qlora_linear_bwd(w, t["X"], o["V"], t["dY"], t["A"], t["B"], ws, dX=o["dX"], dA=o["dA"], dB=o["dB"])
 
 
-def time_rows(wl, pk):
-    """Per-kernel measurements of the other rows of the path (one GPU)."""
+ROW_NAMES = ("quantize", "dequantize", "merge", "gemv", "train_step")
+
+
+def time_rows(wl, pk, which="all"):
+    """Per-kernel measurements of the other rows of the path (one GPU); `which`
+    is "all" or a comma-separated subset of ROW_NAMES."""
+    want = set(ROW_NAMES) if which == "all" else set(which.split(","))
+    unknown = want - set(ROW_NAMES)
+    if unknown:
+        raise SystemExit(f"unknown rows: {sorted(unknown)}")
+    rows = {}
+    if want & {"quantize", "dequantize", "merge"}:
+        rows.update(time_weight_rows(wl, pk, want))
+    if "gemv" in want:
+        rows["gemv"] = time_gemv(pk)
+    if "train_step" in want:
+        rows["train_step_adam"] = time_train_step(wl)
+    return rows
+
+
+def time_weight_rows(wl, pk, want):
+    """Quantize, dequantize and merge on the workload's first weight shape."""
     import torch
     import quantized_rank_fine_b200 as q
     import synth
@@ -232,24 +256,85 @@ def time_rows(wl, pk):
 
     hbm = pk["hbm_gbs"]
     iters = 30
-    t = timed(lambda i: q.qlora_quantize_nf4(W0s[i % reps], out=ws_[i % reps]), q.KERNEL_QUANTIZE, iters)
-    b = n * (4 + 0.5 + 1 / 64) + 4 * math.ceil(n / 64 / 256)
-    rows["quantize"] = {"ms": t, "gbs": b / t / 1e6, "frac_hbm": b / t / 1e6 / hbm, "bytes_per_weight": 4.516}
-    outs = [torch.empty((n_in, n_out), dtype=torch.bfloat16, device="cuda") for _ in range(reps)]
-    t = timed(lambda i: q.qlora_dequantize(ws_[i % reps], torch.bfloat16, out=outs[i % reps]), q.KERNEL_DEQUANTIZE, iters)
-    b = n * (0.5 + 1 / 64 + 2) + 4 * math.ceil(n / 64 / 256)
-    rows["dequantize_bf16"] = {"ms": t, "gbs": b / t / 1e6, "frac_hbm": b / t / 1e6 / hbm}
-    r = wl["r"]
-    A = synth.normal("rowsA", (n_in, r), 1 / math.sqrt(n_in), torch.bfloat16, "cuda")
-    B = synth.normal("rowsB", (r, n_out), 0.01, torch.bfloat16, "cuda")
-    outs32 = [torch.empty((n_in, n_out), dtype=torch.float32, device="cuda") for _ in range(reps)]
-    t = timed(lambda i: q.qlora_merge(ws_[i % reps], A, B, torch.float32, out=outs32[i % reps]), q.KERNEL_MERGE, iters)
-    b = n * (0.5 + 1 / 64 + 4) + 2 * r * (n_in + n_out)
-    rows["merge_f32"] = {"ms": t, "gbs": b / t / 1e6, "frac_hbm": b / t / 1e6 / hbm}
-    del outs, outs32, W0s, ws_
+    if "quantize" in want:
+        t = timed(lambda i: q.qlora_quantize_nf4(W0s[i % reps], out=ws_[i % reps]), q.KERNEL_QUANTIZE, iters)
+        b = n * (4 + 0.5 + 1 / 64) + 4 * math.ceil(n / 64 / 256)
+        rows["quantize"] = {"ms": t, "gbs": b / t / 1e6, "frac_hbm": b / t / 1e6 / hbm, "bytes_per_weight": 4.516}
+    if "dequantize" in want:
+        outs = [torch.empty((n_in, n_out), dtype=torch.bfloat16, device="cuda") for _ in range(reps)]
+        t = timed(lambda i: q.qlora_dequantize(ws_[i % reps], torch.bfloat16, out=outs[i % reps]),
+                  q.KERNEL_DEQUANTIZE, iters)
+        b = n * (0.5 + 1 / 64 + 2) + 4 * math.ceil(n / 64 / 256)
+        rows["dequantize_bf16"] = {"ms": t, "gbs": b / t / 1e6, "frac_hbm": b / t / 1e6 / hbm}
+        del outs
+    if "merge" in want:
+        r = wl["r"]
+        A = synth.normal("rowsA", (n_in, r), 1 / math.sqrt(n_in), torch.bfloat16, "cuda")
+        B = synth.normal("rowsB", (r, n_out), 0.01, torch.bfloat16, "cuda")
+        outs32 = [torch.empty((n_in, n_out), dtype=torch.float32, device="cuda") for _ in range(reps)]
+        t = timed(lambda i: q.qlora_merge(ws_[i % reps], A, B, torch.float32, out=outs32[i % reps]),
+                  q.KERNEL_MERGE, iters)
+        b = n * (0.5 + 1 / 64 + 4) + 2 * r * (n_in + n_out)
+        rows["merge_f32"] = {"ms": t, "gbs": b / t / 1e6, "frac_hbm": b / t / 1e6 / hbm}
+        del outs32
+    del W0s, ws_
     torch.cuda.synchronize()
-    rows["gemv"] = time_gemv(pk)
     return rows
+
+
+def time_train_step(wl):
+    """A whole training step of the workload's layer: forward, then the backward
+    with the fused Adam step on the adapters (qlora_linear_bwd_adam), against the
+    plain forward + backward of the headline step; both captured in CUDA graphs
+    of back-to-back steps over rotated input sets larger than L2."""
+    import torch
+    import quantized_rank_fine_b200 as q
+    M = wl["M"]
+    nsets = max(2, math.ceil(3 * L2_BYTES / set_bytes(wl)))
+    sets = build_sets(wl, nsets, seed_base=7)
+    states = [[q.adam_state(t["A"], t["B"]) for (_, t, _) in layers] for layers in sets]
+    ws = q.Workspace()
+    iters = 20
+
+    def plain(i):
+        run_step(sets[i % nsets], ws)
+
+    def adam_step(i):
+        for li, (w, t, o) in enumerate(sets[i % nsets]):
+            q.qlora_linear_fwd(w, t["X"], t["A"], t["B"], ws, Y=o["Y"], V=o["V"])
+            q.qlora_linear_bwd_adam(w, t["X"], o["V"], t["dY"], t["A"], t["B"], states[i % nsets][li],
+                                    5 + i, ws, dX=o["dX"])
+
+    out = {}
+    for name, fn in (("fwd_bwd", plain), ("fwd_bwd_adam", adam_step)):
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph, stream=side):
+                for i in range(iters):
+                    fn(i)
+        torch.cuda.current_stream().wait_stream(side)
+        graph.replay()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(3):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            graph.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1) / iters)
+        del graph
+        t = statistics.median(times)
+        out[name] = {"ms_per_step": t, "tokens_per_s": M / (t * 1e-3)}
+    if ws.status() != 0:
+        raise RuntimeError("a kernel wait timed out in the training-step row")
+    out["adam_overhead_ms"] = out["fwd_bwd_adam"]["ms_per_step"] - out["fwd_bwd"]["ms_per_step"]
+    return out
 
 
 def graph_timed(fn, which, iters):
@@ -354,27 +439,62 @@ def arm_ours(args, world, rank, local):
     if ws.status() != 0:
         raise RuntimeError("a kernel wait timed out during warm-up")
 
-    timer = q.KernelTimer(q.KERNEL_FWD_GEMM, args.steps * nl)
+    # The K timed steps run as CUDA-graph replays (no host launch gaps): graph G
+    # holds one step on each of the nsets input sets, graph R the K mod nsets
+    # steps left over, so that exactly K steps are timed.  GT is G with the
+    # library's timing hook armed: it records events around each fwd GEMM into
+    # the graph.  GT runs as the last replay inside the timed region (event
+    # nodes between kernels cost a little, so the other replays run G).
     stream = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+
+    def capture(count, timed):
+        timer_ = q.KernelTimer(q.KERNEL_FWD_GEMM, count * nl) if timed else None
+        g = torch.cuda.CUDAGraph()
+        side.wait_stream(stream)
+        c0 = q.qlora_launch_count()
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side, capture_error_mode="relaxed"):
+                for i in range(count):
+                    run_step(sets[i % nsets], ws)
+        stream.wait_stream(side)
+        if timer_ is not None:
+            timer_.disarm()
+        return g, timer_, (q.qlora_launch_count() - c0) // count
+
+    if args.steps >= nsets:
+        n_rep, n_gt, n_rem = args.steps // nsets, nsets, args.steps % nsets
+    else:
+        n_rep, n_gt, n_rem = 1, args.steps, 0
+    G = capture(nsets, False)[0] if n_rep > 1 else None
+    GT, timer, launches_per_step = capture(n_gt, True)
+    R = capture(n_rem, False)[0] if n_rem else None
+    for g in (G, GT, R):
+        if g is not None:
+            g.replay()
+    torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
     smi_id = vis.split(",")[local] if vis and len(vis.split(",")) > local else str(local)
     clocks = ClockSampler(smi_id)
-    launches0 = q.qlora_launch_count()
     barrier(world)
     torch.cuda.synchronize()
     clocks.start()
     ev0.record(stream)
-    for i in range(args.steps):
-        run_step(sets[i % nsets], ws)
+    if R is not None:
+        R.replay()
+    for _ in range(n_rep - 1):
+        G.replay()
+    if GT is not None:
+        GT.replay()
     ev1.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
     barrier(world)
-    launches = q.qlora_launch_count() - launches0
+    launches = launches_per_step * args.steps
     ms_local = ev0.elapsed_time(ev1)
     gemm_ms = timer.times_ms()
-    timer.disarm()
+    del G, GT, R
     if ws.status() != 0:
         raise RuntimeError("a kernel wait timed out in the timed region")
     ms = max_over_ranks(ms_local, world)
@@ -382,7 +502,7 @@ def arm_ours(args, world, rank, local):
     tokens = M * args.steps * world
     value = tokens / (ms / 1e3)
     step_flops = sum(flops_fwd_bwd(a, b, M, r) for a, b in wl["shapes"])
-    gemm_flops = [flops_fwd_gemm(a, b, M, r) for a, b in wl["shapes"]] * args.steps
+    gemm_flops = [flops_fwd_gemm(a, b, M, r) for a, b in wl["shapes"]] * n_gt
     achieved = sum(gemm_flops) / (sum(gemm_ms) / 1e3) / 1e12
     timed_s = ms / 1e3
     peak = pk["bf16_tflops"] if timed_s < 2.0 else pk["bf16_tflops_sustained"]
@@ -427,7 +547,7 @@ def arm_ours(args, world, rank, local):
     line["e2e"] = e2e(args, sets, ws, wl, world)
 
     if world == 1 and not args.no_rows:
-        line["rows"] = time_rows(wl, pk)
+        line["rows"] = time_rows(wl, pk, args.rows)
     if world == 1 and rank == 0 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(args.workload, budget_s=20.0)
     return line
@@ -588,6 +708,9 @@ def main():
     world, rank, local = dist_init(args)
     if args.impl == "reference":
         line = arm_reference(args, world, rank)
+    elif args.rows_only:
+        pk, _ = peaks()
+        line = {"rows": time_rows(WORKLOADS[args.workload], pk, args.rows)} if rank == 0 else None
     else:
         line = arm_ours(args, world, rank, local)
     if rank == 0 and line is not None:
