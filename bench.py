@@ -87,6 +87,11 @@ def flops_fwd_gemm(n_in, n_out, M, r):
     return 2 * M * n_out * (n_in + r)
 
 
+# the fused GEMM's source and every header it includes: traffic counters taken
+# from an ncu capture stay valid only while these are unchanged
+GEMM_SOURCES = ("gemm.cu", "sm100.cuh", "common.cuh")
+
+
 def src_hash(*names):
     h = hashlib.sha1()
     for n in names:
@@ -513,7 +518,7 @@ def arm_ours(args, world, rank, local):
             for line in f:
                 fields = line.split("#", 1)[0].split()
                 if len(fields) == 4 and fields[0] == args.workload and fields[1] == "fwd_gemm" \
-                        and fields[3] == src_hash("gemm.cu"):
+                        and fields[3] == src_hash(*GEMM_SOURCES):
                     traffic = int(fields[2])
 
     line = {
