@@ -136,6 +136,10 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Launched as a programmatic dependent: the set-up above overlaps the kernel
+  // before; nothing in global memory is touched until that kernel has finished.
+  grid_dependency_wait();
+  grid_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -362,13 +366,22 @@ cudaError_t launch_gemm(const CUtensorMap& act, const CUtensorMap& ea, const CUt
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  dim3 grid(static_cast<unsigned>((a.N + kBN - 1) / kBN), static_cast<unsigned>((a.M + kBM - 1) / kBM));
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>((a.N + kBN - 1) / kBN), static_cast<unsigned>((a.M + kBM - 1) / kBM));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
   const int which = kDX ? QLORA_KERNEL_DX_GEMM : QLORA_KERNEL_FWD_GEMM;
   timing_before(which, stream);
-  nf4_gemm_kernel<kDX><<<grid, kThreads, kSmemBytes, stream>>>(act, ea, eb, cm, a);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, nf4_gemm_kernel<kDX>, act, ea, eb, cm, a);
   timing_after(which, stream);
   count_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace

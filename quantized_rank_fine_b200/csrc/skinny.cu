@@ -136,6 +136,10 @@ skinny_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Launched as a programmatic dependent: the set-up above overlaps the kernel
+  // before; nothing in global memory is touched until that kernel has finished.
+  grid_dependency_wait();
+  grid_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -326,13 +330,15 @@ cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows, int 
   cfg.blockDim = dim3(kSkThreads);
   cfg.dynamicSmemBytes = kSkSmem;
   cfg.stream = stream;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = 1;
   at[0].val.clusterDim.y = static_cast<unsigned>(pl.splits);
   at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   timing_before(QLORA_KERNEL_RANK_R, stream);
   const cudaError_t e = cudaLaunchKernelEx(&cfg, skinny_tc_kernel<A_MN, B_MN>, ta, tb, a);
   timing_after(QLORA_KERNEL_RANK_R, stream);
