@@ -185,6 +185,39 @@ QLORA_API qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16_
                               void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Options of the _ex calls (and of qlora_linear_bwd_adam).
+ *   adapter_scale  s in Y = X bf16(w') + s (X A) B: the LoRA scaling alpha / r
+ *                  ("LoRA & QLoRA", "Scaling Factor alpha": it only rescales the
+ *                  learning rate of A and B, which the pages' lab leaves out);
+ *                  1 is the plain layer.  Applied where V = bf16(s X A) and
+ *                  U = bf16(s dY B^T) are formed, so dX, dA and dB carry it.
+ *                  A saved V is the scaled one.  Finite, else QLORA_ERR_INVALID_ARG.
+ *   flags          QLORA_ACCUMULATE_GRADS: the backward adds into dA and dB
+ *                  instead of overwriting them (gradient accumulation over
+ *                  micro-batches); not allowed for the forward or with Adam.
+ * A NULL options pointer means adapter_scale = 1 and no flags.
+ */
+#define QLORA_ACCUMULATE_GRADS 1u
+typedef struct {
+  float adapter_scale;
+  uint32_t flags;
+} qlora_linear_opts;
+
+/* qlora_linear_fwd with options (arguments otherwise as there). */
+QLORA_API qlora_status qlora_linear_fwd_ex(const qlora_nf4_weight* w, const uint16_t* X, int64_t M,
+                                           const uint16_t* A, const uint16_t* B, int r, uint16_t* Y,
+                                           uint16_t* V_save, const qlora_linear_opts* opts, void* ws,
+                                           size_t ws_bytes, void* stream);
+
+/* qlora_linear_bwd with options (arguments otherwise as there).  With
+ * QLORA_ACCUMULATE_GRADS, dA and dB must hold the sums so far (fp32). */
+QLORA_API qlora_status qlora_linear_bwd_ex(const qlora_nf4_weight* w, const uint16_t* X, const uint16_t* V,
+                                           const uint16_t* dY, int64_t M, const uint16_t* A, const uint16_t* B,
+                                           int r, uint16_t* dX, float* dA, float* dB,
+                                           const qlora_linear_opts* opts, void* ws, size_t ws_bytes,
+                                           void* stream);
+
+/*
  * Adam / AdamW on the adapters, fused into the backward ("QLoRA (low-rank adapters
  * on a quantized model)", "The code, line by line": opt = Adam(A + B, lr=lr) is
  * given dA and dB only; "LoRA fine-tuning on GPT-2" trains with AdamW).  The
@@ -224,12 +257,13 @@ typedef struct {
  *   A, B  [device] bf16, read, then overwritten with the updated adapters.
  *   st    [host] pointers to the optimizer state (device arrays, as above).
  *   hp    [host] hyper-parameters; QLORA_ERR_INVALID_ARG if out of range.
+ *   opts  [host] options or NULL (adapter_scale; QLORA_ACCUMULATE_GRADS is refused).
  */
 QLORA_API qlora_status qlora_linear_bwd_adam(const qlora_nf4_weight* w, const uint16_t* X, const uint16_t* V,
                                              const uint16_t* dY, int64_t M, uint16_t* A, uint16_t* B, int r,
                                              uint16_t* dX, const qlora_adam_state* st,
-                                             const qlora_adam_hparams* hp, void* ws, size_t ws_bytes,
-                                             void* stream);
+                                             const qlora_adam_hparams* hp, const qlora_linear_opts* opts,
+                                             void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Merge the adapters into a dense weight ("How it works" step 5):

@@ -35,10 +35,12 @@ def _f64(a) -> np.ndarray:
     return np.asarray(a, dtype=np.float64)
 
 
-def forward(X, A, B, Wq):
-    """Returns (Y, V) with V = X A and Y = X Wq + V B (float64)."""
+def forward(X, A, B, Wq, scale: float = 1.0):
+    """Returns (Y, V) with V = s X A and Y = X Wq + V B (float64); s is the
+    adapter scale alpha / r of "LoRA & QLoRA", "Scaling Factor alpha"
+    (h = W0 x + (alpha / r) B (A x)); 1 is the plain layer."""
     X, A, B, Wq = _f64(X), _f64(A), _f64(B), _f64(Wq)
-    V = X @ A
+    V = scale * (X @ A)
     Y = X @ Wq + V @ B
     return Y, V
 
@@ -49,13 +51,15 @@ def forward_rows(X, A, B, Wq, rows):
     return forward(X, A, B, Wq)
 
 
-def backward(X, A, B, Wq, dY):
-    """Returns dict(dX, dA, dB, U) for L with dL/dY = dY (float64)."""
+def backward(X, A, B, Wq, dY, scale: float = 1.0):
+    """Returns dict(dX, dA, dB, U) for L with dL/dY = dY (float64), for the layer
+    with adapter scale s: U = s dY B^T, dX = dY Wq^T + U A^T, dA = X^T U,
+    dB = s (X A)^T dY."""
     X, A, B, Wq, dY = _f64(X), _f64(A), _f64(B), _f64(Wq), _f64(dY)
-    U = dY @ B.T
+    U = scale * (dY @ B.T)
     dX = dY @ Wq.T + U @ A.T
     dA = X.T @ U
-    dB = (X @ A).T @ dY
+    dB = scale * ((X @ A).T @ dY)
     return {"dX": dX, "dA": dA, "dB": dB, "U": U}
 
 

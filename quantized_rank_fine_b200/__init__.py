@@ -35,8 +35,11 @@ EXPORTS = (
     "qlora_quantize_nf4", "qlora_dequantize", "qlora_linear_fwd", "qlora_linear_bwd", "qlora_merge",
     "qlora_workspace_bytes", "qlora_ws_init", "qlora_ws_status", "qlora_nf4_codebook",
     "qlora_adapter_params", "qlora_status_string", "qlora_time_kernel", "qlora_launch_count",
-    "qlora_linear_fwd_static_ws", "qlora_linear_bwd_adam",
+    "qlora_linear_fwd_static_ws", "qlora_linear_bwd_adam", "qlora_linear_fwd_ex", "qlora_linear_bwd_ex",
 )
+
+# Flag of qlora_linear_opts.flags.
+QLORA_ACCUMULATE_GRADS = 1
 
 # Kernel ids of qlora_time_kernel.
 KERNEL_QUANTIZE, KERNEL_DEQUANTIZE, KERNEL_MERGE, KERNEL_FWD_GEMM, KERNEL_DX_GEMM, KERNEL_RANK_R = 1, 2, 3, 4, 5, 6
@@ -57,6 +60,10 @@ class _Weight(ctypes.Structure):
 class _AdamHparams(ctypes.Structure):
     _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
                 ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float), ("step", ctypes.c_int64)]
+
+
+class _LinearOpts(ctypes.Structure):
+    _fields_ = [("adapter_scale", ctypes.c_float), ("flags", ctypes.c_uint32)]
 
 
 class _AdamState(ctypes.Structure):
@@ -91,7 +98,12 @@ def lib() -> ctypes.CDLL:
             "qlora_launch_count": (ctypes.c_uint64, []),
             "qlora_linear_fwd_static_ws": (i32, [wp, vp, i64, vp, vp, i32, vp, vp, vp]),
             "qlora_linear_bwd_adam": (i32, [wp, vp, vp, vp, i64, vp, vp, i32, vp, ctypes.POINTER(_AdamState),
-                                            ctypes.POINTER(_AdamHparams), vp, sz, vp]),
+                                            ctypes.POINTER(_AdamHparams), ctypes.POINTER(_LinearOpts), vp, sz,
+                                            vp]),
+            "qlora_linear_fwd_ex": (i32, [wp, vp, i64, vp, vp, i32, vp, vp, ctypes.POINTER(_LinearOpts), vp, sz,
+                                          vp]),
+            "qlora_linear_bwd_ex": (i32, [wp, vp, vp, vp, i64, vp, vp, i32, vp, vp, vp,
+                                          ctypes.POINTER(_LinearOpts), vp, sz, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -233,9 +245,14 @@ def qlora_merge(w: NF4Weight, A: torch.Tensor, B: torch.Tensor, dtype=torch.floa
     return out
 
 
+def _opts(adapter_scale: float, accumulate: bool = False):
+    return _LinearOpts(adapter_scale, QLORA_ACCUMULATE_GRADS if accumulate else 0)
+
+
 def qlora_linear_fwd(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, workspace: Workspace,
-                     save_V: bool = True, stream=None, Y=None, V=None):
-    """Returns (Y, V) with V = X A (None when save_V is False)."""
+                     save_V: bool = True, stream=None, Y=None, V=None, adapter_scale: float = 1.0):
+    """Returns (Y, V) with V = s X A (None when save_V is False); s =
+    adapter_scale (alpha / r), 1 for the plain layer."""
     M, r = X.shape[0], A.shape[1]
     if Y is None:
         Y = torch.empty((M, w.n_out), dtype=torch.bfloat16, device=X.device)
@@ -244,15 +261,25 @@ def qlora_linear_fwd(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Te
     nb = qlora_workspace_bytes(QLORA_OP_FWD, M, w.n_in, w.n_out, r)
     buf = workspace.get(nb, stream)
     ws = w.c_struct()
-    _check(lib().qlora_linear_fwd(ctypes.byref(ws), _ptr(X), M, _ptr(A), _ptr(B), r, _ptr(Y),
-                                  _ptr(V) if save_V else None, _ptr(buf), buf.numel(), _stream(stream)),
-           "qlora_linear_fwd")
+    if adapter_scale == 1.0:
+        _check(lib().qlora_linear_fwd(ctypes.byref(ws), _ptr(X), M, _ptr(A), _ptr(B), r, _ptr(Y),
+                                      _ptr(V) if save_V else None, _ptr(buf), buf.numel(), _stream(stream)),
+               "qlora_linear_fwd")
+    else:
+        o = _opts(adapter_scale)
+        _check(lib().qlora_linear_fwd_ex(ctypes.byref(ws), _ptr(X), M, _ptr(A), _ptr(B), r, _ptr(Y),
+                                         _ptr(V) if save_V else None, ctypes.byref(o), _ptr(buf), buf.numel(),
+                                         _stream(stream)), "qlora_linear_fwd_ex")
     return Y, (V if save_V else None)
 
 
 def qlora_linear_bwd(w: NF4Weight, X: torch.Tensor, V, dY: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
-                     workspace: Workspace, need_dX: bool = True, stream=None, dX=None, dA=None, dB=None):
-    """Returns (dX or None, dA fp32 (in, r), dB fp32 (r, out))."""
+                     workspace: Workspace, need_dX: bool = True, stream=None, dX=None, dA=None, dB=None,
+                     adapter_scale: float = 1.0, accumulate: bool = False):
+    """Returns (dX or None, dA fp32 (in, r), dB fp32 (r, out)).  With accumulate,
+    dA and dB (given) receive the sums instead of being overwritten."""
+    if accumulate and (dA is None or dB is None):
+        raise ValueError("accumulate needs the dA and dB to add into")
     M, r = X.shape[0], A.shape[1]
     dev = X.device
     if need_dX and dX is None:
@@ -264,9 +291,15 @@ def qlora_linear_bwd(w: NF4Weight, X: torch.Tensor, V, dY: torch.Tensor, A: torc
     nb = qlora_workspace_bytes(QLORA_OP_BWD, M, w.n_in, w.n_out, r)
     buf = workspace.get(nb, stream)
     ws = w.c_struct()
-    _check(lib().qlora_linear_bwd(ctypes.byref(ws), _ptr(X), _ptr(V), _ptr(dY), M, _ptr(A), _ptr(B), r,
-                                  _ptr(dX) if need_dX else None, _ptr(dA), _ptr(dB), _ptr(buf), buf.numel(),
-                                  _stream(stream)), "qlora_linear_bwd")
+    if adapter_scale == 1.0 and not accumulate:
+        _check(lib().qlora_linear_bwd(ctypes.byref(ws), _ptr(X), _ptr(V), _ptr(dY), M, _ptr(A), _ptr(B), r,
+                                      _ptr(dX) if need_dX else None, _ptr(dA), _ptr(dB), _ptr(buf), buf.numel(),
+                                      _stream(stream)), "qlora_linear_bwd")
+    else:
+        o = _opts(adapter_scale, accumulate)
+        _check(lib().qlora_linear_bwd_ex(ctypes.byref(ws), _ptr(X), _ptr(V), _ptr(dY), M, _ptr(A), _ptr(B), r,
+                                         _ptr(dX) if need_dX else None, _ptr(dA), _ptr(dB), ctypes.byref(o),
+                                         _ptr(buf), buf.numel(), _stream(stream)), "qlora_linear_bwd_ex")
     return (dX if need_dX else None), dA, dB
 
 
@@ -283,7 +316,7 @@ def adam_state(A: torch.Tensor, B: torch.Tensor) -> dict:
 def qlora_linear_bwd_adam(w: NF4Weight, X: torch.Tensor, V, dY: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
                           state: dict, step: int, workspace: Workspace, lr: float = 1e-3, beta1: float = 0.9,
                           beta2: float = 0.999, eps: float = 1e-8, weight_decay: float = 0.0,
-                          need_dX: bool = True, stream=None, dX=None):
+                          need_dX: bool = True, stream=None, dX=None, adapter_scale: float = 1.0):
     """Backward with one fused Adam/AdamW step on the adapters: updates `state`
     (fp32 A32, B32, mA, vA, mB, vB) and the bf16 A and B in place; returns dX or None."""
     M, r = X.shape[0], A.shape[1]
@@ -294,7 +327,35 @@ def qlora_linear_bwd_adam(w: NF4Weight, X: torch.Tensor, V, dY: torch.Tensor, A:
     ws = w.c_struct()
     st = _AdamState(*[_ptr(state[k]) for k in ("A32", "B32", "mA", "vA", "mB", "vB")])
     hp = _AdamHparams(lr, beta1, beta2, eps, weight_decay, step)
+    o = _opts(adapter_scale)
     _check(lib().qlora_linear_bwd_adam(ctypes.byref(ws), _ptr(X), _ptr(V), _ptr(dY), M, _ptr(A), _ptr(B), r,
                                        _ptr(dX) if need_dX else None, ctypes.byref(st), ctypes.byref(hp),
-                                       _ptr(buf), buf.numel(), _stream(stream)), "qlora_linear_bwd_adam")
+                                       ctypes.byref(o), _ptr(buf), buf.numel(), _stream(stream)),
+           "qlora_linear_bwd_adam")
     return dX if need_dX else None
+
+
+# ---------------------------------------------------------------- compositions
+# Built from the library's kernels (and, for the initialisation, a library SVD);
+# they are not on the per-step path.
+
+def requantize_merged(w: NF4Weight, A: torch.Tensor, B: torch.Tensor, stream=None) -> NF4Weight:
+    """Merge the adapters into the weight and quantise the merge again (the round
+    trip that keeps a merged model 4-bit): Q(deq(Wq) + A B), with the library's
+    merge (fp32) and quantiser."""
+    return qlora_quantize_nf4(qlora_merge(w, A, B, torch.float32, stream=stream), stream=stream)
+
+
+def loftq_init(W0: torch.Tensor, r: int, stream=None):
+    """Quantise W0 and start the adapters from the rank-r truncated SVD of the
+    quantisation residual R = W0 - deq(Q(W0)) = U S V^T, split as A = U_r S_r^1/2,
+    B = S_r^1/2 V_r^T (bf16), instead of B = 0.  Returns (NF4Weight, A, B).
+    The SVD is torch.linalg.svd on the device (a library decomposition, run once
+    at initialisation)."""
+    w = qlora_quantize_nf4(W0, stream=stream)
+    R = W0.float() - qlora_dequantize(w, torch.float32, stream=stream)
+    U, S, Vh = torch.linalg.svd(R, full_matrices=False)
+    root = S[:r].sqrt()
+    A = (U[:, :r] * root[None, :]).to(torch.bfloat16).contiguous()
+    B = (root[:, None] * Vh[:r, :]).to(torch.bfloat16).contiguous()
+    return w, A, B

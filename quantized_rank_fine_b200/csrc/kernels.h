@@ -49,17 +49,20 @@ struct AdamParams {
 };
 
 // Rank-r products (tcgen05), split-K reduced inside a thread-block cluster;
-// `status` is the workspace status word.  dA and dB take an optional Adam step
+// `status` is the workspace status word.  V and U are scaled by `scale` (the
+// adapter scale) as they are formed.  dA and dB take an optional Adam step
 // (adam != nullptr): the gradient then updates the optimizer state instead of
-// being stored.
+// being stored; `accumulate` adds them to the stored values instead.
 cudaError_t launch_xa(const uint16_t* X, const uint16_t* A, int64_t M, int64_t n_in, int r, uint16_t* V,
-                      uint32_t* status, cudaStream_t stream);
+                      uint32_t* status, cudaStream_t stream, float scale = 1.0f);
 cudaError_t launch_dybt(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t n_out, int r,
-                        uint16_t* U, uint32_t* status, cudaStream_t stream);
+                        uint16_t* U, uint32_t* status, cudaStream_t stream, float scale = 1.0f);
 cudaError_t launch_xtu(const uint16_t* X, const uint16_t* U, int64_t M, int64_t n_in, int r, float* dA,
-                       uint32_t* status, cudaStream_t stream, const AdamParams* adam = nullptr);
+                       uint32_t* status, cudaStream_t stream, const AdamParams* adam = nullptr,
+                       bool accumulate = false);
 cudaError_t launch_vtdy(const uint16_t* V, const uint16_t* dY, int64_t M, int64_t n_out, int r,
-                        float* dB, uint32_t* status, cudaStream_t stream, const AdamParams* adam = nullptr);
+                        float* dB, uint32_t* status, cudaStream_t stream, const AdamParams* adam = nullptr,
+                        bool accumulate = false);
 
 // Small-M forward (M <= kGemvMaxTokens): base + adapter in one kernel, the
 // K-splits of a column tile reduced inside a thread-block cluster; no workspace.
@@ -69,7 +72,7 @@ bool gemv_supported(int64_t M, int64_t K, int64_t N);
 // V = X A for M <= kGemvMaxTokens on CUDA cores (K split over a cluster); lets
 // the small-M forward launched after it start early.
 cudaError_t launch_xa_small(const uint16_t* X, const uint16_t* A, int64_t M, int64_t K, int r, uint16_t* V,
-                            cudaStream_t stream);
+                            cudaStream_t stream, float scale = 1.0f);
 cudaError_t launch_gemv(const WeightView& w, const uint16_t* X, const uint16_t* V, const uint16_t* B, int64_t M,
                         int r, uint16_t* Y, uint32_t* status, cudaStream_t stream);
 

@@ -50,6 +50,8 @@ struct SkArgs {
   uint32_t* status;
   int adam;              // out_kind 1 or 2: apply the Adam step instead of storing
   AdamParams ap;
+  float scale;           // every value is multiplied by it before the store
+  int accumulate;        // out_kind 1 or 2: add to the stored values instead of overwriting
 };
 
 // One Adam / AdamW step of parameter element i with gradient g (fp32, IEEE
@@ -67,6 +69,8 @@ __device__ __forceinline__ void adam_element(const AdamParams& a, int64_t i, flo
 }
 
 __device__ __forceinline__ void store_pair(const SkArgs& p, int64_t row, int col, float v0, float v1) {
+  v0 *= p.scale;
+  v1 *= p.scale;
   if (p.adam) {
     // dA (in, r): element (row, col); dB (r, out) from dB^T: element (col, row)
     if (p.out_kind == 1) {
@@ -81,11 +85,23 @@ __device__ __forceinline__ void store_pair(const SkArgs& p, int64_t row, int col
   if (p.out_kind == 0) {
     *reinterpret_cast<uint32_t*>(reinterpret_cast<uint16_t*>(p.out) + row * p.r + col) = pack_bf16x2(v0, v1);
   } else if (p.out_kind == 1) {
-    *reinterpret_cast<float2*>(reinterpret_cast<float*>(p.out) + row * p.r + col) = make_float2(v0, v1);
+    float2* d = reinterpret_cast<float2*>(reinterpret_cast<float*>(p.out) + row * p.r + col);
+    if (p.accumulate) {
+      const float2 o = *d;
+      v0 += o.x;
+      v1 += o.y;
+    }
+    *d = make_float2(v0, v1);
   } else {
     float* d = reinterpret_cast<float*>(p.out);
-    d[static_cast<int64_t>(col) * p.rows + row] = v0;
-    d[static_cast<int64_t>(col + 1) * p.rows + row] = v1;
+    float* d0 = d + static_cast<int64_t>(col) * p.rows + row;
+    float* d1 = d + static_cast<int64_t>(col + 1) * p.rows + row;
+    if (p.accumulate) {
+      v0 += *d0;
+      v1 += *d1;
+    }
+    *d0 = v0;
+    *d1 = v1;
   }
 }
 
@@ -311,7 +327,8 @@ Plan plan(int64_t rows, int r, int64_t k_total) {
 
 template <bool A_MN, bool B_MN>
 cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows, int r, int64_t k_total, void* out,
-                int out_kind, uint32_t* status, cudaStream_t stream, const AdamParams* adam = nullptr) {
+                int out_kind, uint32_t* status, cudaStream_t stream, const AdamParams* adam = nullptr,
+                float scale = 1.0f, bool accumulate = false) {
   static bool set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -324,7 +341,8 @@ cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows, int 
     set[dev] = true;
   }
   const Plan pl = plan(rows, r, k_total);
-  SkArgs a{rows, r, k_total, pl.kps, out, out_kind, status, adam ? 1 : 0, adam ? *adam : AdamParams{}};
+  SkArgs a{rows, r, k_total, pl.kps, out, out_kind, status, adam ? 1 : 0, adam ? *adam : AdamParams{}, scale,
+           accumulate ? 1 : 0};
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = pl.grid;
   cfg.blockDim = dim3(kSkThreads);
@@ -350,34 +368,34 @@ cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows, int 
 
 // V = X A: Aop = X (M x in, k contiguous); Bop[j][k] = A[k][j] (j contiguous).
 cudaError_t launch_xa(const uint16_t* X, const uint16_t* A, int64_t M, int64_t n_in, int r, uint16_t* V,
-                      uint32_t* status, cudaStream_t stream) {
+                      uint32_t* status, cudaStream_t stream, float scale) {
   CUtensorMap ta, tb;
   if (!bf16_map(&ta, X, M, n_in, 64, 128) || !bf16_map(&tb, A, n_in, r, 64, 64)) return cudaErrorInvalidValue;
-  return run<false, true>(ta, tb, M, r, n_in, V, 0, status, stream);
+  return run<false, true>(ta, tb, M, r, n_in, V, 0, status, stream, nullptr, scale);
 }
 
 // U = dY B^T: Aop = dY (M x out, k contiguous); Bop = B (r x out, k contiguous).
 cudaError_t launch_dybt(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t n_out, int r, uint16_t* U,
-                        uint32_t* status, cudaStream_t stream) {
+                        uint32_t* status, cudaStream_t stream, float scale) {
   CUtensorMap ta, tb;
   if (!bf16_map(&ta, dY, M, n_out, 64, 128) || !bf16_map(&tb, B, r, n_out, 64, 64)) return cudaErrorInvalidValue;
-  return run<false, false>(ta, tb, M, r, n_out, U, 0, status, stream);
+  return run<false, false>(ta, tb, M, r, n_out, U, 0, status, stream, nullptr, scale);
 }
 
 // dA = X^T U: Aop[i][m] = X[m][i] (i contiguous); Bop[j][m] = U[m][j] (j contiguous).
 cudaError_t launch_xtu(const uint16_t* X, const uint16_t* U, int64_t M, int64_t n_in, int r, float* dA,
-                       uint32_t* status, cudaStream_t stream, const AdamParams* adam) {
+                       uint32_t* status, cudaStream_t stream, const AdamParams* adam, bool accumulate) {
   CUtensorMap ta, tb;
   if (!bf16_map(&ta, X, M, n_in, 64, 64) || !bf16_map(&tb, U, M, r, 64, 64)) return cudaErrorInvalidValue;
-  return run<true, true>(ta, tb, n_in, r, M, dA, 1, status, stream, adam);
+  return run<true, true>(ta, tb, n_in, r, M, dA, 1, status, stream, adam, 1.0f, accumulate);
 }
 
 // dB^T = dY^T V: Aop[o][m] = dY[m][o] (o contiguous); Bop[j][m] = V[m][j]; stored as dB (r x out).
 cudaError_t launch_vtdy(const uint16_t* V, const uint16_t* dY, int64_t M, int64_t n_out, int r, float* dB,
-                        uint32_t* status, cudaStream_t stream, const AdamParams* adam) {
+                        uint32_t* status, cudaStream_t stream, const AdamParams* adam, bool accumulate) {
   CUtensorMap ta, tb;
   if (!bf16_map(&ta, dY, M, n_out, 64, 64) || !bf16_map(&tb, V, M, r, 64, 64)) return cudaErrorInvalidValue;
-  return run<true, true>(ta, tb, n_out, r, M, dB, 2, status, stream, adam);
+  return run<true, true>(ta, tb, n_out, r, M, dB, 2, status, stream, adam, 1.0f, accumulate);
 }
 
 }  // namespace qlora

@@ -43,6 +43,7 @@ struct XaArgs {
   int r;
   int Kc;              // rows per split (multiple of 64)
   uint16_t* V;         // (M, r) bf16
+  float scale;         // V = bf16(scale * X A)
 };
 
 __global__ void __launch_bounds__(kXaThreads) xa_small_kernel(const XaArgs p) {
@@ -144,7 +145,7 @@ __global__ void __launch_bounds__(kXaThreads) xa_small_kernel(const XaArgs p) {
     float y = 0.0f;
     for (int sp = 0; sp < S; ++sp) y += recv[sp * cap + slot];
     const int mm = e / cols, jj = e % cols;
-    p.V[static_cast<int64_t>(mm) * p.r + c0 + jj] = static_cast<uint16_t>(pack_bf16x2(y, 0.0f));
+    p.V[static_cast<int64_t>(mm) * p.r + c0 + jj] = static_cast<uint16_t>(pack_bf16x2(y * p.scale, 0.0f));
   }
 }
 
@@ -163,7 +164,7 @@ void xa_plan(int64_t K, int& S, int& Kc) {
 }  // namespace
 
 cudaError_t launch_xa_small(const uint16_t* X, const uint16_t* A, int64_t M, int64_t K, int r, uint16_t* V,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, float scale) {
   if (M < 1 || M > kGemvMaxTokens) return cudaErrorInvalidValue;
   static bool attr_set[64] = {};
   int dev = 0;
@@ -178,7 +179,7 @@ cudaError_t launch_xa_small(const uint16_t* X, const uint16_t* A, int64_t M, int
   }
   int S, Kc;
   xa_plan(K, S, Kc);
-  XaArgs a{X, A, static_cast<int>(M), K, r, Kc, V};
+  XaArgs a{X, A, static_cast<int>(M), K, r, Kc, V, scale};
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>((r + kXaCols - 1) / kXaCols), static_cast<unsigned>(S));
   cfg.blockDim = dim3(kXaThreads);

@@ -95,8 +95,8 @@ def test_bwd_adam_rejects_before_launch(L):
     hp = q._AdamHparams(1e-3, 0.9, 0.999, 1e-8, 0.0, 1)
     f = L.qlora_linear_bwd_adam
 
-    def call(st_, hp_, r=8, ws_bytes=1 << 30):
-        return f(wp, FAKE, None, FAKE, 64, FAKE, FAKE, r, None, st_, hp_, FAKE, ws_bytes, None)
+    def call(st_, hp_, r=8, ws_bytes=1 << 30, opts=None):
+        return f(wp, FAKE, None, FAKE, 64, FAKE, FAKE, r, None, st_, hp_, opts, FAKE, ws_bytes, None)
 
     assert call(None, ctypes.byref(hp)) == 1                                        # state NULL
     assert call(ctypes.byref(st), None) == 1                                        # hparams NULL
@@ -110,6 +110,25 @@ def test_bwd_adam_rejects_before_launch(L):
         assert call(ctypes.byref(st), ctypes.byref(h)) == 1, bad
     assert call(ctypes.byref(st), ctypes.byref(hp), r=12) == 2                      # r % 8
     assert call(ctypes.byref(st), ctypes.byref(hp), ws_bytes=8) == 4                # workspace too small
+    acc = q._LinearOpts(1.0, q.QLORA_ACCUMULATE_GRADS)
+    assert call(ctypes.byref(st), ctypes.byref(hp), opts=ctypes.byref(acc)) == 1    # accumulate + Adam
+
+
+def test_ex_options_rejected_before_launch(L):
+    """Bad options of the _ex calls are refused on the host."""
+    w = q._Weight(0x10000, 0x10000, 0x10000, 256, 256)
+    wp = ctypes.byref(w)
+    bad_flags = q._LinearOpts(1.0, 0x80)
+    nan_scale = q._LinearOpts(float("nan"), 0)
+    acc = q._LinearOpts(2.0, q.QLORA_ACCUMULATE_GRADS)
+    fwd, bwd = L.qlora_linear_fwd_ex, L.qlora_linear_bwd_ex
+    for o in (bad_flags, nan_scale, acc):                                          # acc: no grads in fwd
+        assert fwd(wp, FAKE, 64, FAKE, FAKE, 8, FAKE, None, ctypes.byref(o), FAKE, 1 << 30, None) == 1
+    for o in (bad_flags, nan_scale):
+        assert bwd(wp, FAKE, None, FAKE, 64, FAKE, FAKE, 8, None, FAKE, FAKE, ctypes.byref(o), FAKE, 1 << 30,
+                   None) == 1
+    assert bwd(wp, FAKE, None, FAKE, 64, FAKE, FAKE, 12, None, FAKE, FAKE, ctypes.byref(acc), FAKE, 1 << 30,
+               None) == 2                                                          # r % 8
 
 
 def test_dequant_merge_reject_before_launch(L):

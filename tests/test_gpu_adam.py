@@ -126,3 +126,20 @@ def test_repeated_steps_track_the_oracle():
     A0, B0 = _f64(t["A"]), _f64(t["B"])
     assert_close(_f64(st["A32"]) - A0, ref_A - A0, "A after 3 steps")
     assert_close(_f64(st["B32"]) - B0, ref_B - B0, "B after 3 steps")
+
+
+def test_fused_adam_with_adapter_scale():
+    """The fused step uses the scaled layer's gradients (s = 2)."""
+    t, w = layer_on_gpu(512, 256, 64, 8, tag="adams")
+    Wq = oracle_weight(w)
+    g = linear.backward(t["X"], t["A"], t["B"], Wq, t["dY"], 2.0)
+    st = _prior_state(t["A"], t["B"], g["dA"], g["dB"], "adams")
+    st0 = {k: _f64(v) for k, v in st.items()}
+    ws = q.Workspace()
+    A, B = t["A"].clone(), t["B"].clone()
+    q.qlora_linear_bwd_adam(w, t["X"], None, t["dY"], A, B, st, 5, ws, need_dX=False, adapter_scale=2.0)
+    torch.cuda.synchronize()
+    A1, B1, _ = adam.adapter_adam_step(st0["A32"], st0["B32"], g["dA"], g["dB"],
+                                       {k: st0[k] for k in ("mA", "vA", "mB", "vB")}, 5, lr=1e-3)
+    assert_close(_f64(st["A32"]) - st0["A32"], A1 - st0["A32"], "A step (scaled)")
+    assert_close(_f64(st["B32"]) - st0["B32"], B1 - st0["B32"], "B step (scaled)")

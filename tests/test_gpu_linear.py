@@ -172,3 +172,42 @@ def test_linear_stack_layer_sample():
         t, w = layer_on_gpu(n_in, n_out, 2048, 16, tag=f"stack{i}")
         out = run_fwd_bwd(t, w)
         sampled_check(t, w, out, rows)
+
+
+@pytest.mark.parametrize("M,n_in,n_out,r", [(8, 512, 768, 16), (300, 320, 192, 24)])
+def test_adapter_scale(M, n_in, n_out, r):
+    """Y = X w' + s (X A) B and its backward with s = alpha / r = 2 ("Scaling
+    Factor alpha"), on the small-M and the GEMM paths, against the oracle."""
+    t, w = layer_on_gpu(n_in, n_out, M, r, tag="scale")
+    s = 2.0
+    ws = q.Workspace()
+    Y, V = q.qlora_linear_fwd(w, t["X"], t["A"], t["B"], ws, adapter_scale=s)
+    dX, dA, dB = q.qlora_linear_bwd(w, t["X"], V, t["dY"], t["A"], t["B"], ws, adapter_scale=s)
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+    Wq = oracle_weight(w)
+    Yr, Vr = linear.forward(t["X"], t["A"], t["B"], Wq, s)
+    g = linear.backward(t["X"], t["A"], t["B"], Wq, t["dY"], s)
+    for got, ref, name in ((Y, Yr, "Y"), (V, Vr, "V"), (dX, g["dX"], "dX"), (dA, g["dA"], "dA"), (dB, g["dB"], "dB")):
+        assert_close(got, ref, name)
+
+
+def test_accumulated_gradients():
+    """QLORA_ACCUMULATE_GRADS adds into the given dA and dB (two micro-batches on
+    top of a nonzero start) instead of overwriting them."""
+    t, w = layer_on_gpu(256, 384, 96, 16, tag="acc")
+    t2, _ = layer_on_gpu(256, 384, 96, 16, tag="acc2")
+    ws = q.Workspace()
+    dA0 = synth.normal("acc_dA0", (256, 16), 1.0, device="cuda")
+    dB0 = synth.normal("acc_dB0", (16, 384), 1.0, device="cuda")
+    dA, dB = dA0.clone(), dB0.clone()
+    for tt in (t, t2):
+        _, V = q.qlora_linear_fwd(w, tt["X"], t["A"], t["B"], ws)
+        q.qlora_linear_bwd(w, tt["X"], V, tt["dY"], t["A"], t["B"], ws, need_dX=False, dA=dA, dB=dB,
+                           accumulate=True)
+    torch.cuda.synchronize()
+    Wq = oracle_weight(w)
+    g1 = linear.backward(t["X"], t["A"], t["B"], Wq, t["dY"])
+    g2 = linear.backward(t2["X"], t["A"], t["B"], Wq, t2["dY"])
+    assert_close(dA, dA0.double().cpu().numpy() + g1["dA"] + g2["dA"], "dA accumulated")
+    assert_close(dB, dB0.double().cpu().numpy() + g1["dB"] + g2["dB"], "dB accumulated")

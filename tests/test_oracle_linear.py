@@ -1,6 +1,7 @@
 """Pins of the forward / backward / merge oracle (CPU only)."""
 
 import numpy as np
+import pytest
 import torch
 
 import synth
@@ -64,10 +65,11 @@ def test_backward_factored_equals_dense_form():
     assert np.array_equal(a["dA"], g["dA"]) and np.array_equal(a["dB"], g["dB"])
 
 
-def test_backward_finite_differences():
+@pytest.mark.parametrize("scale", [1.0, 2.5])
+def test_backward_finite_differences(scale):
     """Central differences of L = <dY, Y>: L is linear in each of X, A, B alone,
     so the differences are exact up to rounding (catches a dropped term, a
-    transposed operand or a sign)."""
+    transposed operand, a sign, or the adapter scale missing from one side)."""
     rng = np.random.default_rng(8)
     n_in, n_out, M, r = 64, 64, 16, 8
     X = rng.standard_normal((M, n_in))
@@ -75,10 +77,10 @@ def test_backward_finite_differences():
     B = rng.standard_normal((r, n_out)) * 0.1
     Wq = rng.standard_normal((n_in, n_out)) * 0.02
     dY = rng.standard_normal((M, n_out))
-    g = linear.backward(X, A, B, Wq, dY)
+    g = linear.backward(X, A, B, Wq, dY, scale)
 
     def L(X_, A_, B_):
-        return linear.loss_inner(linear.forward(X_, A_, B_, Wq)[0], dY)
+        return linear.loss_inner(linear.forward(X_, A_, B_, Wq, scale)[0], dY)
 
     h = 0.5
     for name, P in (("dX", X), ("dA", A), ("dB", B)):
@@ -91,6 +93,15 @@ def test_backward_finite_differences():
             argm = {"dX": (Pm, A, B), "dA": (X, Pm, B), "dB": (X, A, Pm)}[name]
             num[idx] = (L(*args) - L(*argm)) / (2 * h)
         assert np.allclose(num, g[name], rtol=1e-9, atol=1e-9), name
+
+
+def test_scale_is_the_forward_of_scaled_adapters():
+    """The scaled layer's output is the plain layer's with A replaced by s A (one
+    of the rescalings "Scaling Factor alpha" calls equivalent)."""
+    t, Wq = _layer()
+    Y_s, _ = linear.forward(t["X"], t["A"], t["B"], Wq, 2.0)
+    Y_1, _ = linear.forward(t["X"], 2.0 * t["A"].double().numpy(), t["B"], Wq)
+    np.testing.assert_allclose(Y_s, Y_1, rtol=1e-12, atol=1e-12)
 
 
 def test_B_zero_gives_zero_dA():
