@@ -220,7 +220,8 @@ QLORA_API qlora_status qlora_linear_bwd_ex(const qlora_nf4_weight* w, const uint
 /*
  * Adam / AdamW on the adapters, fused into the backward ("QLoRA (low-rank adapters
  * on a quantized model)", "The code, line by line": opt = Adam(A + B, lr=lr) is
- * given dA and dB only; "LoRA fine-tuning on GPT-2" trains with AdamW).  The
+ * given dA and dB only; "LoRA and QLoRA: Efficient Fine-Tuning Explained", "A real
+ * run", trains with AdamW).  The
  * rule (Kingma & Ba with bias correction, weight decay decoupled as in AdamW):
  *   theta <- theta (1 - lr wd);  m <- b1 m + (1 - b1) g;  v <- b2 v + (1 - b2) g^2;
  *   theta <- theta - lr (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps)

@@ -5,10 +5,11 @@ TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).
 "QLoRA (low-rank adapters on a quantized model)", "The code, line by line":
 ``opt = Adam(A + B, lr=lr)`` hands the optimizer only the adapter matrices, and
 ``opt.step(...)`` is given dA = dW B^T and dB = A^T dW; the frozen base never
-changes.  The "LoRA fine-tuning on GPT-2" page trains the same way with
-``torch.optim.AdamW(..., lr=1e-3)``.  Neither page prints the update rule, so
-the reading is Adam (Kingma & Ba) with bias correction, in the form torch uses,
-and AdamW's decoupled weight decay applied before the moment step:
+changes.  "LoRA and QLoRA: Efficient Fine-Tuning Explained", "A real run",
+trains the same way with ``torch.optim.AdamW(..., lr=1e-3)``.  Neither page
+prints the update rule, so the reading is Adam (Kingma & Ba) with bias
+correction, in the form torch uses, and AdamW's decoupled weight decay applied
+before the moment step:
 
     theta <- theta * (1 - lr * wd)                    (wd = 0: plain Adam)
     m     <- beta1 m + (1 - beta1) g
