@@ -39,6 +39,13 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+# one Llama-7B decoder layer's projections, in order: q, k, v and o take 4096
+# inputs; gate and up expand to 11008; down projects back.  q, k and v read the
+# same input activations, as do gate and up (the model feeds them one tensor).
+LLAMA7B_LAYER = (("q", 4096, 4096, "attn_in"), ("k", 4096, 4096, "attn_in"), ("v", 4096, 4096, "attn_in"),
+                 ("o", 4096, 4096, "o_in"), ("gate", 4096, 11008, "mlp_in"), ("up", 4096, 11008, "mlp_in"),
+                 ("down", 11008, 4096, "down_in"))
+
 WORKLOADS = {
     # Llama-7B attention projection (the headline configuration)
     "attn4096_m4096_r16": dict(shapes=[(4096, 4096)], M=4096, r=16),
@@ -46,6 +53,11 @@ WORKLOADS = {
     "mlp4096x11008_m8192_r64": dict(shapes=[(4096, 11008), (11008, 4096)], M=8192, r=64),
     # the smallest configuration (launch-bound)
     "linear256_m64_r8": dict(shapes=[(256, 256)], M=64, r=8),
+    # the whole Llama-7B linear stack: 32 layers x 7 projections, 6.48e9 weights
+    # quantised on the device, r = 16 on every linear; one step is the forward
+    # and backward of all 224 linears
+    "llama7b_stack_m2048_r16": dict(shapes=[(a, b) for _, a, b, _ in LLAMA7B_LAYER] * 32, M=2048, r=16,
+                                    layer=LLAMA7B_LAYER, layers=32, steps=20, warmup=3),
 }
 DEFAULT_WORKLOAD = "attn4096_m4096_r16"
 L2_BYTES = 126 * 2 ** 20
@@ -55,17 +67,36 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=2000)
-    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--steps", type=int, default=None, help="timed steps (default: 2000; 20 for the stack)")
+    p.add_argument("--warmup", type=int, default=None, help="warm-up steps (default: 10; 3 for the stack)")
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-rows", action="store_true", help="skip the per-kernel row measurements")
-    p.add_argument("--rows", default="all",
-                   help="comma-separated subset of the rows: quantize, dequantize, merge, gemv, train_step")
+    p.add_argument("--rows", default=None,
+                   help="comma-separated subset of the rows: quantize, dequantize, merge, gemv, train_step "
+                        "(default: all of them; none for the stack, whose quantize pass is always measured)")
     p.add_argument("--rows-only", action="store_true",
                    help="measure only the rows (no headline step); prints {'rows': ...}")
     p.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
-    return p.parse_args()
+    a = p.parse_args()
+    wl = WORKLOADS[a.workload]
+    if a.steps is None:
+        a.steps = wl.get("steps", 2000)
+    if a.warmup is None:
+        a.warmup = wl.get("warmup", 10)
+    if a.rows is None:
+        a.rows = "" if "layer" in wl else "all"
+    return a
+
+
+def workload_config(name):
+    wl = WORKLOADS[name]
+    c = {"workload": name, "M": wl["M"], "r": wl["r"]}
+    if "layer" in wl:
+        c.update(layers=wl["layers"], layer=[f"{n} {a}x{b}" for n, a, b, _ in wl["layer"]])
+    else:
+        c["shapes"] = wl["shapes"]
+    return c
 
 
 def peaks():
@@ -207,12 +238,77 @@ def build_sets(wl, nsets, seed_base):
     return sets
 
 
+def build_stack(wl, seed, pk):
+    """The Llama-7B linear stack as one input set, and its quantize pass.
+
+    Every linear gets its own W0, adapters and output gradient dY; q, k and v
+    share one input X, gate and up another.  All 224 W0 (fp32, 26 GB) are drawn
+    on the device first; the quantize pass quantises each into its NF4 weight,
+    once to build the weights and then twice more timed with CUDA events
+    (identical results), after which the W0 are freed."""
+    import torch
+    import quantized_rank_fine_b200 as q
+    import synth
+    M, r = wl["M"], wl["r"]
+    W0s, plan = [], []
+    for li in range(wl["layers"]):
+        acts = {}
+        for name, n_in, n_out, x_key in wl["layer"]:
+            p = f"stack{li}.{name}:"
+            W0s.append(synth.normal(p + "W0", (n_in, n_out), 0.02, torch.float32, "cuda", seed))
+            if x_key not in acts:
+                acts[x_key] = synth.normal(f"stack{li}.{x_key}:X", (M, n_in), 1.0, torch.bfloat16, "cuda", seed)
+            t = {"X": acts[x_key],
+                 "A": synth.normal(p + "A", (n_in, r), 1.0 / math.sqrt(n_in), torch.bfloat16, "cuda", seed),
+                 "B": synth.normal(p + "B", (r, n_out), 0.01, torch.bfloat16, "cuda", seed),
+                 "dY": synth.normal(p + "dY", (M, n_out), 1.0, torch.bfloat16, "cuda", seed)}
+            out = {
+                "Y": torch.empty((M, n_out), dtype=torch.bfloat16, device="cuda"),
+                "V": torch.empty((M, r), dtype=torch.bfloat16, device="cuda"),
+                "dX": torch.empty((M, n_in), dtype=torch.bfloat16, device="cuda"),
+                "dA": torch.empty((n_in, r), dtype=torch.float32, device="cuda"),
+                "dB": torch.empty((r, n_out), dtype=torch.float32, device="cuda"),
+            }
+            plan.append((t, out))
+    weights = [q.qlora_quantize_nf4(W) for W in W0s]
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(2):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for W, w in zip(W0s, weights):
+            q.qlora_quantize_nf4(W, out=w)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    n = sum(W.numel() for W in W0s)
+    del W0s
+    torch.cuda.empty_cache()
+    ms = min(times)
+    b = sum(a * o * (4 + 0.5 + 1 / 64) + 4 * math.ceil(a * o / 64 / 256) for a, o in wl["shapes"])
+    row = {"ms": ms, "weights": n, "launches": len(weights), "gbs": b / ms / 1e6,
+           "frac_hbm": b / ms / 1e6 / pk["hbm_gbs"],
+           "note": "all 224 W0 of the stack quantised back to back (fp32 in, NF4 codes + absmax codes + "
+                   "scales out); the better of two timed passes"}
+    layers = [(w, t, o) for w, (t, o) in zip(weights, plan)]
+    return [layers], row
+
+
 def set_bytes(wl):
+    """HBM bytes one step of one input set touches at least: NF4 weights, the
+    adapters and their gradients, and the activations (X and dY read, Y and dX
+    written), each distinct activation tensor counted once."""
     M, r = wl["M"], wl["r"]
     tot = 0
     for n_in, n_out in wl["shapes"]:
         n = n_in * n_out
-        tot += n // 2 + n // 64 + 2 * M * (n_in + n_out) * 2 + 2 * r * (n_in + n_out) + 4 * r * (n_in + n_out)
+        tot += n // 2 + n // 64 + 2 * r * (n_in + n_out) + 4 * r * (n_in + n_out)
+        tot += 2 * M * (2 * n_out + n_in)          # dY read, Y written, dX written
+        tot += 2 * M * n_in                        # X read (the stack shares some; below)
+    if "layer" in wl:
+        x_width = {key: n_in for _, n_in, _, key in wl["layer"]}      # one X per key
+        counted = sum(n_in for _, n_in, _, _ in wl["layer"])
+        tot -= 2 * M * (counted - sum(x_width.values())) * wl["layers"]
     return tot
 
 
@@ -229,6 +325,8 @@ ROW_NAMES = ("quantize", "dequantize", "merge", "gemv", "train_step")
 def time_rows(wl, pk, which="all"):
     """Per-kernel measurements of the other rows of the path (one GPU); `which`
     is "all" or a comma-separated subset of ROW_NAMES."""
+    if not which:
+        return {}
     want = set(ROW_NAMES) if which == "all" else set(which.split(","))
     unknown = want - set(ROW_NAMES)
     if unknown:
@@ -433,8 +531,14 @@ def arm_ours(args, world, rank, local):
     wl = WORKLOADS[args.workload]
     pk, pk_src = peaks()
     M, r = wl["M"], wl["r"]
-    nsets = max(2, math.ceil(3 * L2_BYTES / set_bytes(wl)))
-    sets = build_sets(wl, nsets, seed_base=100 * rank)
+    quantize_pass = None
+    if "layer" in wl:
+        # one set of the stack streams 23 GB per step: nothing stays in L2
+        sets, quantize_pass = build_stack(wl, 100 * rank, pk)
+        nsets = 1
+    else:
+        nsets = max(2, math.ceil(3 * L2_BYTES / set_bytes(wl)))
+        sets = build_sets(wl, nsets, seed_base=100 * rank)
     ws = q.Workspace()
     nl = len(wl["shapes"])
 
@@ -534,14 +638,16 @@ def arm_ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded; W0 ~ N(0,0.02) fp32 quantised on device, X/dY ~ N(0,1) bf16)",
-        "config": {"workload": args.workload, "M": M, "shapes": wl["shapes"], "r": r,
+        "config": {**workload_config(args.workload),
                    "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": f"{nsets} rotating input sets of {set_bytes(wl) / 2**20:.0f} MiB each (> L2 per cycle)"},
+                   "l2": f"{nsets} rotating input sets of {set_bytes(wl) / 2**20:.0f} MiB each (> L2 per cycle)"
+                   if nsets > 1 else f"one input set of {set_bytes(wl) / 2**30:.1f} GiB per step (> L2)"},
         "tflops": step_flops * args.steps * world / (ms / 1e3) / 1e12,
         "roofline": {"kernel": "nf4_gemm_kernel<fwd> (fused dequant GEMM, tcgen05)", "bound": "tensor",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{pk_src} {'burst' if timed_s < 2.0 else 'sustained'} bf16",
-                     "flops_per_launch": gemm_flops[0] if nl == 1 else gemm_flops[:nl],
+                     "flops_per_launch": gemm_flops[0] if nl == 1 else
+                     {f"{a}x{b}": flops_fwd_gemm(a, b, M, r) for a, b in wl["shapes"]},
                      "mean_launch_ms": statistics.mean(gemm_ms), "traffic": traffic},
         "gpu_launches": launches,
         "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"],
@@ -553,6 +659,12 @@ def arm_ours(args, world, rank, local):
 
     if world == 1 and not args.no_rows:
         line["rows"] = time_rows(wl, pk, args.rows)
+    if quantize_pass is not None:
+        # per GPU (each rank quantises its own replica of the stack); slowest rank
+        slow = max_over_ranks(quantize_pass["ms"], world) / quantize_pass["ms"]
+        quantize_pass.update(ms=quantize_pass["ms"] * slow, gbs=quantize_pass["gbs"] / slow,
+                             frac_hbm=quantize_pass["frac_hbm"] / slow)
+        line.setdefault("rows", {})["quantize_pass"] = quantize_pass
     if world == 1 and rank == 0 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(args.workload, budget_s=20.0)
     return line
@@ -564,27 +676,28 @@ def e2e(args, sets, ws, wl, world):
     import torch
     M = wl["M"]
     nsets = len(sets)
-    host = []
+    host = []          # per set: ([(device input, pinned host copy)], [(device gradient, pinned host buffer)])
     for layers in sets:
-        hl = []
+        ins, seen = [], set()
         for w, t, o in layers:
-            hl.append({"X": t["X"].cpu().pin_memory(), "dY": t["dY"].cpu().pin_memory(),
-                       "dA": torch.empty(o["dA"].shape, dtype=torch.float32).pin_memory(),
-                       "dB": torch.empty(o["dB"].shape, dtype=torch.float32).pin_memory()})
-        host.append(hl)
-    h2d = sum(h["X"].numel() * 2 + h["dY"].numel() * 2 for h in host[0])
-    d2h = sum(h["dA"].numel() * 4 + h["dB"].numel() * 4 for h in host[0])
-    steps = max(10, args.steps // 4)
+            for d in (t["X"], t["dY"]):
+                if d.data_ptr() not in seen:      # the stack's shared activations are copied once
+                    seen.add(d.data_ptr())
+                    ins.append((d, torch.empty(d.shape, dtype=d.dtype, pin_memory=True).copy_(d)))
+        outs = [(o[k], torch.empty(o[k].shape, dtype=torch.float32).pin_memory())
+                for w, t, o in layers for k in ("dA", "dB")]
+        host.append((ins, outs))
+    h2d = sum(d.numel() * d.element_size() for d, _ in host[0][0])
+    d2h = sum(d.numel() * d.element_size() for d, _ in host[0][1])
+    steps = 10 if "layer" in wl else max(10, args.steps // 4)
 
     def step(i):
-        layers, hl = sets[i % nsets], host[i % nsets]
-        for (w, t, o), h in zip(layers, hl):
-            t["X"].copy_(h["X"], non_blocking=True)
-            t["dY"].copy_(h["dY"], non_blocking=True)
-        run_step(layers, ws)
-        for (w, t, o), h in zip(layers, hl):
-            h["dA"].copy_(o["dA"], non_blocking=True)
-            h["dB"].copy_(o["dB"], non_blocking=True)
+        ins, outs = host[i % nsets]
+        for d, h in ins:
+            d.copy_(h, non_blocking=True)
+        run_step(sets[i % nsets], ws)
+        for d, h in outs:
+            h.copy_(d, non_blocking=True)
 
     for i in range(3):
         step(i)
@@ -622,13 +735,15 @@ def oracle_cores():
 def oracle_inputs(workload, rows_frac, tokens):
     """Oracle inputs of a bounded sample: the first rows_frac of each weight's
     input rows (whole double-quant groups) and `tokens` tokens, quantised by the
-    oracle itself."""
+    oracle itself.  For the stack the sample is one decoder layer's seven
+    projections (all 32 layers have the same shapes)."""
     import synth
     from oracle import nf4
     wl = WORKLOADS[workload]
     r = wl["r"]
+    shapes = [(a, b) for _, a, b, _ in wl["layer"]] if "layer" in wl else wl["shapes"]
     layers = []
-    for li, (n_in, n_out) in enumerate(wl["shapes"]):
+    for li, (n_in, n_out) in enumerate(shapes):
         rows_per_group = max(1, (64 * 256) // n_out)
         n_rows = max(rows_per_group, int(n_in * rows_frac) // rows_per_group * rows_per_group)
         t = synth.layer_inputs(n_rows, n_out, tokens, r, tag=f"oracle{li}:")
@@ -661,8 +776,14 @@ def oracle_sample_time(workload, budget_s):
         if dt * 2 > budget_s or frac >= 1.0:
             break
         frac = min(1.0, frac * 2)
-    row_frac = sum(l[2] for l in layers) / sum(l[4] for l in layers)
+    # the sampled share of the whole step's work (work ~ rows x columns x tokens)
+    row_frac = sum(l[2] * l[3] for l in layers) / sum(l[4] * l[3] for l in layers) / wl.get("layers", 1)
     return layers, dt, row_frac, tokens
+
+
+def sample_layers(workload):
+    wl = WORKLOADS[workload]
+    return f" (of the whole stack: one layer's 7 projections, x {wl['layers']} layers)" if "layer" in wl else ""
 
 
 def cpu_baseline(workload, budget_s=20.0):
@@ -675,10 +796,11 @@ def cpu_baseline(workload, budget_s=20.0):
         oracle_step(layers)
         ts.append(time.perf_counter() - t0)
     dt = statistics.median(ts)
-    value = tokens * row_frac / dt   # tokens/s of the full layer (work scales with the weight rows)
+    value = tokens * row_frac / dt   # tokens/s of the full step (work scales with the weights' size)
     return {"value": value, "unit": "tokens/s", "cores": used, "kind": "oracle",
-            "sample": f"float64 oracle fwd+bwd incl. dequantisation, {tokens} tokens x {row_frac:.4f} of each "
-                      f"weight's input rows, median of {len(ts)} runs, scaled to the full layer"}
+            "sample": f"float64 oracle fwd+bwd incl. dequantisation: {tokens} tokens through the leading input "
+                      f"rows of each weight{sample_layers(workload)}, {row_frac:.5f} of the step's weights; "
+                      f"median of {len(ts)} runs, scaled to the full step"}
 
 
 def arm_reference(args, world, rank):
@@ -696,13 +818,14 @@ def arm_reference(args, world, rank):
     dt = time.perf_counter() - t0
     cores, used = oracle_cores()
     value = tokens * row_frac * args.steps / dt
-    sample = (f"float64 oracle fwd+bwd incl. dequantisation, per step {tokens} tokens x {row_frac:.4f} of each "
-              f"weight's input rows, scaled to the full layer")
+    sample = (f"float64 oracle fwd+bwd incl. dequantisation, per step {tokens} tokens through the leading "
+              f"input rows of each weight{sample_layers(args.workload)}, {row_frac:.5f} of the step's weights; "
+              f"scaled to the full step")
     return {
         "impl": "reference", "metric": "QLoRA linear fwd+bwd tokens/s", "value": value, "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "M": wl["M"], "shapes": wl["shapes"], "r": wl["r"]},
+        "config": workload_config(args.workload),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": used, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }

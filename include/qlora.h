@@ -276,14 +276,25 @@ QLORA_API qlora_status qlora_merge(const qlora_nf4_weight* w, const uint16_t* A,
 
 /* ---------------------------------------------------------------- helpers */
 
-/* Bytes of workspace qlora_linear_fwd / qlora_linear_bwd need for these sizes
- * (0 for an unknown op or invalid sizes).  Host only, no device access. */
+/* Bytes of workspace qlora_linear_fwd / qlora_linear_bwd use at these sizes on
+ * the current device (0 for an unknown op or invalid sizes).  Host only: it reads
+ * the device's SM count, no device memory.
+ * Layout: a 1280-byte prefix (the 256-byte status word, then 1 KB of counters
+ * of the fused dequant GEMM); V (M x r bf16, rounded up to 256 bytes); for the
+ * backward U (the same size); then the GEMM's partial tiles: when the layer's
+ * 256 x 256 output tiles do not divide evenly over the SMs, the K-steps of the
+ * last tiles are shared between CTAs, which hand over one 256 KB fp32 partial
+ * tile per SM.  A workspace that stops before the partial tiles is accepted too:
+ * the GEMM then keeps every tile whole (slower by up to one wave of tiles). */
 QLORA_API size_t qlora_workspace_bytes(int op, int64_t M, int64_t in, int64_t out, int r);
 
-/* Zero the whole workspace (once, before its first use).  Its first 256 bytes
- * hold a status word that the kernels set when a bounded wait gives up and
- * qlora_ws_status() clears; the rest is scratch (V, U) that every call rewrites.
- * Calls that share one workspace must be ordered on one stream. */
+/* Zero the whole workspace (once, before its first use; QLORA_ERR_WORKSPACE if
+ * it is shorter than the 1280-byte prefix).  Its first 256 bytes hold a status
+ * word that the kernels set when a bounded wait gives up and qlora_ws_status()
+ * clears; the GEMM's counters after it are zero again whenever a call's kernels
+ * end; the rest is scratch (V, U, partial tiles) that every call rewrites.
+ * Forward and backward calls of any sizes may share one workspace (the prefix
+ * has one layout), but calls that share one must be ordered on one stream. */
 QLORA_API qlora_status qlora_ws_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronise `stream`, then report QLORA_ERR_TIMEOUT if a bounded wait in a
@@ -317,6 +328,13 @@ typedef enum qlora_kernel {
  * in a CUDA graph.  n = 0 disarms.  Process-wide state; not for concurrent callers.
  * Returns QLORA_ERR_INVALID_ARG for an unknown kernel or NULL arrays with n > 0. */
 QLORA_API qlora_status qlora_time_kernel(int which, void* const* starts, void* const* stops, int n);
+
+/* Most CTAs the fused dequant GEMMs use (0, the default: one per SM; larger
+ * values are capped at the SM count).  A testing and tuning knob: a small count
+ * makes small layers exercise the shared-K-step schedule.  Process-wide; takes
+ * effect for calls (and workspace sizes) after it.  QLORA_ERR_INVALID_ARG if
+ * ctas < 0. */
+QLORA_API qlora_status qlora_gemm_set_ctas(int ctas);
 
 /* Number of kernel launches libqlora has issued in this process. */
 QLORA_API uint64_t qlora_launch_count(void);

@@ -36,6 +36,7 @@ EXPORTS = (
     "qlora_workspace_bytes", "qlora_ws_init", "qlora_ws_status", "qlora_nf4_codebook",
     "qlora_adapter_params", "qlora_status_string", "qlora_time_kernel", "qlora_launch_count",
     "qlora_linear_fwd_static_ws", "qlora_linear_bwd_adam", "qlora_linear_fwd_ex", "qlora_linear_bwd_ex",
+    "qlora_gemm_set_ctas",
 )
 
 # Flag of qlora_linear_opts.flags.
@@ -96,6 +97,7 @@ def lib() -> ctypes.CDLL:
             "qlora_status_string": (ctypes.c_char_p, [i32]),
             "qlora_time_kernel": (i32, [i32, ctypes.POINTER(vp), ctypes.POINTER(vp), i32]),
             "qlora_launch_count": (ctypes.c_uint64, []),
+            "qlora_gemm_set_ctas": (i32, [i32]),
             "qlora_linear_fwd_static_ws": (i32, [wp, vp, i64, vp, vp, i32, vp, vp, vp]),
             "qlora_linear_bwd_adam": (i32, [wp, vp, vp, vp, i64, vp, vp, i32, vp, ctypes.POINTER(_AdamState),
                                             ctypes.POINTER(_AdamHparams), ctypes.POINTER(_LinearOpts), vp, sz,
@@ -162,6 +164,11 @@ def qlora_status_string(status: int) -> str:
 
 def qlora_launch_count() -> int:
     return lib().qlora_launch_count()
+
+
+def qlora_gemm_set_ctas(ctas: int) -> None:
+    """Most CTAs the fused GEMMs use (0: one per SM); a testing/tuning knob."""
+    _check(lib().qlora_gemm_set_ctas(ctas), "qlora_gemm_set_ctas")
 
 
 class KernelTimer:

@@ -15,7 +15,6 @@ using qlora::WeightView;
 
 namespace {
 
-constexpr size_t kStatusBytes = 256;
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -89,29 +88,52 @@ qlora_status check_weight(const qlora_nf4_weight* w) {
 WeightView view(const qlora_nf4_weight* w) { return WeightView{w->codes, w->dq_codes, w->dq_scales, w->in, w->out}; }
 
 // Workspace layout (byte offsets), shared by the size query and the calls:
-// the status prefix, V (when the caller does not keep it) and U (backward).
+// the fixed prefix (status word, the GEMM's split counters), V (when the
+// caller does not keep it), U (backward), and last the fused GEMM's partial
+// tiles for the tiles whose K-steps several CTAs share.  A smaller workspace
+// may leave the partial tiles out: the GEMM then keeps every tile whole.
 struct WsLayout {
-  size_t v_off, u_off, total;
+  size_t v_off, u_off, part_off, min_total, total;
 };
 
 constexpr size_t kFixedBytes = qlora::kWsFixedBytes;
 
 WsLayout ws_layout(int op, int64_t M, int64_t in, int64_t out, int r) {
-  (void)in;
-  (void)out;
   WsLayout L{};
   const size_t mr = align256(static_cast<size_t>(M) * r * 2);
   size_t off = kFixedBytes;
   L.v_off = off;
   off += mr;
+  size_t part = 0;
   if (op == QLORA_OP_FWD) {
     L.u_off = 0;
+    if (!qlora::gemv_supported(M, in, out)) part = qlora::fwd_gemm_split_bytes(M, in, out, r);
   } else {
     L.u_off = off;
     off += mr;
+    part = qlora::dx_gemm_split_bytes(M, in, out, r);
   }
-  L.total = off;
+  L.part_off = off;
+  L.min_total = off;
+  L.total = off + align256(part);
   return L;
+}
+
+struct SplitRegion {
+  uint32_t* counters;
+  void* partials;
+  size_t partial_bytes;
+};
+
+// The GEMM's hand-over buffers: the partial tiles only in a full-size workspace.
+SplitRegion split_region(void* ws, size_t ws_bytes, const WsLayout& L) {
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  SplitRegion R{reinterpret_cast<uint32_t*>(base + qlora::kWsStatusBytes), nullptr, 0};
+  if (ws_bytes >= L.total && L.total > L.min_total) {
+    R.partials = base + L.part_off;
+    R.partial_bytes = ws_bytes - L.part_off;
+  }
+  return R;
 }
 
 std::atomic<uint64_t> g_launches{0};
@@ -126,6 +148,10 @@ struct TimingHook {
 }  // namespace
 
 namespace qlora {
+size_t ws_min_bytes(int op, int64_t M, int64_t in, int64_t out, int r) {
+  if ((op != QLORA_OP_FWD && op != QLORA_OP_BWD) || !linear_shape_ok(M, in, out, r)) return 0;
+  return ws_layout(op, M, in, out, r).min_total;
+}
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 // Record `e` on `stream`; inside a stream capture as an external event node, so
 // that it is recorded at every replay of the graph.
@@ -188,8 +214,14 @@ size_t qlora_workspace_bytes(int op, int64_t M, int64_t in, int64_t out, int r) 
   return ws_layout(op, M, in, out, r).total;
 }
 
+qlora_status qlora_gemm_set_ctas(int ctas) {
+  if (ctas < 0) return QLORA_ERR_INVALID_ARG;
+  qlora::set_gemm_ctas(ctas);
+  return QLORA_OK;
+}
+
 qlora_status qlora_ws_init(void* ws, size_t ws_bytes, void* stream) {
-  if (!ws || ws_bytes < kStatusBytes) return QLORA_ERR_WORKSPACE;
+  if (!ws || ws_bytes < qlora::kWsFixedBytes) return QLORA_ERR_WORKSPACE;
   QLORA_TRY(check_device());
   QLORA_TRY(check_ptr(ws));
   QLORA_CUDA(cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)));
@@ -256,7 +288,7 @@ static qlora_status fwd_impl(const qlora_nf4_weight* w, const uint16_t* X, int64
   if (!X || !A || !B || !Y) return QLORA_ERR_INVALID_ARG;
   QLORA_TRY(check_weight_shape(w));
   if (!linear_shape_ok(M, w->in, w->out, r)) return QLORA_ERR_SHAPE;
-  if (!ws || ws_bytes < ws_layout(QLORA_OP_FWD, M, w->in, w->out, r).total) return QLORA_ERR_WORKSPACE;
+  if (!ws || ws_bytes < ws_layout(QLORA_OP_FWD, M, w->in, w->out, r).min_total) return QLORA_ERR_WORKSPACE;
   QLORA_TRY(check_device());
   QLORA_TRY(check_weight(w));
   QLORA_TRY(check_ptr(X));
@@ -265,7 +297,7 @@ static qlora_status fwd_impl(const qlora_nf4_weight* w, const uint16_t* X, int64
   QLORA_TRY(check_ptr(Y));
   QLORA_TRY(check_ptr(V_save, false));
   const WsLayout L = ws_layout(QLORA_OP_FWD, M, w->in, w->out, r);
-  if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  if (!ws || ws_bytes < L.min_total) return QLORA_ERR_WORKSPACE;
   QLORA_TRY(check_ptr(ws));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
@@ -277,7 +309,8 @@ static qlora_status fwd_impl(const qlora_nf4_weight* w, const uint16_t* X, int64
     QLORA_CUDA(qlora::launch_gemv(wv, X, V, B, M, r, Y, status, s));
   } else {
     QLORA_CUDA(qlora::launch_xa(X, A, M, w->in, r, V, status, s, scale));
-    QLORA_CUDA(qlora::launch_fwd_gemm(wv, X, V, B, M, r, Y, status, s));
+    const SplitRegion sr = split_region(ws, ws_bytes, L);
+    QLORA_CUDA(qlora::launch_fwd_gemm(wv, X, V, B, M, r, Y, status, sr.counters, sr.partials, sr.partial_bytes, s));
   }
   return QLORA_OK;
 }
@@ -316,7 +349,7 @@ static qlora_status bwd_impl(const qlora_nf4_weight* w, const uint16_t* X, const
   if (!X || !dY || !A || !B || !dA || !dB) return QLORA_ERR_INVALID_ARG;
   QLORA_TRY(check_weight_shape(w));
   if (!linear_shape_ok(M, w->in, w->out, r)) return QLORA_ERR_SHAPE;
-  if (!ws || ws_bytes < ws_layout(QLORA_OP_BWD, M, w->in, w->out, r).total) return QLORA_ERR_WORKSPACE;
+  if (!ws || ws_bytes < ws_layout(QLORA_OP_BWD, M, w->in, w->out, r).min_total) return QLORA_ERR_WORKSPACE;
   QLORA_TRY(check_device());
   QLORA_TRY(check_weight(w));
   QLORA_TRY(check_ptr(X));
@@ -328,7 +361,7 @@ static qlora_status bwd_impl(const qlora_nf4_weight* w, const uint16_t* X, const
   QLORA_TRY(check_ptr(dA));
   QLORA_TRY(check_ptr(dB));
   const WsLayout L = ws_layout(QLORA_OP_BWD, M, w->in, w->out, r);
-  if (!ws || ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  if (!ws || ws_bytes < L.min_total) return QLORA_ERR_WORKSPACE;
   QLORA_TRY(check_ptr(ws));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
@@ -343,7 +376,10 @@ static qlora_status bwd_impl(const qlora_nf4_weight* w, const uint16_t* X, const
   QLORA_CUDA(qlora::launch_dybt(dY, B, M, w->out, r, U, status, s, scale));
   QLORA_CUDA(qlora::launch_vtdy(V, dY, M, w->out, r, dB, status, s, nullptr, accumulate));
   QLORA_CUDA(qlora::launch_xtu(X, U, M, w->in, r, dA, status, s, nullptr, accumulate));
-  if (dX) QLORA_CUDA(qlora::launch_dx_gemm(wv, dY, U, A, M, r, dX, status, s));
+  if (dX) {
+    const SplitRegion sr = split_region(ws, ws_bytes, L);
+    QLORA_CUDA(qlora::launch_dx_gemm(wv, dY, U, A, M, r, dX, status, sr.counters, sr.partials, sr.partial_bytes, s));
+  }
   return QLORA_OK;
 }
 
@@ -377,7 +413,7 @@ qlora_status qlora_linear_bwd_adam(const qlora_nf4_weight* w, const uint16_t* X,
     return QLORA_ERR_INVALID_ARG;
   QLORA_TRY(check_weight_shape(w));
   if (!linear_shape_ok(M, w->in, w->out, r)) return QLORA_ERR_SHAPE;
-  if (!ws || ws_bytes < ws_layout(QLORA_OP_BWD, M, w->in, w->out, r).total) return QLORA_ERR_WORKSPACE;
+  if (!ws || ws_bytes < ws_layout(QLORA_OP_BWD, M, w->in, w->out, r).min_total) return QLORA_ERR_WORKSPACE;
   QLORA_TRY(check_device());
   QLORA_TRY(check_weight(w));
   QLORA_TRY(check_ptr(X));
@@ -427,7 +463,10 @@ qlora_status qlora_linear_bwd_adam(const qlora_nf4_weight* w, const uint16_t* X,
   }
   QLORA_CUDA(qlora::launch_dybt(dY, B, M, w->out, r, U, status, s, scale));
   QLORA_CUDA(qlora::launch_vtdy(V, dY, M, w->out, r, nullptr, status, s, &pB));
-  if (dX) QLORA_CUDA(qlora::launch_dx_gemm(wv, dY, U, A, M, r, dX, status, s));
+  if (dX) {
+    const SplitRegion sr = split_region(ws, ws_bytes, L);
+    QLORA_CUDA(qlora::launch_dx_gemm(wv, dY, U, A, M, r, dX, status, sr.counters, sr.partials, sr.partial_bytes, s));
+  }
   QLORA_CUDA(qlora::launch_xtu(X, U, M, w->in, r, nullptr, status, s, &pA));
   return QLORA_OK;
 }

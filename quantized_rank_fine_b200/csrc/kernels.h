@@ -12,10 +12,15 @@ namespace qlora {
 
 constexpr int kMaxSplits = 16;   // most K/M splits of the rank-r kernels
 
-// Workspace prefix shared by every call: the status word(s), which must start
-// at zero (the only part of a workspace that needs initialising).
+// Workspace prefix shared by every call, which must start at zero (the only
+// part of a workspace that needs initialising): the status word(s), then the
+// counters of the fused GEMM's split tiles (one per CTA, left zero by every
+// launch).  The prefix has the same layout for every call, so calls of
+// different kinds can share a workspace.
 constexpr size_t kWsStatusBytes = 256;
-constexpr size_t kWsFixedBytes = kWsStatusBytes;
+constexpr int kMaxGemmCtas = 256;
+constexpr size_t kWsCounterBytes = kMaxGemmCtas * sizeof(uint32_t);
+constexpr size_t kWsFixedBytes = kWsStatusBytes + kWsCounterBytes;
 
 // Bookkeeping of the measurement helpers (defined in api.cu): every kernel
 // launch is counted; an armed timing hook brackets launches of one kernel kind.
@@ -76,10 +81,25 @@ cudaError_t launch_xa_small(const uint16_t* X, const uint16_t* A, int64_t M, int
 cudaError_t launch_gemv(const WeightView& w, const uint16_t* X, const uint16_t* V, const uint16_t* B, int64_t M,
                         int r, uint16_t* Y, uint32_t* status, cudaStream_t stream);
 
-// Fused dequant GEMMs (tcgen05); `status` is the workspace status word.
+// Fused dequant GEMMs (tcgen05, persistent grid); `status` is the workspace
+// status word.  When the tile count does not divide evenly over the CTAs the
+// K-steps of the last tiles are shared between CTAs: `counters` (the
+// workspace's kMaxGemmCtas counters, zero) and `partials` (one 256 x 256 fp32
+// tile per CTA, *_gemm_split_bytes) hold their hand-over.  With partials ==
+// nullptr, or fewer bytes, every tile stays whole.
 cudaError_t launch_fwd_gemm(const WeightView& w, const uint16_t* X, const uint16_t* V, const uint16_t* B,
-                            int64_t M, int r, uint16_t* Y, uint32_t* status, cudaStream_t stream);
+                            int64_t M, int r, uint16_t* Y, uint32_t* status, uint32_t* counters,
+                            void* partials, size_t partial_bytes, cudaStream_t stream);
 cudaError_t launch_dx_gemm(const WeightView& w, const uint16_t* dY, const uint16_t* U, const uint16_t* A,
-                           int64_t M, int r, uint16_t* dX, uint32_t* status, cudaStream_t stream);
+                           int64_t M, int r, uint16_t* dX, uint32_t* status, uint32_t* counters,
+                           void* partials, size_t partial_bytes, cudaStream_t stream);
+size_t fwd_gemm_split_bytes(int64_t M, int64_t n_in, int64_t n_out, int r);
+size_t dx_gemm_split_bytes(int64_t M, int64_t n_in, int64_t n_out, int r);
+// Most CTAs the GEMMs use (0: one per SM); a testing and tuning knob.
+void set_gemm_ctas(int ctas);
+
+// Smallest workspace a forward/backward call accepts (no split tiles); the
+// size qlora_workspace_bytes returns also holds the split region.
+size_t ws_min_bytes(int op, int64_t M, int64_t in, int64_t out, int r);
 
 }  // namespace qlora

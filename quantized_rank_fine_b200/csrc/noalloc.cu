@@ -58,7 +58,9 @@ extern "C" qlora_status qlora_linear_fwd_static_ws(const qlora_nf4_weight* w, co
                                                    const uint16_t* A, const uint16_t* B, int r, uint16_t* Y,
                                                    uint16_t* V_save, void* stream) {
   if (!w) return QLORA_ERR_INVALID_ARG;
-  const size_t need = qlora_workspace_bytes(QLORA_OP_FWD, M, w->in, w->out, r);
+  // the smallest workspace the forward accepts: the GEMM keeps its tiles whole
+  // (the split region would not fit the fixed array at the usual sizes)
+  const size_t need = qlora::ws_min_bytes(QLORA_OP_FWD, M, w->in, w->out, r);
   if (need == 0) return QLORA_ERR_SHAPE;
   if (need > kStaticWsBytes) return QLORA_ERR_WORKSPACE;   // larger than the fixed array
   void* ws = nullptr;
@@ -66,5 +68,5 @@ extern "C" qlora_status qlora_linear_fwd_static_ws(const qlora_nf4_weight* w, co
   if (st != QLORA_OK) return st;
   if (cudaMemsetAsync(ws, 0, qlora::kWsFixedBytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return QLORA_ERR_CUDA;
-  return qlora_linear_fwd(w, X, M, A, B, r, Y, V_save, ws, kStaticWsBytes, stream);
+  return qlora_linear_fwd(w, X, M, A, B, r, Y, V_save, ws, need, stream);
 }

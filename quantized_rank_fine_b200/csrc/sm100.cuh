@@ -116,6 +116,17 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
 }
 
+// Arrive on a barrier of a cluster peer (shared::cluster address from mapa)
+// with the default semantics, release at CTA scope.  This is how the pair MMA's
+// operand producers publish a stage: the data lies in the arriving CTA's own
+// shared memory (made visible to the tensor core by fence.proxy.async before
+// the arrive), or is TMEM the arriving CTA has finished reading.  Much cheaper
+// than a cluster-scope release, which waits for all of the thread's
+// outstanding memory operations.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
@@ -174,6 +185,44 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
 __device__ __forceinline__ void umma_commit_multicast(uint32_t bar, uint16_t cta_mask) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(cta_mask)
+      : "memory");
+}
+
+// ---------------------------------------------------------------- CTA pairs (cta_group::2)
+//
+// Two CTAs of a cluster whose ranks differ only in bit 0 act as one MMA unit:
+// an MMA issued by one of them reads its A rows and B columns from both CTAs'
+// shared memory (same offsets) and writes each CTA's rows into that CTA's TMEM.
+
+// Both CTAs' warps with the same warp index allocate the same TMEM columns.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols));
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::);
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
+}
+
+// D[tmem of both CTAs] (+)= A * B^T for M = 256 rows split 128 per CTA, N split
+// N/2 per CTA; descriptors give the (common) shared-memory offsets.
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on the barrier at this shared-memory offset in every CTA of `cta_mask`
+// once all pair MMAs issued so far by this thread have completed.
+__device__ __forceinline__ void umma_commit_pair_multicast(uint32_t bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
       "h"(cta_mask)
       : "memory");
 }
@@ -278,6 +327,37 @@ __device__ __forceinline__ float4 ld_shared_cluster_v4(uint32_t addr) {
                : "r"(addr)
                : "memory");
   return v;
+}
+
+// ---------------------------------------------------------------- counters in global memory
+
+// Add to a counter with release semantics at GPU scope: the calling thread's
+// earlier writes (and those it has observed) are visible to a thread that
+// acquires the new value.
+__device__ __forceinline__ void red_release_gpu_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Wait until *p >= target (acquire); false after the wait limit, with the flag
+// raised in the status word.
+__device__ __forceinline__ bool wait_counter(const uint32_t* p, uint32_t target, uint32_t* status,
+                                             uint32_t flag) {
+  if (ld_acquire_gpu(p) >= target) return true;
+  const uint64_t t0 = global_timer();
+  while (ld_acquire_gpu(p) < target) {
+    __nanosleep(128);
+    if (global_timer() - t0 > kWaitLimitNs) {
+      raise_flag(status, flag);
+      return false;
+    }
+  }
+  return true;
 }
 
 // ---------------------------------------------------------------- dependent launches

@@ -77,3 +77,15 @@ def run_fwd_bwd(t, w, ws=None, need_dX=True):
     torch.cuda.synchronize()
     assert ws.status() == 0, "a kernel wait timed out"
     return {"Y": Y, "V": V, "dX": dX, "dA": dA, "dB": dB}
+
+
+def full_check(t, w, out):
+    """Every output of one forward + backward against the oracle on the same bytes."""
+    Wq = oracle_weight(w)
+    Y, V = linear.forward(t["X"], t["A"], t["B"], Wq)
+    g = linear.backward(t["X"], t["A"], t["B"], Wq, t["dY"])
+    assert_close(out["Y"], Y, "Y")
+    assert_close(out["V"], V, "V")
+    assert_close(out["dX"], g["dX"], "dX")
+    assert_close(out["dA"], g["dA"], "dA")
+    assert_close(out["dB"], g["dB"], "dB")

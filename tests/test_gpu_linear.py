@@ -9,7 +9,7 @@ import torch
 import quantized_rank_fine_b200 as q
 import synth
 from oracle import linear
-from tests.helpers import assert_close, layer_on_gpu, oracle_weight, require_gpu, run_fwd_bwd
+from tests.helpers import assert_close, full_check, layer_on_gpu, oracle_weight, require_gpu, run_fwd_bwd
 
 pytestmark = pytest.mark.gpu
 
@@ -17,17 +17,6 @@ pytestmark = pytest.mark.gpu
 @pytest.fixture(scope="module", autouse=True)
 def _gpu():
     require_gpu()
-
-
-def full_check(t, w, out):
-    Wq = oracle_weight(w)
-    Y, V = linear.forward(t["X"], t["A"], t["B"], Wq)
-    g = linear.backward(t["X"], t["A"], t["B"], Wq, t["dY"])
-    assert_close(out["Y"], Y, "Y")
-    assert_close(out["V"], V, "V")
-    assert_close(out["dX"], g["dX"], "dX")
-    assert_close(out["dA"], g["dA"], "dA")
-    assert_close(out["dB"], g["dB"], "dB")
 
 
 def test_linear_256_m64_r8_full():
