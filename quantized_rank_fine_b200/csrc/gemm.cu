@@ -375,28 +375,30 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
         valid = (nh + nr) < p.N;
         blk = (nh + nr) * blocks_per_row;
       }
-      // absmax codes and scales, two K-steps ahead
-      uint8_t dqc0 = 0, dqc1 = 0;
-      float dqs0 = 0.0f, dqs1 = 0.0f;
+      // Absmax code and scale of a K-step, loaded two K-steps ahead into one of
+      // two register slots; the loop is unrolled by two so that a slot is
+      // consumed and refilled in place (moving a pending load's register to
+      // another would wait for the load one step early).
+      uint8_t dqcA = 0, dqcB = 0;
+      float dqsA = 0.0f, dqsB = 0.0f;
       if (valid && w.kb0 < nkb_w) {
         const int64_t b0 = blk + w.kb0 * blk_step;
-        dqc0 = __ldg(p.dq_codes + b0);
-        dqs0 = __ldg(p.dq_scales + b0 / kGroup);
+        dqcA = __ldg(p.dq_codes + b0);
+        dqsA = __ldg(p.dq_scales + b0 / kGroup);
       }
       if (valid && w.kb0 + 1 < nkb_w) {
         const int64_t b1 = blk + (w.kb0 + 1) * blk_step;
-        dqc1 = __ldg(p.dq_codes + b1);
-        dqs1 = __ldg(p.dq_scales + b1 / kGroup);
+        dqcB = __ldg(p.dq_codes + b1);
+        dqsB = __ldg(p.dq_scales + b1 / kGroup);
       }
-      for (int kb = w.kb0; kb < w.kb1; ++kb, ++g) {
+      // one K-step with the absmax in (dqc, dqs); refills them for kb + 2
+      auto step = [&](int kb, uint8_t& dqc, float& dqs) -> bool {
         const int s = g % kStages;
         const uint32_t ph = (g / kStages) & 1;
+        ++g;
         // every lane waits; the warp leaves the loop together if the wait gave up
         const bool got = mbar_wait(loaded0 + 8 * s, ph, p.status, kFlagTimeoutProducer);
-        if (!__all_sync(0xffffffffu, got)) {
-          alive = false;
-          break;
-        }
+        if (!__all_sync(0xffffffffu, got)) return false;
         if (kb < nkb_w) {
           const uint32_t stage = smem_addr(smem + s * kStageBytes);
           const uint32_t dst = stage + kABytes + row_off;
@@ -404,13 +406,11 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
           uint32_t wd[4];
           asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                        : "=r"(wd[0]), "=r"(wd[1]), "=r"(wd[2]), "=r"(wd[3]) : "r"(csrc + code_off));
-          const BlockLut lut = make_lut(valid ? absmax_deq(dqc0, dqs0) : 0.0f);
-          dqc0 = dqc1;
-          dqs0 = dqs1;
+          const BlockLut lut = make_lut(valid ? absmax_deq(dqc, dqs) : 0.0f);
           if (valid && kb + 2 < nkb_w) {
             const int64_t nb = blk + (kb + 2) * blk_step;
-            dqc1 = __ldg(p.dq_codes + nb);
-            dqs1 = __ldg(p.dq_scales + nb / kGroup);
+            dqc = __ldg(p.dq_codes + nb);
+            dqs = __ldg(p.dq_scales + nb / kGroup);
           }
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -423,6 +423,13 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
         }
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(ready_lead + 8 * s);
+        return true;
+      };
+      for (int kb = w.kb0; kb < w.kb1; kb += 2) {
+        if (!step(kb, dqcA, dqsA) || (kb + 1 < w.kb1 && !step(kb + 1, dqcB, dqsB))) {
+          alive = false;
+          break;
+        }
       }
       if (!alive) break;
 
