@@ -198,11 +198,12 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
   const int64_t sk_units = static_cast<int64_t>(p.sk_tiles) * S;
 
   if (threadIdx.x == 0) {
-    // `ready` and `tmem_empty` are used in the even CTA: the 8 dequant warps
-    // of each CTA arrive on them
+    // `ready` and `tmem_empty` are used in the even CTA: a stage's `ready`
+    // counts the 4 dequant warps of each CTA that took it, `tmem_empty` all 8
+    // epilogue warps of each CTA
     for (int s = 0; s < kStages; ++s) {
       mbar_init(loaded0 + 8 * s, 1);
-      mbar_init(ready0 + 8 * s, 2 * kDeqWarps);
+      mbar_init(ready0 + 8 * s, kDeqWarps);          // 4 warps of each CTA per stage
       mbar_init(free0 + 8 * s, 1);
     }
     mbar_init(tmem_full, 1);
@@ -323,30 +324,33 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
     __syncwarp();
   } else {
     // ------------------------------------------------------------ dequant producers + epilogue
-    const int t = threadIdx.x - 64;                 // 0..255: 32 weights each per K-step
+    // The 8 warps form two groups of 4 that take alternate K-steps (group 0 the
+    // even stage counts, group 1 the odd ones), so each group has two pipeline
+    // periods per stage; within a group each thread dequantises one whole
+    // 64-weight block of the CTA's half tile (one table per block).
+    const int group = (warp - 2) >> 2;
+    const int t = threadIdx.x - 64 - 128 * group;   // 0..127
     const int64_t blocks_per_row = p.w_out / kBlock;
-    // Fixed per thread: which 32 weights of this CTA's half tile it dequantises
-    // (half `hh` of a 64-weight block) and where they go in the weight tile.
-    int kr = 0, j = 0, hh = 0, nr = 0;
-    uint32_t row_off, code_off;
+    int kr = 0, j = 0, nr = 0;
+    uint32_t row_off, code_off0, code_off1;
     int swz;
     if (!kDX) {
-      // Quarter-warps (8 lanes) take 8 consecutive k rows of one 32-wide n
-      // chunk, so their 16-byte stores fall in 8 distinct bank groups.
+      // Quarter-warps (8 lanes) take 8 consecutive k rows of one 64-wide n
+      // block, so their 16-byte stores fall in 8 distinct bank groups.
       kr = (t & 7) + (((t >> 3) & 7) << 3);        // 0..63
-      j = t >> 7;                                   // which 64-wide n block of the half
-      hh = (t >> 6) & 1;                            // which 32 columns of that block
+      j = t >> 6;                                   // which 64-wide n block of the half
       row_off = j * 8192 + (kr >> 3) * 1024 + (kr & 7) * 128;
       swz = kr & 7;
       // codes tile: 64 rows of 64 bytes, 64-byte swizzle (16-byte chunk ^ (row >> 1) & 3)
-      code_off = kr * 64 + (((2 * j + hh) ^ ((kr >> 1) & 3)) << 4);
+      code_off0 = kr * 64 + (((2 * j) ^ ((kr >> 1) & 3)) << 4);
+      code_off1 = kr * 64 + (((2 * j + 1) ^ ((kr >> 1) & 3)) << 4);
     } else {
-      nr = t >> 1;                                  // n row of the half tile, 0..127
-      hh = t & 1;                                   // which 32 k values of the row
+      nr = t;                                       // n row of the half tile, 0..127
       row_off = nr * 128;
       swz = nr & 7;
       // codes tile: 128 rows of 32 bytes, 32-byte swizzle (16-byte chunk ^ (row >> 2) & 1)
-      code_off = nr * 32 + ((hh ^ ((nr >> 2) & 1)) << 4);
+      code_off0 = nr * 32 + ((0 ^ ((nr >> 2) & 1)) << 4);
+      code_off1 = nr * 32 + ((1 ^ ((nr >> 2) & 1)) << 4);
     }
     // K-step kb moves the block index by 64 rows (forward) or 1 block (dX).
     const int64_t blk_step = kDX ? 1 : 64 * blocks_per_row;
@@ -375,27 +379,31 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
         valid = (nh + nr) < p.N;
         blk = (nh + nr) * blocks_per_row;
       }
-      // Absmax code and scale of a K-step, loaded two K-steps ahead into one of
-      // two register slots; the loop is unrolled by two so that a slot is
-      // consumed and refilled in place (moving a pending load's register to
-      // another would wait for the load one step early).
+      // This group's K-steps of the item: those whose stage count has its parity.
+      const int g0 = g;
+      const int kb_first = w.kb0 + ((group - g0) & 1);
+      g += w.kb1 - w.kb0;
+      // Absmax code and scale of the group's next K-steps, loaded two of its
+      // steps ahead into one of two register slots; the loop is unrolled by two
+      // so that a slot is consumed and refilled in place (moving a pending
+      // load's register to another would wait for the load one step early).
       uint8_t dqcA = 0, dqcB = 0;
       float dqsA = 0.0f, dqsB = 0.0f;
-      if (valid && w.kb0 < nkb_w) {
-        const int64_t b0 = blk + w.kb0 * blk_step;
+      if (valid && kb_first < nkb_w) {
+        const int64_t b0 = blk + kb_first * blk_step;
         dqcA = __ldg(p.dq_codes + b0);
         dqsA = __ldg(p.dq_scales + b0 / kGroup);
       }
-      if (valid && w.kb0 + 1 < nkb_w) {
-        const int64_t b1 = blk + (w.kb0 + 1) * blk_step;
+      if (valid && kb_first + 2 < nkb_w) {
+        const int64_t b1 = blk + (kb_first + 2) * blk_step;
         dqcB = __ldg(p.dq_codes + b1);
         dqsB = __ldg(p.dq_scales + b1 / kGroup);
       }
-      // one K-step with the absmax in (dqc, dqs); refills them for kb + 2
+      // one K-step with the absmax in (dqc, dqs); refills them for kb + 4
       auto step = [&](int kb, uint8_t& dqc, float& dqs) -> bool {
-        const int s = g % kStages;
-        const uint32_t ph = (g / kStages) & 1;
-        ++g;
+        const int gg = g0 + (kb - w.kb0);
+        const int s = gg % kStages;
+        const uint32_t ph = (gg / kStages) & 1;
         // every lane waits; the warp leaves the loop together if the wait gave up
         const bool got = mbar_wait(loaded0 + 8 * s, ph, p.status, kFlagTimeoutProducer);
         if (!__all_sync(0xffffffffu, got)) return false;
@@ -403,21 +411,23 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
           const uint32_t stage = smem_addr(smem + s * kStageBytes);
           const uint32_t dst = stage + kABytes + row_off;
           const uint32_t csrc = stage + kABytes + kBBytes;
-          uint32_t wd[4];
+          uint32_t wd[8];
           asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(wd[0]), "=r"(wd[1]), "=r"(wd[2]), "=r"(wd[3]) : "r"(csrc + code_off));
+                       : "=r"(wd[0]), "=r"(wd[1]), "=r"(wd[2]), "=r"(wd[3]) : "r"(csrc + code_off0));
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(wd[4]), "=r"(wd[5]), "=r"(wd[6]), "=r"(wd[7]) : "r"(csrc + code_off1));
           const BlockLut lut = make_lut(valid ? absmax_deq(dqc, dqs) : 0.0f);
-          if (valid && kb + 2 < nkb_w) {
-            const int64_t nb = blk + (kb + 2) * blk_step;
+          if (valid && kb + 4 < nkb_w) {
+            const int64_t nb = blk + (kb + 4) * blk_step;
             dqc = __ldg(p.dq_codes + nb);
             dqs = __ldg(p.dq_scales + nb / kGroup);
           }
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
+          for (int c = 0; c < 8; ++c) {
             uint32_t o0, o1, o2, o3;
             lut4(lut, wd[c] & 0xFFFFu, o0, o1);
             lut4(lut, wd[c] >> 16, o2, o3);
-            st_shared_v4(dst + (((hh * 4 + c) ^ swz) << 4), o0, o1, o2, o3);
+            st_shared_v4(dst + ((c ^ swz) << 4), o0, o1, o2, o3);
           }
           fence_proxy_async_smem();
         }
@@ -425,8 +435,8 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
         if (lane == 0) mbar_arrive_cluster(ready_lead + 8 * s);
         return true;
       };
-      for (int kb = w.kb0; kb < w.kb1; kb += 2) {
-        if (!step(kb, dqcA, dqsA) || (kb + 1 < w.kb1 && !step(kb + 1, dqcB, dqsB))) {
+      for (int kb = kb_first; kb < w.kb1; kb += 4) {
+        if (!step(kb, dqcA, dqsA) || (kb + 2 < w.kb1 && !step(kb + 2, dqcB, dqsB))) {
           alive = false;
           break;
         }
