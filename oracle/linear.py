@@ -17,6 +17,12 @@ tokens X (M x in) maps to X @ W.
   dX = dY Wq^T + U A^T, is what "Forward and backward as usual" (step 3) implies
   for a layer inside a network; Wq receives no update ("What QLoRA adds over
   LoRA", last paragraph).
+* Dropout on the low-rank intermediate ("LoRA & QLoRA", "Dropout": dropout is
+  applied to A x during training).  Reading: inverted dropout with a given keep
+  mask (1 = keep) and drop probability p, V = s (X A) * keep / (1 - p), so that
+  E[V] = s X A; the same mask enters the backward, U = (s keep / (1 - p)) *
+  (dY B^T), and dB = V^T dY uses the dropped V.  The mask is an input: both the
+  oracle and the CUDA path receive the same bytes.
 * Merge: W = Wq + A B as a dense float matrix ("How it works", step 5).
 * Adapter size r (in + out) per layer ("How it works", paragraph after step 5).
 
@@ -35,12 +41,23 @@ def _f64(a) -> np.ndarray:
     return np.asarray(a, dtype=np.float64)
 
 
-def forward(X, A, B, Wq, scale: float = 1.0):
+def _factor(scale: float, keep, p: float):
+    """The factor each element of X A (and of dY B^T) is multiplied by: the
+    adapter scale s, times keep / (1 - p) under dropout."""
+    if keep is None:
+        return scale
+    if not 0.0 <= p < 1.0:
+        raise ValueError("the drop probability must lie in [0, 1)")
+    return scale * _f64(keep) / (1.0 - p)
+
+
+def forward(X, A, B, Wq, scale: float = 1.0, keep=None, p: float = 0.0):
     """Returns (Y, V) with V = s X A and Y = X Wq + V B (float64); s is the
     adapter scale alpha / r of "LoRA & QLoRA", "Scaling Factor alpha"
-    (h = W0 x + (alpha / r) B (A x)); 1 is the plain layer."""
+    (h = W0 x + (alpha / r) B (A x)); 1 is the plain layer.  With a keep mask
+    (M x r, 1 = keep) V is dropped out: V = s (X A) * keep / (1 - p)."""
     X, A, B, Wq = _f64(X), _f64(A), _f64(B), _f64(Wq)
-    V = scale * (X @ A)
+    V = _factor(scale, keep, p) * (X @ A)
     Y = X @ Wq + V @ B
     return Y, V
 
@@ -51,15 +68,18 @@ def forward_rows(X, A, B, Wq, rows):
     return forward(X, A, B, Wq)
 
 
-def backward(X, A, B, Wq, dY, scale: float = 1.0):
+def backward(X, A, B, Wq, dY, scale: float = 1.0, keep=None, p: float = 0.0):
     """Returns dict(dX, dA, dB, U) for L with dL/dY = dY (float64), for the layer
     with adapter scale s: U = s dY B^T, dX = dY Wq^T + U A^T, dA = X^T U,
-    dB = s (X A)^T dY."""
+    dB = s (X A)^T dY.  Under dropout with keep mask `keep` the factor
+    f = s keep / (1 - p) replaces s elementwise: U = f * (dY B^T), dB = V^T dY
+    with V = f * (X A)."""
     X, A, B, Wq, dY = _f64(X), _f64(A), _f64(B), _f64(Wq), _f64(dY)
-    U = scale * (dY @ B.T)
+    f = _factor(scale, keep, p)
+    U = f * (dY @ B.T)
     dX = dY @ Wq.T + U @ A.T
     dA = X.T @ U
-    dB = scale * ((X @ A).T @ dY)
+    dB = (f * (X @ A)).T @ dY
     return {"dX": dX, "dA": dA, "dB": dB, "U": U}
 
 

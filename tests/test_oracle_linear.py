@@ -65,11 +65,12 @@ def test_backward_factored_equals_dense_form():
     assert np.array_equal(a["dA"], g["dA"]) and np.array_equal(a["dB"], g["dB"])
 
 
-@pytest.mark.parametrize("scale", [1.0, 2.5])
-def test_backward_finite_differences(scale):
-    """Central differences of L = <dY, Y>: L is linear in each of X, A, B alone,
-    so the differences are exact up to rounding (catches a dropped term, a
-    transposed operand, a sign, or the adapter scale missing from one side)."""
+@pytest.mark.parametrize("scale,p", [(1.0, None), (2.5, None), (2.0, 0.3)])
+def test_backward_finite_differences(scale, p):
+    """Central differences of L = <dY, Y>: L is linear in each of X, A, B alone
+    (for a fixed dropout mask too), so the differences are exact up to rounding
+    (catches a dropped term, a transposed operand, a sign, the adapter scale or
+    the dropout mask missing from one side)."""
     rng = np.random.default_rng(8)
     n_in, n_out, M, r = 64, 64, 16, 8
     X = rng.standard_normal((M, n_in))
@@ -77,10 +78,12 @@ def test_backward_finite_differences(scale):
     B = rng.standard_normal((r, n_out)) * 0.1
     Wq = rng.standard_normal((n_in, n_out)) * 0.02
     dY = rng.standard_normal((M, n_out))
-    g = linear.backward(X, A, B, Wq, dY, scale)
+    keep = None if p is None else (rng.random((M, r)) >= p).astype(np.uint8)
+    pp = 0.0 if p is None else p
+    g = linear.backward(X, A, B, Wq, dY, scale, keep, pp)
 
     def L(X_, A_, B_):
-        return linear.loss_inner(linear.forward(X_, A_, B_, Wq, scale)[0], dY)
+        return linear.loss_inner(linear.forward(X_, A_, B_, Wq, scale, keep, pp)[0], dY)
 
     h = 0.5
     for name, P in (("dX", X), ("dA", A), ("dB", B)):
@@ -155,3 +158,50 @@ def test_synth_inputs_are_seeded_and_distributed():
     assert abs(a["W0"].std().item() - 0.02) < 1e-3
     assert abs(a["A"].float().std().item() - 1 / 16) < 5e-3
     assert abs(a["B"].float().std().item() - 0.01) < 1e-3
+
+
+def test_dropout_keep_all_and_drop_all():
+    """A mask that keeps everything at p = 0 is the plain layer; a mask that drops
+    everything leaves the frozen base alone: Y = X Wq, dA = dB = 0 exactly, dX =
+    dY Wq^T."""
+    t, Wq = _layer()
+    M, r = t["X"].shape[0], t["A"].shape[1]
+    Y0, V0 = linear.forward(t["X"], t["A"], t["B"], Wq)
+    Y1, V1 = linear.forward(t["X"], t["A"], t["B"], Wq, 1.0, np.ones((M, r), np.uint8), 0.0)
+    assert np.array_equal(Y0, Y1) and np.array_equal(V0, V1)
+    zero = np.zeros((M, r), np.uint8)
+    Yd, Vd = linear.forward(t["X"], t["A"], t["B"], Wq, 1.0, zero, 0.5)
+    X, W = t["X"].double().numpy(), np.asarray(Wq, np.float64)
+    assert np.array_equal(Yd, X @ W) and not np.any(Vd)
+    g = linear.backward(t["X"], t["A"], t["B"], Wq, t["dY"], 1.0, zero, 0.5)
+    assert not np.any(g["dA"]) and not np.any(g["dB"])
+    assert np.array_equal(g["dX"], t["dY"].double().numpy() @ W.T)
+
+
+def test_dropout_preserves_the_mean():
+    """Inverted dropout: averaged over masks drawn with keep probability 1 - p,
+    the dropped V and the layer output match the undropped ones (the 1 / (1 - p)
+    rescale; a missing or inverted rescale is off by a factor of 2 here)."""
+    rng = np.random.default_rng(3)
+    n_in, n_out, M, r, p = 32, 24, 6, 4, 0.5
+    X = rng.standard_normal((M, n_in))
+    A = rng.standard_normal((n_in, r))
+    B = rng.standard_normal((r, n_out))
+    Wq = rng.standard_normal((n_in, n_out)) * 0.02
+    Y_ref, V_ref = linear.forward(X, A, B, Wq)
+    n = 4000
+    V_sum = np.zeros_like(V_ref)
+    for _ in range(n):
+        keep = (rng.random((M, r)) >= p).astype(np.uint8)
+        V_sum += linear.forward(X, A, B, Wq, 1.0, keep, p)[1]
+    V_mean = V_sum / n
+    # per element the sample mean has standard deviation |V| sqrt(p / ((1 - p) n))
+    tol = 5 * np.abs(V_ref) * np.sqrt(p / ((1 - p) * n)) + 1e-12
+    assert np.all(np.abs(V_mean - V_ref) <= tol)
+
+
+def test_dropout_probability_out_of_range():
+    t, Wq = _layer()
+    keep = np.ones((t["X"].shape[0], t["A"].shape[1]), np.uint8)
+    with pytest.raises(ValueError):
+        linear.forward(t["X"], t["A"], t["B"], Wq, 1.0, keep, 1.0)
