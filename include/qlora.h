@@ -195,12 +195,23 @@ QLORA_API qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16_
  *   flags          QLORA_ACCUMULATE_GRADS: the backward adds into dA and dB
  *                  instead of overwriting them (gradient accumulation over
  *                  micro-batches); not allowed for the forward or with Adam.
- * A NULL options pointer means adapter_scale = 1 and no flags.
+ *   dropout_keep   [device] uint8 (M, r), row-major, 1 = keep, 0 = drop, or NULL
+ *                  for no dropout.  Dropout on the low-rank intermediate
+ *                  ("LoRA & QLoRA", "Dropout": applied to A x during training),
+ *                  inverted: V = s (X A) keep / (1 - p), and the backward uses
+ *                  U = s keep / (1 - p) (dY B^T), so the forward and the backward
+ *                  of one micro-batch must get the same mask (the caller draws
+ *                  it, e.g. Bernoulli(1 - p), and keeps it).  Read only.
+ *   dropout_p      the drop probability p in [0, 1) the kept values are rescaled
+ *                  by; checked only with a mask, else QLORA_ERR_INVALID_ARG.
+ * A NULL options pointer means adapter_scale = 1, no flags and no dropout.
  */
 #define QLORA_ACCUMULATE_GRADS 1u
 typedef struct {
   float adapter_scale;
   uint32_t flags;
+  const uint8_t* dropout_keep;
+  float dropout_p;
 } qlora_linear_opts;
 
 /* qlora_linear_fwd with options (arguments otherwise as there). */

@@ -64,7 +64,8 @@ class _AdamHparams(ctypes.Structure):
 
 
 class _LinearOpts(ctypes.Structure):
-    _fields_ = [("adapter_scale", ctypes.c_float), ("flags", ctypes.c_uint32)]
+    _fields_ = [("adapter_scale", ctypes.c_float), ("flags", ctypes.c_uint32),
+                ("dropout_keep", ctypes.c_void_p), ("dropout_p", ctypes.c_float)]
 
 
 class _AdamState(ctypes.Structure):
@@ -252,14 +253,27 @@ def qlora_merge(w: NF4Weight, A: torch.Tensor, B: torch.Tensor, dtype=torch.floa
     return out
 
 
-def _opts(adapter_scale: float, accumulate: bool = False):
-    return _LinearOpts(adapter_scale, QLORA_ACCUMULATE_GRADS if accumulate else 0)
+def _opts(adapter_scale: float, accumulate: bool = False, dropout_keep=None, dropout_p: float = 0.0):
+    return _LinearOpts(adapter_scale, QLORA_ACCUMULATE_GRADS if accumulate else 0,
+                       _ptr(dropout_keep) if dropout_keep is not None else None, dropout_p)
+
+
+def dropout_mask(M: int, r: int, p: float, generator=None, device="cuda") -> torch.Tensor:
+    """A dropout keep mask for the low-rank intermediate: uint8 (M, r), 1 with
+    probability 1 - p.  Pass the same mask to the forward and the backward of one
+    micro-batch."""
+    if not 0.0 <= p < 1.0:
+        raise ValueError("p must lie in [0, 1)")
+    u = torch.rand((M, r), generator=generator, device=device)
+    return (u >= p).to(torch.uint8)
 
 
 def qlora_linear_fwd(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, workspace: Workspace,
-                     save_V: bool = True, stream=None, Y=None, V=None, adapter_scale: float = 1.0):
+                     save_V: bool = True, stream=None, Y=None, V=None, adapter_scale: float = 1.0,
+                     dropout_keep=None, dropout_p: float = 0.0):
     """Returns (Y, V) with V = s X A (None when save_V is False); s =
-    adapter_scale (alpha / r), 1 for the plain layer."""
+    adapter_scale (alpha / r), 1 for the plain layer.  With dropout_keep (uint8
+    (M, r) on the device, 1 = keep) V is dropped out: s (X A) keep / (1 - p)."""
     M, r = X.shape[0], A.shape[1]
     if Y is None:
         Y = torch.empty((M, w.n_out), dtype=torch.bfloat16, device=X.device)
@@ -268,12 +282,12 @@ def qlora_linear_fwd(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Te
     nb = qlora_workspace_bytes(QLORA_OP_FWD, M, w.n_in, w.n_out, r)
     buf = workspace.get(nb, stream)
     ws = w.c_struct()
-    if adapter_scale == 1.0:
+    if adapter_scale == 1.0 and dropout_keep is None:
         _check(lib().qlora_linear_fwd(ctypes.byref(ws), _ptr(X), M, _ptr(A), _ptr(B), r, _ptr(Y),
                                       _ptr(V) if save_V else None, _ptr(buf), buf.numel(), _stream(stream)),
                "qlora_linear_fwd")
     else:
-        o = _opts(adapter_scale)
+        o = _opts(adapter_scale, False, dropout_keep, dropout_p)
         _check(lib().qlora_linear_fwd_ex(ctypes.byref(ws), _ptr(X), M, _ptr(A), _ptr(B), r, _ptr(Y),
                                          _ptr(V) if save_V else None, ctypes.byref(o), _ptr(buf), buf.numel(),
                                          _stream(stream)), "qlora_linear_fwd_ex")
@@ -282,9 +296,11 @@ def qlora_linear_fwd(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Te
 
 def qlora_linear_bwd(w: NF4Weight, X: torch.Tensor, V, dY: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
                      workspace: Workspace, need_dX: bool = True, stream=None, dX=None, dA=None, dB=None,
-                     adapter_scale: float = 1.0, accumulate: bool = False):
+                     adapter_scale: float = 1.0, accumulate: bool = False, dropout_keep=None,
+                     dropout_p: float = 0.0):
     """Returns (dX or None, dA fp32 (in, r), dB fp32 (r, out)).  With accumulate,
-    dA and dB (given) receive the sums instead of being overwritten."""
+    dA and dB (given) receive the sums instead of being overwritten.  Under
+    dropout pass the forward's mask and p."""
     if accumulate and (dA is None or dB is None):
         raise ValueError("accumulate needs the dA and dB to add into")
     M, r = X.shape[0], A.shape[1]
@@ -298,12 +314,12 @@ def qlora_linear_bwd(w: NF4Weight, X: torch.Tensor, V, dY: torch.Tensor, A: torc
     nb = qlora_workspace_bytes(QLORA_OP_BWD, M, w.n_in, w.n_out, r)
     buf = workspace.get(nb, stream)
     ws = w.c_struct()
-    if adapter_scale == 1.0 and not accumulate:
+    if adapter_scale == 1.0 and not accumulate and dropout_keep is None:
         _check(lib().qlora_linear_bwd(ctypes.byref(ws), _ptr(X), _ptr(V), _ptr(dY), M, _ptr(A), _ptr(B), r,
                                       _ptr(dX) if need_dX else None, _ptr(dA), _ptr(dB), _ptr(buf), buf.numel(),
                                       _stream(stream)), "qlora_linear_bwd")
     else:
-        o = _opts(adapter_scale, accumulate)
+        o = _opts(adapter_scale, accumulate, dropout_keep, dropout_p)
         _check(lib().qlora_linear_bwd_ex(ctypes.byref(ws), _ptr(X), _ptr(V), _ptr(dY), M, _ptr(A), _ptr(B), r,
                                          _ptr(dX) if need_dX else None, _ptr(dA), _ptr(dB), ctypes.byref(o),
                                          _ptr(buf), buf.numel(), _stream(stream)), "qlora_linear_bwd_ex")
@@ -323,7 +339,8 @@ def adam_state(A: torch.Tensor, B: torch.Tensor) -> dict:
 def qlora_linear_bwd_adam(w: NF4Weight, X: torch.Tensor, V, dY: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
                           state: dict, step: int, workspace: Workspace, lr: float = 1e-3, beta1: float = 0.9,
                           beta2: float = 0.999, eps: float = 1e-8, weight_decay: float = 0.0,
-                          need_dX: bool = True, stream=None, dX=None, adapter_scale: float = 1.0):
+                          need_dX: bool = True, stream=None, dX=None, adapter_scale: float = 1.0,
+                          dropout_keep=None, dropout_p: float = 0.0):
     """Backward with one fused Adam/AdamW step on the adapters: updates `state`
     (fp32 A32, B32, mA, vA, mB, vB) and the bf16 A and B in place; returns dX or None."""
     M, r = X.shape[0], A.shape[1]
@@ -334,7 +351,7 @@ def qlora_linear_bwd_adam(w: NF4Weight, X: torch.Tensor, V, dY: torch.Tensor, A:
     ws = w.c_struct()
     st = _AdamState(*[_ptr(state[k]) for k in ("A32", "B32", "mA", "vA", "mB", "vB")])
     hp = _AdamHparams(lr, beta1, beta2, eps, weight_decay, step)
-    o = _opts(adapter_scale)
+    o = _opts(adapter_scale, False, dropout_keep, dropout_p)
     _check(lib().qlora_linear_bwd_adam(ctypes.byref(ws), _ptr(X), _ptr(V), _ptr(dY), M, _ptr(A), _ptr(B), r,
                                        _ptr(dX) if need_dX else None, ctypes.byref(st), ctypes.byref(hp),
                                        ctypes.byref(o), _ptr(buf), buf.numel(), _stream(stream)),

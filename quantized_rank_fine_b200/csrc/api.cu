@@ -282,9 +282,32 @@ qlora_status qlora_merge(const qlora_nf4_weight* w, const uint16_t* A, const uin
   return QLORA_OK;
 }
 
+// Options of the _ex calls (adapter scale, flags, dropout), checked on the host.
+struct LinearOpts {
+  float scale = 1.0f;
+  bool accumulate = false;
+  qlora::Dropout drop;
+};
+
+static qlora_status read_opts(const qlora_linear_opts* o, LinearOpts& lo) {
+  lo = LinearOpts{};
+  if (!o) return QLORA_OK;
+  if (!std::isfinite(o->adapter_scale) || (o->flags & ~static_cast<uint32_t>(QLORA_ACCUMULATE_GRADS)) != 0u)
+    return QLORA_ERR_INVALID_ARG;
+  lo.scale = o->adapter_scale;
+  lo.accumulate = (o->flags & QLORA_ACCUMULATE_GRADS) != 0u;
+  if (o->dropout_keep) {
+    if (!(o->dropout_p >= 0.0f && o->dropout_p < 1.0f)) return QLORA_ERR_INVALID_ARG;
+    QLORA_TRY(check_ptr(o->dropout_keep));
+    lo.drop.keep = o->dropout_keep;
+    lo.drop.keep_scale = static_cast<float>(1.0 / (1.0 - static_cast<double>(o->dropout_p)));
+  }
+  return QLORA_OK;
+}
+
 static qlora_status fwd_impl(const qlora_nf4_weight* w, const uint16_t* X, int64_t M, const uint16_t* A,
                              const uint16_t* B, int r, uint16_t* Y, uint16_t* V_save, void* ws, size_t ws_bytes,
-                             void* stream, float scale) {
+                             void* stream, const LinearOpts& lo) {
   if (!X || !A || !B || !Y) return QLORA_ERR_INVALID_ARG;
   QLORA_TRY(check_weight_shape(w));
   if (!linear_shape_ok(M, w->in, w->out, r)) return QLORA_ERR_SHAPE;
@@ -305,47 +328,34 @@ static qlora_status fwd_impl(const qlora_nf4_weight* w, const uint16_t* X, int64
   uint16_t* V = V_save ? V_save : reinterpret_cast<uint16_t*>(base + L.v_off);
   const WeightView wv = view(w);
   if (qlora::gemv_supported(M, w->in, w->out)) {
-    QLORA_CUDA(qlora::launch_xa_small(X, A, M, w->in, r, V, s, scale));
+    QLORA_CUDA(qlora::launch_xa_small(X, A, M, w->in, r, V, s, lo.scale, lo.drop));
     QLORA_CUDA(qlora::launch_gemv(wv, X, V, B, M, r, Y, status, s));
   } else {
-    QLORA_CUDA(qlora::launch_xa(X, A, M, w->in, r, V, status, s, scale));
+    QLORA_CUDA(qlora::launch_xa(X, A, M, w->in, r, V, status, s, lo.scale, lo.drop));
     const SplitRegion sr = split_region(ws, ws_bytes, L);
     QLORA_CUDA(qlora::launch_fwd_gemm(wv, X, V, B, M, r, Y, status, sr.counters, sr.partials, sr.partial_bytes, s));
   }
   return QLORA_OK;
 }
 
-// Options of the _ex calls: adapter scale and flags, checked on the host.
-static qlora_status read_opts(const qlora_linear_opts* o, float& scale, bool& accumulate) {
-  scale = 1.0f;
-  accumulate = false;
-  if (!o) return QLORA_OK;
-  if (!std::isfinite(o->adapter_scale) || (o->flags & ~static_cast<uint32_t>(QLORA_ACCUMULATE_GRADS)) != 0u)
-    return QLORA_ERR_INVALID_ARG;
-  scale = o->adapter_scale;
-  accumulate = (o->flags & QLORA_ACCUMULATE_GRADS) != 0u;
-  return QLORA_OK;
-}
-
 qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16_t* X, int64_t M, const uint16_t* A,
                               const uint16_t* B, int r, uint16_t* Y, uint16_t* V_save, void* ws, size_t ws_bytes,
                               void* stream) {
-  return fwd_impl(w, X, M, A, B, r, Y, V_save, ws, ws_bytes, stream, 1.0f);
+  return fwd_impl(w, X, M, A, B, r, Y, V_save, ws, ws_bytes, stream, LinearOpts{});
 }
 
 qlora_status qlora_linear_fwd_ex(const qlora_nf4_weight* w, const uint16_t* X, int64_t M, const uint16_t* A,
                                  const uint16_t* B, int r, uint16_t* Y, uint16_t* V_save,
                                  const qlora_linear_opts* opts, void* ws, size_t ws_bytes, void* stream) {
-  float scale;
-  bool accumulate;
-  QLORA_TRY(read_opts(opts, scale, accumulate));
-  if (accumulate) return QLORA_ERR_INVALID_ARG;   // the forward has no gradients
-  return fwd_impl(w, X, M, A, B, r, Y, V_save, ws, ws_bytes, stream, scale);
+  LinearOpts lo;
+  QLORA_TRY(read_opts(opts, lo));
+  if (lo.accumulate) return QLORA_ERR_INVALID_ARG;   // the forward has no gradients
+  return fwd_impl(w, X, M, A, B, r, Y, V_save, ws, ws_bytes, stream, lo);
 }
 
 static qlora_status bwd_impl(const qlora_nf4_weight* w, const uint16_t* X, const uint16_t* V, const uint16_t* dY,
                              int64_t M, const uint16_t* A, const uint16_t* B, int r, uint16_t* dX, float* dA,
-                             float* dB, void* ws, size_t ws_bytes, void* stream, float scale, bool accumulate) {
+                             float* dB, void* ws, size_t ws_bytes, void* stream, const LinearOpts& lo) {
   if (!X || !dY || !A || !B || !dA || !dB) return QLORA_ERR_INVALID_ARG;
   QLORA_TRY(check_weight_shape(w));
   if (!linear_shape_ok(M, w->in, w->out, r)) return QLORA_ERR_SHAPE;
@@ -370,12 +380,12 @@ static qlora_status bwd_impl(const qlora_nf4_weight* w, const uint16_t* X, const
   const WeightView wv = view(w);
   if (!V) {
     uint16_t* Vw = reinterpret_cast<uint16_t*>(base + L.v_off);
-    QLORA_CUDA(qlora::launch_xa(X, A, M, w->in, r, Vw, status, s, scale));
+    QLORA_CUDA(qlora::launch_xa(X, A, M, w->in, r, Vw, status, s, lo.scale, lo.drop));
     V = Vw;
   }
-  QLORA_CUDA(qlora::launch_dybt(dY, B, M, w->out, r, U, status, s, scale));
-  QLORA_CUDA(qlora::launch_vtdy(V, dY, M, w->out, r, dB, status, s, nullptr, accumulate));
-  QLORA_CUDA(qlora::launch_xtu(X, U, M, w->in, r, dA, status, s, nullptr, accumulate));
+  QLORA_CUDA(qlora::launch_dybt(dY, B, M, w->out, r, U, status, s, lo.scale, lo.drop));
+  QLORA_CUDA(qlora::launch_vtdy(V, dY, M, w->out, r, dB, status, s, nullptr, lo.accumulate));
+  QLORA_CUDA(qlora::launch_xtu(X, U, M, w->in, r, dA, status, s, nullptr, lo.accumulate));
   if (dX) {
     const SplitRegion sr = split_region(ws, ws_bytes, L);
     QLORA_CUDA(qlora::launch_dx_gemm(wv, dY, U, A, M, r, dX, status, sr.counters, sr.partials, sr.partial_bytes, s));
@@ -386,16 +396,15 @@ static qlora_status bwd_impl(const qlora_nf4_weight* w, const uint16_t* X, const
 qlora_status qlora_linear_bwd(const qlora_nf4_weight* w, const uint16_t* X, const uint16_t* V, const uint16_t* dY,
                               int64_t M, const uint16_t* A, const uint16_t* B, int r, uint16_t* dX, float* dA,
                               float* dB, void* ws, size_t ws_bytes, void* stream) {
-  return bwd_impl(w, X, V, dY, M, A, B, r, dX, dA, dB, ws, ws_bytes, stream, 1.0f, false);
+  return bwd_impl(w, X, V, dY, M, A, B, r, dX, dA, dB, ws, ws_bytes, stream, LinearOpts{});
 }
 
 qlora_status qlora_linear_bwd_ex(const qlora_nf4_weight* w, const uint16_t* X, const uint16_t* V, const uint16_t* dY,
                                  int64_t M, const uint16_t* A, const uint16_t* B, int r, uint16_t* dX, float* dA,
                                  float* dB, const qlora_linear_opts* opts, void* ws, size_t ws_bytes, void* stream) {
-  float scale;
-  bool accumulate;
-  QLORA_TRY(read_opts(opts, scale, accumulate));
-  return bwd_impl(w, X, V, dY, M, A, B, r, dX, dA, dB, ws, ws_bytes, stream, scale, accumulate);
+  LinearOpts lo;
+  QLORA_TRY(read_opts(opts, lo));
+  return bwd_impl(w, X, V, dY, M, A, B, r, dX, dA, dB, ws, ws_bytes, stream, lo);
 }
 
 qlora_status qlora_linear_bwd_adam(const qlora_nf4_weight* w, const uint16_t* X, const uint16_t* V,
@@ -403,10 +412,9 @@ qlora_status qlora_linear_bwd_adam(const qlora_nf4_weight* w, const uint16_t* X,
                                    const qlora_adam_state* st, const qlora_adam_hparams* hp,
                                    const qlora_linear_opts* opts, void* ws, size_t ws_bytes, void* stream) {
   if (!X || !dY || !A || !B || !st || !hp) return QLORA_ERR_INVALID_ARG;
-  float scale;
-  bool accumulate;
-  QLORA_TRY(read_opts(opts, scale, accumulate));
-  if (accumulate) return QLORA_ERR_INVALID_ARG;   // the step consumes the gradients
+  LinearOpts lo;
+  QLORA_TRY(read_opts(opts, lo));
+  if (lo.accumulate) return QLORA_ERR_INVALID_ARG;   // the step consumes the gradients
   if (!st->A32 || !st->B32 || !st->mA || !st->vA || !st->mB || !st->vB) return QLORA_ERR_INVALID_ARG;
   if (!(hp->lr >= 0.0f) || !(hp->beta1 >= 0.0f && hp->beta1 < 1.0f) || !(hp->beta2 >= 0.0f && hp->beta2 < 1.0f) ||
       !(hp->eps > 0.0f) || !(hp->weight_decay >= 0.0f) || hp->step < 1 || !std::isfinite(hp->lr))
@@ -458,10 +466,10 @@ qlora_status qlora_linear_bwd_adam(const qlora_nf4_weight* w, const uint16_t* X,
   // B step follows U, dX reads A before the A step.
   if (!V) {
     uint16_t* Vw = reinterpret_cast<uint16_t*>(base + L.v_off);
-    QLORA_CUDA(qlora::launch_xa(X, A, M, w->in, r, Vw, status, s, scale));
+    QLORA_CUDA(qlora::launch_xa(X, A, M, w->in, r, Vw, status, s, lo.scale, lo.drop));
     V = Vw;
   }
-  QLORA_CUDA(qlora::launch_dybt(dY, B, M, w->out, r, U, status, s, scale));
+  QLORA_CUDA(qlora::launch_dybt(dY, B, M, w->out, r, U, status, s, lo.scale, lo.drop));
   QLORA_CUDA(qlora::launch_vtdy(V, dY, M, w->out, r, nullptr, status, s, &pB));
   if (dX) {
     const SplitRegion sr = split_region(ws, ws_bytes, L);

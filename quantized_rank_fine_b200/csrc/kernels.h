@@ -58,10 +58,19 @@ struct AdamParams {
 // adapter scale) as they are formed.  dA and dB take an optional Adam step
 // (adam != nullptr): the gradient then updates the optimizer state instead of
 // being stored; `accumulate` adds them to the stored values instead.
+//
+// Dropout on the low-rank intermediate: with keep != nullptr (device, M x r,
+// 1 = keep) every stored element of V and U is also multiplied by keep_scale
+// (1 / (1 - p)) where it is kept and by 0 where it is dropped.
+struct Dropout {
+  const uint8_t* keep = nullptr;
+  float keep_scale = 1.0f;
+};
 cudaError_t launch_xa(const uint16_t* X, const uint16_t* A, int64_t M, int64_t n_in, int r, uint16_t* V,
-                      uint32_t* status, cudaStream_t stream, float scale = 1.0f);
+                      uint32_t* status, cudaStream_t stream, float scale = 1.0f, Dropout drop = {});
 cudaError_t launch_dybt(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t n_out, int r,
-                        uint16_t* U, uint32_t* status, cudaStream_t stream, float scale = 1.0f);
+                        uint16_t* U, uint32_t* status, cudaStream_t stream, float scale = 1.0f,
+                        Dropout drop = {});
 cudaError_t launch_xtu(const uint16_t* X, const uint16_t* U, int64_t M, int64_t n_in, int r, float* dA,
                        uint32_t* status, cudaStream_t stream, const AdamParams* adam = nullptr,
                        bool accumulate = false);
@@ -77,7 +86,7 @@ bool gemv_supported(int64_t M, int64_t K, int64_t N);
 // V = X A for M <= kGemvMaxTokens on CUDA cores (K split over a cluster); lets
 // the small-M forward launched after it start early.
 cudaError_t launch_xa_small(const uint16_t* X, const uint16_t* A, int64_t M, int64_t K, int r, uint16_t* V,
-                            cudaStream_t stream, float scale = 1.0f);
+                            cudaStream_t stream, float scale = 1.0f, Dropout drop = {});
 cudaError_t launch_gemv(const WeightView& w, const uint16_t* X, const uint16_t* V, const uint16_t* B, int64_t M,
                         int r, uint16_t* Y, uint32_t* status, cudaStream_t stream);
 

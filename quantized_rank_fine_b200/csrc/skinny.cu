@@ -52,6 +52,8 @@ struct SkArgs {
   AdamParams ap;
   float scale;           // every value is multiplied by it before the store
   int accumulate;        // out_kind 1 or 2: add to the stored values instead of overwriting
+  const uint8_t* keep;   // out_kind 0: dropout keep mask [row][r] (1 = keep), or nullptr
+  float keep_scale;      // factor of the kept values (1 / (1 - p))
 };
 
 // One Adam / AdamW step of parameter element i with gradient g (fp32, IEEE
@@ -83,6 +85,11 @@ __device__ __forceinline__ void store_pair(const SkArgs& p, int64_t row, int col
     return;
   }
   if (p.out_kind == 0) {
+    if (p.keep) {
+      const uint8_t* k = p.keep + row * p.r + col;
+      v0 *= k[0] ? p.keep_scale : 0.0f;
+      v1 *= k[1] ? p.keep_scale : 0.0f;
+    }
     *reinterpret_cast<uint32_t*>(reinterpret_cast<uint16_t*>(p.out) + row * p.r + col) = pack_bf16x2(v0, v1);
   } else if (p.out_kind == 1) {
     float2* d = reinterpret_cast<float2*>(reinterpret_cast<float*>(p.out) + row * p.r + col);
@@ -328,7 +335,7 @@ Plan plan(int64_t rows, int r, int64_t k_total) {
 template <bool A_MN, bool B_MN>
 cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows, int r, int64_t k_total, void* out,
                 int out_kind, uint32_t* status, cudaStream_t stream, const AdamParams* adam = nullptr,
-                float scale = 1.0f, bool accumulate = false) {
+                float scale = 1.0f, bool accumulate = false, Dropout drop = {}) {
   static bool set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -342,7 +349,7 @@ cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows, int 
   }
   const Plan pl = plan(rows, r, k_total);
   SkArgs a{rows, r, k_total, pl.kps, out, out_kind, status, adam ? 1 : 0, adam ? *adam : AdamParams{}, scale,
-           accumulate ? 1 : 0};
+           accumulate ? 1 : 0, drop.keep, drop.keep_scale};
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = pl.grid;
   cfg.blockDim = dim3(kSkThreads);
@@ -368,18 +375,18 @@ cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows, int 
 
 // V = X A: Aop = X (M x in, k contiguous); Bop[j][k] = A[k][j] (j contiguous).
 cudaError_t launch_xa(const uint16_t* X, const uint16_t* A, int64_t M, int64_t n_in, int r, uint16_t* V,
-                      uint32_t* status, cudaStream_t stream, float scale) {
+                      uint32_t* status, cudaStream_t stream, float scale, Dropout drop) {
   CUtensorMap ta, tb;
   if (!bf16_map(&ta, X, M, n_in, 64, 128) || !bf16_map(&tb, A, n_in, r, 64, 64)) return cudaErrorInvalidValue;
-  return run<false, true>(ta, tb, M, r, n_in, V, 0, status, stream, nullptr, scale);
+  return run<false, true>(ta, tb, M, r, n_in, V, 0, status, stream, nullptr, scale, false, drop);
 }
 
 // U = dY B^T: Aop = dY (M x out, k contiguous); Bop = B (r x out, k contiguous).
 cudaError_t launch_dybt(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t n_out, int r, uint16_t* U,
-                        uint32_t* status, cudaStream_t stream, float scale) {
+                        uint32_t* status, cudaStream_t stream, float scale, Dropout drop) {
   CUtensorMap ta, tb;
   if (!bf16_map(&ta, dY, M, n_out, 64, 128) || !bf16_map(&tb, B, r, n_out, 64, 64)) return cudaErrorInvalidValue;
-  return run<false, false>(ta, tb, M, r, n_out, U, 0, status, stream, nullptr, scale);
+  return run<false, false>(ta, tb, M, r, n_out, U, 0, status, stream, nullptr, scale, false, drop);
 }
 
 // dA = X^T U: Aop[i][m] = X[m][i] (i contiguous); Bop[j][m] = U[m][j] (j contiguous).

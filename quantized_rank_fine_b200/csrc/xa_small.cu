@@ -44,6 +44,8 @@ struct XaArgs {
   int Kc;              // rows per split (multiple of 64)
   uint16_t* V;         // (M, r) bf16
   float scale;         // V = bf16(scale * X A)
+  const uint8_t* keep; // dropout keep mask (M, r), 1 = keep, or nullptr
+  float keep_scale;    // factor of the kept values (1 / (1 - p))
 };
 
 __global__ void __launch_bounds__(kXaThreads) xa_small_kernel(const XaArgs p) {
@@ -145,7 +147,10 @@ __global__ void __launch_bounds__(kXaThreads) xa_small_kernel(const XaArgs p) {
     float y = 0.0f;
     for (int sp = 0; sp < S; ++sp) y += recv[sp * cap + slot];
     const int mm = e / cols, jj = e % cols;
-    p.V[static_cast<int64_t>(mm) * p.r + c0 + jj] = static_cast<uint16_t>(pack_bf16x2(y * p.scale, 0.0f));
+    const int64_t at = static_cast<int64_t>(mm) * p.r + c0 + jj;
+    float v = y * p.scale;
+    if (p.keep) v *= p.keep[at] ? p.keep_scale : 0.0f;
+    p.V[at] = static_cast<uint16_t>(pack_bf16x2(v, 0.0f));
   }
 }
 
@@ -164,7 +169,7 @@ void xa_plan(int64_t K, int& S, int& Kc) {
 }  // namespace
 
 cudaError_t launch_xa_small(const uint16_t* X, const uint16_t* A, int64_t M, int64_t K, int r, uint16_t* V,
-                            cudaStream_t stream, float scale) {
+                            cudaStream_t stream, float scale, Dropout drop) {
   if (M < 1 || M > kGemvMaxTokens) return cudaErrorInvalidValue;
   static bool attr_set[64] = {};
   int dev = 0;
@@ -179,7 +184,7 @@ cudaError_t launch_xa_small(const uint16_t* X, const uint16_t* A, int64_t M, int
   }
   int S, Kc;
   xa_plan(K, S, Kc);
-  XaArgs a{X, A, static_cast<int>(M), K, r, Kc, V, scale};
+  XaArgs a{X, A, static_cast<int>(M), K, r, Kc, V, scale, drop.keep, drop.keep_scale};
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>((r + kXaCols - 1) / kXaCols), static_cast<unsigned>(S));
   cfg.blockDim = dim3(kXaThreads);

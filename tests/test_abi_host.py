@@ -129,6 +129,15 @@ def test_ex_options_rejected_before_launch(L):
                    None) == 1
     assert bwd(wp, FAKE, None, FAKE, 64, FAKE, FAKE, 12, None, FAKE, FAKE, ctypes.byref(acc), FAKE, 1 << 30,
                None) == 2                                                          # r % 8
+    # dropout: with a keep mask the drop probability must lie in [0, 1)
+    for p in (1.0, -0.25, float("nan")):
+        o = q._LinearOpts(1.0, 0, FAKE, p)
+        assert fwd(wp, FAKE, 64, FAKE, FAKE, 8, FAKE, None, ctypes.byref(o), FAKE, 1 << 30, None) == 1
+        assert bwd(wp, FAKE, None, FAKE, 64, FAKE, FAKE, 8, None, FAKE, FAKE, ctypes.byref(o), FAKE, 1 << 30,
+                   None) == 1
+    # without a mask p is not read: the call gets past the options (r % 8 fails next)
+    o = q._LinearOpts(1.0, 0, None, 7.0)
+    assert fwd(wp, FAKE, 64, FAKE, FAKE, 12, FAKE, None, ctypes.byref(o), FAKE, 1 << 30, None) == 2
 
 
 def test_dequant_merge_reject_before_launch(L):

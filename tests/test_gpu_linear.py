@@ -200,3 +200,55 @@ def test_accumulated_gradients():
     g2 = linear.backward(t2["X"], t["A"], t["B"], Wq, t2["dY"])
     assert_close(dA, dA0.double().cpu().numpy() + g1["dA"] + g2["dA"], "dA accumulated")
     assert_close(dB, dB0.double().cpu().numpy() + g1["dB"] + g2["dB"], "dB accumulated")
+
+
+@pytest.mark.parametrize("M,n_in,n_out,r,p", [
+    (300, 320, 192, 24, 0.05), (1000, 576, 704, 40, 0.5), (4, 512, 768, 16, 0.3), (16, 4096, 4096, 16, 0.05),
+])
+def test_dropout(M, n_in, n_out, r, p):
+    """Dropout on X A ("LoRA & QLoRA", "Dropout") with adapter scale 2: a keep mask
+    drawn with torch on the device, the same bytes to both sides; every output of
+    the forward and backward against the oracle (M <= 16 takes the small-M
+    forward), and the backward that recomputes V matches the one given V."""
+    t, w = layer_on_gpu(n_in, n_out, M, r, tag="drop")
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(5)
+    keep = q.dropout_mask(M, r, p, generator=gen)
+    s = 2.0
+    ws = q.Workspace()
+    Y, V = q.qlora_linear_fwd(w, t["X"], t["A"], t["B"], ws, adapter_scale=s, dropout_keep=keep, dropout_p=p)
+    dX, dA, dB = q.qlora_linear_bwd(w, t["X"], V, t["dY"], t["A"], t["B"], ws, adapter_scale=s,
+                                    dropout_keep=keep, dropout_p=p)
+    dX2, dA2, dB2 = q.qlora_linear_bwd(w, t["X"], None, t["dY"], t["A"], t["B"], ws, adapter_scale=s,
+                                       dropout_keep=keep, dropout_p=p)
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+    assert torch.equal(dX, dX2) and torch.equal(dA, dA2) and torch.equal(dB, dB2)
+    k = keep.cpu().numpy()
+    assert 0 < k.sum() < k.size or p < 0.1
+    Wq = oracle_weight(w)
+    Yr, Vr = linear.forward(t["X"], t["A"], t["B"], Wq, s, k, p)
+    g = linear.backward(t["X"], t["A"], t["B"], Wq, t["dY"], s, k, p)
+    assert_close(Y, Yr, "Y")
+    assert_close(V, Vr, "V")
+    assert_close(dX, g["dX"], "dX")
+    assert_close(dA, g["dA"], "dA")
+    assert_close(dB, g["dB"], "dB")
+    # dropped elements of V are exact zeros
+    assert torch.count_nonzero(V[keep == 0]).item() == 0
+
+
+@pytest.mark.parametrize("M", [8, 300])
+def test_dropout_drop_all(M):
+    """A mask that drops every element leaves the frozen base alone: Y is the
+    forward with B = 0, bit for bit, and dA = dB = 0 exactly."""
+    n_in, n_out, r = 512, 320, 16
+    t, w = layer_on_gpu(n_in, n_out, M, r, tag="dropall")
+    ws = q.Workspace()
+    keep = torch.zeros((M, r), dtype=torch.uint8, device="cuda")
+    Y, V = q.qlora_linear_fwd(w, t["X"], t["A"], t["B"], ws, dropout_keep=keep, dropout_p=0.5)
+    dX, dA, dB = q.qlora_linear_bwd(w, t["X"], V, t["dY"], t["A"], t["B"], ws, dropout_keep=keep, dropout_p=0.5)
+    Y0, _ = q.qlora_linear_fwd(w, t["X"], t["A"], torch.zeros_like(t["B"]), ws)
+    torch.cuda.synchronize()
+    assert torch.equal(Y, Y0)
+    assert torch.count_nonzero(dA).item() == 0 and torch.count_nonzero(dB).item() == 0
