@@ -23,6 +23,11 @@ What is computed, and where the pages say so:
   float ("LoRA & QLoRA", "Double Quantization").  Reading: OCP FP8 E4M3,
   one fp32 scale per 256 consecutive absmax values, s = fl32(max / 448),
   code = E4M3_RNE_satfinite(fl32(absmax / s)); no mean-centering.
+* Alternative double quantisation (``dq_format="u8"``): the same 8 bits read as
+  a linear unsigned integer ("QLoRA (low-rank adapters on a quantized model)",
+  "What QLoRA adds over LoRA": the per-block scales are quantised to 8 bits,
+  no format named).  Per group of 256 absmax values s = fl32(max / 255) and
+  code = min(255, rint(fl32(absmax / s))) with ties to even; a' = fl32(code s).
 * Dequantisation: level[code] * absmax' in fp32, then bf16 for the matmul
   ("QLoRA (low-rank adapters on a quantized model)", last paragraph of
   "What QLoRA adds over LoRA"; "LLMs · QLoRA", ``levels[idx] * scale``).
@@ -44,6 +49,8 @@ import numpy as np
 BLOCK = 64          # weights per absmax block
 GROUP = 256         # absmax values per double-quantisation fp32 scale
 E4M3_MAX = 448.0    # largest finite OCP FP8 E4M3 value
+U8_MAX = 255.0      # largest linear uint8 absmax code
+DQ_FORMATS = ("e4m3", "u8")
 DELTA = 0.5 * (31.0 / 32.0 + 29.0 / 30.0)   # quantile offset of the NF4 construction
 
 
@@ -203,10 +210,15 @@ def unpack_nibbles(packed: np.ndarray) -> np.ndarray:
     return out
 
 
-def double_quant(absmax: np.ndarray, group: int = GROUP):
+def double_quant(absmax: np.ndarray, group: int = GROUP, dq_format: str = "e4m3"):
     """Per group of ``group`` consecutive absmax values: s = fl32(max / 448),
-    c_b = E4M3(fl32(a_b / s)).  A group whose scale is 0 stores codes 0.
-    Returns (uint8 codes [nb], float32 scales [ceil(nb / group)])."""
+    c_b = E4M3(fl32(a_b / s)) (``dq_format="e4m3"``), or s = fl32(max / 255),
+    c_b = min(255, rint(fl32(a_b / s))) with ties to even (``"u8"``).  A group
+    whose scale is 0 stores codes 0.  Returns (uint8 codes [nb], float32 scales
+    [ceil(nb / group)])."""
+    if dq_format not in DQ_FORMATS:
+        raise ValueError(f"unknown double-quant format {dq_format!r}")
+    top = E4M3_MAX if dq_format == "e4m3" else U8_MAX
     a = np.asarray(absmax, dtype=np.float32)
     nb = a.size
     ng = (nb + group - 1) // group
@@ -214,17 +226,21 @@ def double_quant(absmax: np.ndarray, group: int = GROUP):
     scales = np.zeros(ng, dtype=np.float32)
     for g in range(ng):
         seg = a[g * group:(g + 1) * group]
-        s = fl32(np.float64(seg.max()) / E4M3_MAX)
+        s = fl32(np.float64(seg.max()) / top)
         scales[g] = s
         if s > 0:
             y = fl32(seg.astype(np.float64) / np.float64(s))
-            codes[g * group:(g + 1) * group] = e4m3_encode(y)
+            if dq_format == "e4m3":
+                codes[g * group:(g + 1) * group] = e4m3_encode(y)
+            else:
+                codes[g * group:(g + 1) * group] = np.minimum(np.rint(y.astype(np.float64)), U8_MAX).astype(np.uint8)
     return codes, scales
 
 
-def quantize_nf4(W0: np.ndarray):
+def quantize_nf4(W0: np.ndarray, dq_format: str = "e4m3"):
     """fp32 W0 (in, out), row-major -> (packed NF4 codes [in*out/2],
-    E4M3 absmax codes [in*out/64], fp32 group scales [ceil(in*out/64/256)]).
+    E4M3 (or linear uint8) absmax codes [in*out/64], fp32 group scales
+    [ceil(in*out/64/256)]).
 
     Weights are coded against the exact fp32 absmax first; the absmax values are
     quantised afterwards (the order the pages list the two steps in)."""
@@ -235,29 +251,33 @@ def quantize_nf4(W0: np.ndarray):
         raise ValueError("W0 must be finite")
     a = block_absmax(w)
     codes = nearest_level(scaled(w, a), nf4_codebook())
-    dq_codes, dq_scales = double_quant(a)
+    dq_codes, dq_scales = double_quant(a, dq_format=dq_format)
     return pack_nibbles(codes), dq_codes, dq_scales
 
 
-def absmax_dequant(dq_codes: np.ndarray, dq_scales: np.ndarray, group: int = GROUP) -> np.ndarray:
-    """a'_b = fl32(e4m3(c_b) * s_g) (float32 [nb])."""
+def absmax_dequant(dq_codes: np.ndarray, dq_scales: np.ndarray, group: int = GROUP,
+                   dq_format: str = "e4m3") -> np.ndarray:
+    """a'_b = fl32(e4m3(c_b) * s_g), or fl32(c_b * s_g) for ``"u8"`` (float32 [nb])."""
+    if dq_format not in DQ_FORMATS:
+        raise ValueError(f"unknown double-quant format {dq_format!r}")
     c = np.asarray(dq_codes, dtype=np.uint8)
     s = np.asarray(dq_scales, dtype=np.float32).astype(np.float64)
     g = np.arange(c.size) // group
-    return fl32(e4m3_decode(c) * s[g])
+    v = e4m3_decode(c) if dq_format == "e4m3" else c.astype(np.float64)
+    return fl32(v * s[g])
 
 
-def dequantize(codes, dq_codes, dq_scales, n_in: int, n_out: int) -> np.ndarray:
+def dequantize(codes, dq_codes, dq_scales, n_in: int, n_out: int, dq_format: str = "e4m3") -> np.ndarray:
     """w' = fl32(level[code] * a'_b) as float32 (n_in, n_out)."""
     lv = nf4_codebook().astype(np.float64)
     c = unpack_nibbles(codes).reshape(-1, BLOCK)
-    a = absmax_dequant(dq_codes, dq_scales).astype(np.float64)
+    a = absmax_dequant(dq_codes, dq_scales, dq_format=dq_format).astype(np.float64)
     return fl32(lv[c] * a[:, None]).reshape(n_in, n_out)
 
 
-def dequantize_bf16(codes, dq_codes, dq_scales, n_in: int, n_out: int) -> np.ndarray:
+def dequantize_bf16(codes, dq_codes, dq_scales, n_in: int, n_out: int, dq_format: str = "e4m3") -> np.ndarray:
     """bf16(w'): the operand the matmuls use (float32 array holding bf16 values)."""
-    return round_bf16(dequantize(codes, dq_codes, dq_scales, n_in, n_out))
+    return round_bf16(dequantize(codes, dq_codes, dq_scales, n_in, n_out, dq_format))
 
 
 # --------------------------------------------------------------------------

@@ -279,3 +279,76 @@ def test_quantize_rejects_bad_input():
         nf4.quantize_nf4(np.full((2, 64), np.nan, dtype=np.float32))
     with pytest.raises(ValueError):
         nf4.quantize_nf4(np.zeros((3, 7), dtype=np.float32))
+
+
+# ---------------------------------------------------------------------------
+# the linear-uint8 reading of the 8-bit double quantisation
+
+
+def test_u8_double_quant_grid_points_and_ends():
+    """Values on the grid k * s come back as code k; the group maximum is code
+    255 and zero is code 0; the scale is fl32(max / 255)."""
+    top = np.float32(3.0)
+    s = np.float32(np.float64(top) / 255.0)
+    ks = np.array([0, 1, 2, 17, 128, 200, 254], dtype=np.int64)
+    vals = (ks.astype(np.float64) * np.float64(s)).astype(np.float32)
+    a = np.concatenate([vals, [top]]).astype(np.float32)
+    codes, scales = nf4.double_quant(a, dq_format="u8")
+    assert scales[0] == s
+    assert list(codes[:-1]) == list(ks) and codes[-1] == 255
+
+
+def test_u8_double_quant_ties_to_even():
+    """Half-way values (k + 1/2) s, exactly representable, round to the even
+    neighbour (a round-half-up coder would give k + 1 for every even k)."""
+    s = np.float32(0.25)                       # max = 63.75 -> s = 0.25 exactly
+    top = np.float32(63.75)
+    a = np.array([top] + [(k + 0.5) * 0.25 for k in range(0, 20)], dtype=np.float32)
+    codes, scales = nf4.double_quant(a, dq_format="u8")
+    assert scales[0] == s
+    for k in range(20):
+        assert codes[1 + k] == (k if k % 2 == 0 else k + 1), k
+
+
+def test_u8_double_quant_error_bound_and_monotone():
+    """Decoded absmax within half a step (plus rounding) of the exact value, and
+    codes non-decreasing in the absmax, on a group of random values."""
+    rng = np.random.default_rng(11)
+    a = np.sort(rng.uniform(0.0, 0.07, 256)).astype(np.float32)
+    codes, scales = nf4.double_quant(a, dq_format="u8")
+    dec = nf4.absmax_dequant(codes, scales, dq_format="u8").astype(np.float64)
+    s = float(scales[0])
+    assert np.all(np.abs(dec - a.astype(np.float64)) <= 0.5 * s * (1 + 1e-6) + 1e-9)
+    assert np.all(np.diff(codes.astype(int)) >= 0)
+
+
+def test_u8_zero_group_and_weight_codes_independent_of_format():
+    """An all-zero group has scale 0 and codes 0; the packed NF4 weight codes are
+    the same in both formats (they use the exact absmax), only the stored absmax
+    differs."""
+    codes, scales = nf4.double_quant(np.zeros(300, np.float32), dq_format="u8")
+    assert not np.any(codes) and not np.any(scales)
+    W = np.random.default_rng(2).standard_normal((64, 512)).astype(np.float32) * 0.02
+    c8, q8, s8 = nf4.quantize_nf4(W, dq_format="e4m3")
+    cu, qu, su = nf4.quantize_nf4(W, dq_format="u8")
+    assert np.array_equal(c8, cu)
+    assert not np.array_equal(q8, qu)
+
+
+def test_u8_more_precise_for_large_blocks():
+    """Where a group's absmax values all lie in [max/2, max] the linear code's
+    relative error (<= 1/255) is below E4M3's worst case (2^-4), and on such a
+    group it is smaller on average."""
+    rng = np.random.default_rng(5)
+    a = rng.uniform(0.5, 1.0, 256).astype(np.float32)
+    cu, su = nf4.double_quant(a, dq_format="u8")
+    ce, se = nf4.double_quant(a, dq_format="e4m3")
+    eu = np.abs(nf4.absmax_dequant(cu, su, dq_format="u8") - a) / a
+    ee = np.abs(nf4.absmax_dequant(ce, se) - a) / a
+    assert eu.max() <= 1 / 255 * (1 + 1e-6) and ee.max() <= 2 ** -4
+    assert eu.mean() < ee.mean()
+
+
+def test_unknown_dq_format_rejected():
+    with pytest.raises(ValueError):
+        nf4.double_quant(np.ones(4, np.float32), dq_format="fp16")
