@@ -73,16 +73,23 @@ typedef enum qlora_op { QLORA_OP_FWD = 1, QLORA_OP_BWD = 2 } qlora_op;
 #define QLORA_BLOCK 64   /* weights per absmax block */
 #define QLORA_GROUP 256  /* absmax values per double-quantisation fp32 scale */
 
+/* Formats of the 8-bit absmax codes (qlora_nf4_weight.dq_format). */
+#define QLORA_DQ_E4M3 0  /* OCP FP8 E4M3, s = max / 448 ("LoRA & QLoRA": an 8-bit float) */
+#define QLORA_DQ_U8 1    /* linear unsigned integer, s = max / 255 ("8 bits", pigeon guide) */
+
 /*
  * The frozen, quantised weight (non-owning view; all pointers [device]).
  *   codes     : uint8[in*out/2]  NF4 codes of the flattened row-major (in, out) W0;
  *               element 2k in the low nibble of byte k, element 2k+1 in the high nibble.
- *   dq_codes  : uint8[in*out/64] E4M3 code of each block's absmax (block b = elements
- *               64b .. 64b+63 of the flattened W0).
+ *   dq_codes  : uint8[in*out/64] 8-bit code of each block's absmax (block b = elements
+ *               64b .. 64b+63 of the flattened W0), in the format dq_format.
  *   dq_scales : fp32[ceil(in*out/64/256)] scale of each group of 256 consecutive blocks.
  *   in, out   : matrix shape.
+ *   dq_format : QLORA_DQ_E4M3 (0, what a zero-initialised descriptor holds) or
+ *               QLORA_DQ_U8; anything else is QLORA_ERR_INVALID_ARG.
  * Dequantised weight ("What QLoRA adds over LoRA"; "LLMs · QLoRA" levels[idx]*scale):
- *   absmax'_b = fl32(e4m3(dq_codes[b]) * dq_scales[b/256])
+ *   absmax'_b = fl32(e4m3(dq_codes[b]) * dq_scales[b/256])   (E4M3)
+ *             = fl32(dq_codes[b] * dq_scales[b/256])         (U8)
  *   w'        = fl32(nf4_level[code] * absmax'_b)   (fl32 = IEEE binary32 round-to-nearest)
  * and the matmuls use bf16(w') (round to nearest even).
  */
@@ -92,6 +99,7 @@ typedef struct qlora_nf4_weight {
   const float* dq_scales;
   int64_t in;
   int64_t out;
+  int32_t dq_format;
 } qlora_nf4_weight;
 
 /*
@@ -111,6 +119,16 @@ typedef struct qlora_nf4_weight {
  */
 QLORA_API qlora_status qlora_quantize_nf4(const float* W0, int64_t in, int64_t out, uint8_t* codes,
                                 uint8_t* dq_codes, float* dq_scales, void* stream);
+
+/*
+ * qlora_quantize_nf4 with a choice of absmax code format (dq_format, as in
+ * qlora_nf4_weight).  QLORA_DQ_U8: per group s_g = fl32(max_b a_b / 255) and
+ * dq_codes[b] = min(255, rint(fl32(a_b / s_g))) with ties to even (0 when
+ * s_g = 0).  The NF4 codes are the same in both formats (they use the exact
+ * absmax).  Unknown formats give QLORA_ERR_INVALID_ARG.
+ */
+QLORA_API qlora_status qlora_quantize_nf4_ex(const float* W0, int64_t in, int64_t out, uint8_t* codes,
+                                             uint8_t* dq_codes, float* dq_scales, int dq_format, void* stream);
 
 /*
  * Dequantise the frozen weight to a dense (in, out) matrix: W_out[k][n] = w'

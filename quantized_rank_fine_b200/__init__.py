@@ -36,8 +36,11 @@ EXPORTS = (
     "qlora_workspace_bytes", "qlora_ws_init", "qlora_ws_status", "qlora_nf4_codebook",
     "qlora_adapter_params", "qlora_status_string", "qlora_time_kernel", "qlora_launch_count",
     "qlora_linear_fwd_static_ws", "qlora_linear_bwd_adam", "qlora_linear_fwd_ex", "qlora_linear_bwd_ex",
-    "qlora_gemm_set_ctas",
+    "qlora_gemm_set_ctas", "qlora_quantize_nf4_ex",
 )
+
+# Formats of the absmax codes (NF4Weight.dq_format).
+QLORA_DQ_E4M3, QLORA_DQ_U8 = 0, 1
 
 # Flag of qlora_linear_opts.flags.
 QLORA_ACCUMULATE_GRADS = 1
@@ -55,7 +58,7 @@ class QLoRAError(RuntimeError):
 
 class _Weight(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("dq_codes", ctypes.c_void_p), ("dq_scales", ctypes.c_void_p),
-                ("in_", ctypes.c_int64), ("out", ctypes.c_int64)]
+                ("in_", ctypes.c_int64), ("out", ctypes.c_int64), ("dq_format", ctypes.c_int32)]
 
 
 class _AdamHparams(ctypes.Structure):
@@ -99,6 +102,7 @@ def lib() -> ctypes.CDLL:
             "qlora_time_kernel": (i32, [i32, ctypes.POINTER(vp), ctypes.POINTER(vp), i32]),
             "qlora_launch_count": (ctypes.c_uint64, []),
             "qlora_gemm_set_ctas": (i32, [i32]),
+            "qlora_quantize_nf4_ex": (i32, [vp, i64, i64, vp, vp, vp, i32, vp]),
             "qlora_linear_fwd_static_ws": (i32, [wp, vp, i64, vp, vp, i32, vp, vp, vp]),
             "qlora_linear_bwd_adam": (i32, [wp, vp, vp, vp, i64, vp, vp, i32, vp, ctypes.POINTER(_AdamState),
                                             ctypes.POINTER(_AdamHparams), ctypes.POINTER(_LinearOpts), vp, sz,
@@ -138,15 +142,18 @@ def _stream(stream=None):
 
 @dataclass
 class NF4Weight:
-    """The frozen quantised weight: packed codes, E4M3 absmax codes, fp32 group scales."""
+    """The frozen quantised weight: packed codes, 8-bit absmax codes (E4M3, or
+    linear uint8 with dq_format = QLORA_DQ_U8), fp32 group scales."""
     codes: torch.Tensor       # uint8 [in*out/2]
     dq_codes: torch.Tensor    # uint8 [in*out/64]
     dq_scales: torch.Tensor   # float32 [ceil(in*out/64/256)]
     n_in: int
     n_out: int
+    dq_format: int = 0        # QLORA_DQ_E4M3
 
     def c_struct(self) -> _Weight:
-        return _Weight(_ptr(self.codes), _ptr(self.dq_codes), _ptr(self.dq_scales), self.n_in, self.n_out)
+        return _Weight(_ptr(self.codes), _ptr(self.dq_codes), _ptr(self.dq_scales), self.n_in, self.n_out,
+                       self.dq_format)
 
 
 def qlora_nf4_codebook() -> list:
@@ -218,8 +225,11 @@ class Workspace:
         return lib().qlora_ws_status(_ptr(self.buf), _stream(stream))
 
 
-def qlora_quantize_nf4(W0: torch.Tensor, stream=None, out: NF4Weight | None = None) -> NF4Weight:
-    """W0 fp32 (in, out) on the GPU -> NF4Weight (outputs allocated unless given)."""
+def qlora_quantize_nf4(W0: torch.Tensor, stream=None, out: NF4Weight | None = None,
+                       dq_format: int | None = None) -> NF4Weight:
+    """W0 fp32 (in, out) on the GPU -> NF4Weight (outputs allocated unless given).
+    dq_format: QLORA_DQ_E4M3 (default) or QLORA_DQ_U8 (linear uint8 absmax codes);
+    a given `out` keeps its own format unless one is passed."""
     n_in, n_out = W0.shape
     n = n_in * n_out
     if out is None:
@@ -228,8 +238,15 @@ def qlora_quantize_nf4(W0: torch.Tensor, stream=None, out: NF4Weight | None = No
                         torch.empty(n // BLOCK, dtype=torch.uint8, device=dev),
                         torch.empty((n // BLOCK + GROUP - 1) // GROUP, dtype=torch.float32, device=dev),
                         n_in, n_out)
-    _check(lib().qlora_quantize_nf4(_ptr(W0), n_in, n_out, _ptr(out.codes), _ptr(out.dq_codes),
-                                    _ptr(out.dq_scales), _stream(stream)), "qlora_quantize_nf4")
+    if dq_format is not None:
+        out.dq_format = dq_format
+    if out.dq_format == QLORA_DQ_E4M3:
+        _check(lib().qlora_quantize_nf4(_ptr(W0), n_in, n_out, _ptr(out.codes), _ptr(out.dq_codes),
+                                        _ptr(out.dq_scales), _stream(stream)), "qlora_quantize_nf4")
+    else:
+        _check(lib().qlora_quantize_nf4_ex(_ptr(W0), n_in, n_out, _ptr(out.codes), _ptr(out.dq_codes),
+                                           _ptr(out.dq_scales), out.dq_format, _stream(stream)),
+               "qlora_quantize_nf4_ex")
     return out
 
 

@@ -72,6 +72,7 @@ bool linear_shape_ok(int64_t M, int64_t in, int64_t out, int r) {
 
 qlora_status check_weight_shape(const qlora_nf4_weight* w) {
   if (!w || !w->codes || !w->dq_codes || !w->dq_scales) return QLORA_ERR_INVALID_ARG;
+  if (w->dq_format != QLORA_DQ_E4M3 && w->dq_format != QLORA_DQ_U8) return QLORA_ERR_INVALID_ARG;
   if (w->in < 1 || w->out < 1 || w->in > (int64_t(1) << 40) / w->out || (w->in * w->out) % QLORA_BLOCK != 0)
     return QLORA_ERR_SHAPE;
   return QLORA_OK;
@@ -85,7 +86,9 @@ qlora_status check_weight(const qlora_nf4_weight* w) {
   return QLORA_OK;
 }
 
-WeightView view(const qlora_nf4_weight* w) { return WeightView{w->codes, w->dq_codes, w->dq_scales, w->in, w->out}; }
+WeightView view(const qlora_nf4_weight* w) {
+  return WeightView{w->codes, w->dq_codes, w->dq_scales, w->in, w->out, w->dq_format == QLORA_DQ_U8};
+}
 
 // Workspace layout (byte offsets), shared by the size query and the calls:
 // the fixed prefix (status word, the GEMM's split counters), V (when the
@@ -245,14 +248,21 @@ qlora_status qlora_ws_status(void* ws, void* stream) {
 
 qlora_status qlora_quantize_nf4(const float* W0, int64_t in, int64_t out, uint8_t* codes, uint8_t* dq_codes,
                                 float* dq_scales, void* stream) {
+  return qlora_quantize_nf4_ex(W0, in, out, codes, dq_codes, dq_scales, QLORA_DQ_E4M3, stream);
+}
+
+qlora_status qlora_quantize_nf4_ex(const float* W0, int64_t in, int64_t out, uint8_t* codes, uint8_t* dq_codes,
+                                   float* dq_scales, int dq_format, void* stream) {
   if (!W0 || !codes || !dq_codes || !dq_scales) return QLORA_ERR_INVALID_ARG;
+  if (dq_format != QLORA_DQ_E4M3 && dq_format != QLORA_DQ_U8) return QLORA_ERR_INVALID_ARG;
   if (in < 1 || out < 1 || in > (int64_t(1) << 40) / out || (in * out) % QLORA_BLOCK != 0) return QLORA_ERR_SHAPE;
   QLORA_TRY(check_device());
   QLORA_TRY(check_ptr(W0));
   QLORA_TRY(check_ptr(codes));
   QLORA_TRY(check_ptr(dq_codes));
   QLORA_TRY(check_ptr(dq_scales));
-  QLORA_CUDA(qlora::launch_quantize_nf4(W0, in * out, codes, dq_codes, dq_scales, static_cast<cudaStream_t>(stream)));
+  QLORA_CUDA(qlora::launch_quantize_nf4(W0, in * out, codes, dq_codes, dq_scales, static_cast<cudaStream_t>(stream),
+                                        dq_format == QLORA_DQ_U8));
   return QLORA_OK;
 }
 
@@ -263,7 +273,7 @@ qlora_status qlora_dequantize(const qlora_nf4_weight* w, void* W_out, int out_dt
   QLORA_TRY(check_weight(w));
   QLORA_TRY(check_ptr(W_out));
   QLORA_CUDA(qlora::launch_dequantize(w->codes, w->dq_codes, w->dq_scales, w->in * w->out, out_dtype == QLORA_BF16,
-                                      W_out, static_cast<cudaStream_t>(stream)));
+                                      W_out, static_cast<cudaStream_t>(stream), w->dq_format == QLORA_DQ_U8));
   return QLORA_OK;
 }
 
@@ -278,7 +288,8 @@ qlora_status qlora_merge(const qlora_nf4_weight* w, const uint16_t* A, const uin
   QLORA_TRY(check_ptr(B));
   QLORA_TRY(check_ptr(W_out));
   QLORA_CUDA(qlora::launch_merge(w->codes, w->dq_codes, w->dq_scales, A, B, r, w->in, w->out,
-                                 out_dtype == QLORA_BF16, W_out, static_cast<cudaStream_t>(stream)));
+                                 out_dtype == QLORA_BF16, W_out, static_cast<cudaStream_t>(stream),
+                                 w->dq_format == QLORA_DQ_U8));
   return QLORA_OK;
 }
 

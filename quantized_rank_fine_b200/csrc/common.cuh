@@ -64,9 +64,10 @@ __device__ __forceinline__ float e4m3_to_float(uint8_t c) {
   return __half2float(__half(h));
 }
 
-// Dequantised block absmax: fl32(e4m3(c) * s).
-__device__ __forceinline__ float absmax_deq(uint8_t c, float s) {
-  return mul_rn(e4m3_to_float(c), s);
+// Dequantised block absmax: fl32(e4m3(c) * s), or fl32(c * s) when the absmax
+// codes are linear uint8 (u8; the same for every thread of a launch).
+__device__ __forceinline__ float absmax_deq(uint8_t c, float s, bool u8) {
+  return mul_rn(u8 ? static_cast<float>(c) : e4m3_to_float(c), s);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

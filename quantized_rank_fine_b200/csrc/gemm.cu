@@ -87,6 +87,7 @@ struct GemmArgs {
   int r;
   uint16_t* D;        // bf16 (M, N)
   uint32_t* status;
+  int dq_u8;          // absmax codes are linear uint8 (else E4M3)
   // schedule (see the file header)
   int tiles_n;        // pair tiles along N; tile t covers rows (t / tiles_n) * 512, columns (t % tiles_n) * 256
   int dp_tiles;       // tiles [0, dp_tiles): whole items, round robin over the pairs
@@ -416,7 +417,7 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
                        : "=r"(wd[0]), "=r"(wd[1]), "=r"(wd[2]), "=r"(wd[3]) : "r"(csrc + code_off0));
           asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                        : "=r"(wd[4]), "=r"(wd[5]), "=r"(wd[6]), "=r"(wd[7]) : "r"(csrc + code_off1));
-          const BlockLut lut = make_lut(valid ? absmax_deq(dqc, dqs) : 0.0f);
+          const BlockLut lut = make_lut(valid ? absmax_deq(dqc, dqs, p.dq_u8 != 0) : 0.0f);
           if (valid && kb + 4 < nkb_w) {
             const int64_t nb = blk + (kb + 4) * blk_step;
             dqc = __ldg(p.dq_codes + nb);
@@ -697,7 +698,8 @@ cudaError_t launch_fwd_gemm(const WeightView& w, const uint16_t* X, const uint16
       !make_map(&eb, B, r, w.out, 64, 64) ||
       !make_map_t(&cm, w.codes, w.in, w.out / 2, 64, 64, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
-  GemmArgs a{w.codes, w.dq_codes, w.dq_scales, w.out, M, w.out, w.in, r, Y, status, 0, 0, 0, nullptr, nullptr};
+  GemmArgs a{w.codes, w.dq_codes, w.dq_scales, w.out, M, w.out, w.in, r, Y, status, w.dq_u8 ? 1 : 0,
+             0, 0, 0, nullptr, nullptr};
   return launch_gemm<false>(act, ea, eb, cm, a, counters, partials, partial_bytes, stream);
 }
 
@@ -712,7 +714,8 @@ cudaError_t launch_dx_gemm(const WeightView& w, const uint16_t* dY, const uint16
       !make_map(&eb, A, w.in, r, 64, 128) ||
       !make_map_t(&cm, w.codes, w.in, w.out / 2, 32, 128, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, CU_TENSOR_MAP_SWIZZLE_32B))
     return cudaErrorInvalidValue;
-  GemmArgs a{w.codes, w.dq_codes, w.dq_scales, w.out, M, w.in, w.out, r, dX, status, 0, 0, 0, nullptr, nullptr};
+  GemmArgs a{w.codes, w.dq_codes, w.dq_scales, w.out, M, w.in, w.out, r, dX, status, w.dq_u8 ? 1 : 0,
+             0, 0, 0, nullptr, nullptr};
   return launch_gemm<true>(act, ea, eb, cm, a, counters, partials, partial_bytes, stream);
 }
 

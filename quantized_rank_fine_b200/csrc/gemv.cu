@@ -83,6 +83,7 @@ struct GemvArgs {
   uint16_t* Y;           // (M, N) bf16
   int Kc;                // rows per split (multiple of 64)
   uint32_t* status;
+  int dq_u8;             // absmax codes are linear uint8 (else E4M3)
 };
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -237,7 +238,7 @@ nf4_gemv_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
       const int s = i % kGvStages;
       const uint32_t ph = (i / kGvStages) & 1;
       if (i < nstage) {
-        asl[lane] = absmax_deq(static_cast<uint8_t>(qc), qs);
+        asl[lane] = absmax_deq(static_cast<uint8_t>(qc), qs, p.dq_u8 != 0);
         load_scale(i + 2, qc, qs);
         __syncwarp();   // the slice is complete
       }
@@ -526,7 +527,7 @@ cudaError_t launch_gemv(const WeightView& w, const uint16_t* X, const uint16_t* 
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  GemvArgs a{w.dq_codes, w.dq_scales, w.in, w.out, static_cast<int>(M), r, Y, Kc, status};
+  GemvArgs a{w.dq_codes, w.dq_scales, w.in, w.out, static_cast<int>(M), r, Y, Kc, status, w.dq_u8 ? 1 : 0};
 
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>((w.out + kTileCols - 1) / kTileCols), static_cast<unsigned>(S));

@@ -33,15 +33,17 @@ struct WeightView {
   const uint8_t* dq_codes;
   const float* dq_scales;
   int64_t in, out;
+  bool dq_u8;         // absmax codes are linear uint8 (else E4M3)
 };
 
+// dq_u8 / u8: the absmax codes are linear uint8 (s = max / 255) instead of E4M3.
 cudaError_t launch_quantize_nf4(const float* W0, int64_t n, uint8_t* codes, uint8_t* dq_codes,
-                                float* dq_scales, cudaStream_t stream);
+                                float* dq_scales, cudaStream_t stream, bool dq_u8 = false);
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* dq_codes, const float* dq_scales,
-                              int64_t n, bool bf16, void* out, cudaStream_t stream);
+                              int64_t n, bool bf16, void* out, cudaStream_t stream, bool u8 = false);
 cudaError_t launch_merge(const uint8_t* codes, const uint8_t* dq_codes, const float* dq_scales,
                          const uint16_t* A, const uint16_t* B, int r, int64_t n_in, int64_t n_out,
-                         bool bf16, void* out, cudaStream_t stream);
+                         bool bf16, void* out, cudaStream_t stream, bool u8 = false);
 
 // One Adam step fused into a gradient's final store (see qlora_linear_bwd_adam):
 // the element g of parameter index i updates theta[i], m[i], v[i] and p16[i].

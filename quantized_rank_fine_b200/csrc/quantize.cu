@@ -5,7 +5,9 @@
 //   per block of 64 consecutive weights:  a = max |w|,  x = fl32(w / a),
 //     code = index of the nearest NF4 level (ties to the lower level);
 //   per group of 256 consecutive blocks:  s = fl32(max a / 448),
-//     dq_code = E4M3_RNE_satfinite(fl32(a / s))   (0 when s = 0).
+//     dq_code = E4M3_RNE_satfinite(fl32(a / s))   (0 when s = 0);
+//   or, with linear uint8 absmax codes, s = fl32(max a / 255) and
+//     dq_code = min(255, rint(fl32(a / s)))  (ties to even; 0 when s = 0).
 //
 // Layout: a persistent grid of two 256-thread CTAs per SM walks the groups
 // (16,384 weights = 64 KB of fp32 each), every group as two halves of 128 blocks.
@@ -94,7 +96,7 @@ __device__ __forceinline__ void issue_half(int64_t j, const float* W0, int64_t n
 
 __global__ void __launch_bounds__(kQThreads, 2)
 quantize_nf4_kernel(const float* __restrict__ W0, int64_t nblocks, int64_t ngroups, uint8_t* __restrict__ codes,
-                    uint8_t* __restrict__ dq_codes, float* __restrict__ dq_scales) {
+                    uint8_t* __restrict__ dq_codes, float* __restrict__ dq_scales, bool dq_u8) {
   extern __shared__ __align__(128) uint8_t qsmem[];
   __shared__ uint32_t lut[kCells];
   __shared__ float thr_exact[16];
@@ -205,12 +207,13 @@ quantize_nf4_kernel(const float* __restrict__ W0, int64_t nblocks, int64_t ngrou
     gm = red[0];
 #pragma unroll
     for (int w = 1; w < kQThreads / 32; ++w) gm = fmaxf(gm, red[w]);
-    const float sc = __fdiv_rn(gm, 448.0f);
+    const float sc = __fdiv_rn(gm, dq_u8 ? 255.0f : 448.0f);
     if (tid < nblk) {
       uint8_t c = 0;
       if (sc > 0.0f) {
         const float y = __fdiv_rn(amax[tid], sc);
-        c = static_cast<uint8_t>(__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3));
+        c = dq_u8 ? static_cast<uint8_t>(fminf(rintf(y), 255.0f))
+                  : static_cast<uint8_t>(__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3));
       }
       dq_codes[blk0 + tid] = c;
     }
@@ -232,7 +235,7 @@ quantize_nf4_kernel(const float* __restrict__ W0, int64_t nblocks, int64_t ngrou
 }  // namespace
 
 cudaError_t launch_quantize_nf4(const float* W0, int64_t n, uint8_t* codes, uint8_t* dq_codes,
-                                float* dq_scales, cudaStream_t stream) {
+                                float* dq_scales, cudaStream_t stream, bool dq_u8) {
   const int64_t nblocks = n / kBlock;
   const int64_t ngroups = (nblocks + kGroup - 1) / kGroup;
   if (ngroups == 0) return cudaSuccess;
@@ -250,7 +253,7 @@ cudaError_t launch_quantize_nf4(const float* W0, int64_t n, uint8_t* codes, uint
   const int64_t grid = std::min<int64_t>(ngroups, 2 * (dev < 64 ? sms[dev] : 148));
   timing_before(QLORA_KERNEL_QUANTIZE, stream);
   quantize_nf4_kernel<<<static_cast<unsigned>(grid), kQThreads, kQBuf * kHalfBytes, stream>>>(
-      W0, nblocks, ngroups, codes, dq_codes, dq_scales);
+      W0, nblocks, ngroups, codes, dq_codes, dq_scales, dq_u8);
   timing_after(QLORA_KERNEL_QUANTIZE, stream);
   count_launch();
   return cudaGetLastError();

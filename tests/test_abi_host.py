@@ -140,6 +140,16 @@ def test_ex_options_rejected_before_launch(L):
     assert fwd(wp, FAKE, 64, FAKE, FAKE, 12, FAKE, None, ctypes.byref(o), FAKE, 1 << 30, None) == 2
 
 
+def test_unknown_absmax_format_rejected(L):
+    """A weight descriptor or a quantise call with an unknown absmax code format
+    is refused before any launch."""
+    w = q._Weight(0x10000, 0x10000, 0x10000, 256, 256, 9)
+    assert L.qlora_dequantize(ctypes.byref(w), FAKE, 0, None) == 1
+    assert L.qlora_linear_fwd(ctypes.byref(w), FAKE, 64, FAKE, FAKE, 8, FAKE, None, FAKE, 1 << 30, None) == 1
+    assert L.qlora_quantize_nf4_ex(FAKE, 64, 64, FAKE, FAKE, FAKE, 2, None) == 1
+    assert L.qlora_quantize_nf4_ex(FAKE, 64, 64, FAKE, FAKE, FAKE, -1, None) == 1
+
+
 def test_dequant_merge_reject_before_launch(L):
     w = q._Weight(0x10000, 0x10000, 0x10000, 256, 256)
     assert L.qlora_dequantize(ctypes.byref(w), FAKE, 5, None) == 1                      # bad dtype
