@@ -24,7 +24,12 @@ Modules:
 
 * ``oracle.nf4``    -- codebook, blockwise absmax, nearest-level encode, E4M3
   double quantisation, dequantisation, bf16 rounding, the blog's experiment.
-* ``oracle.linear`` -- forward, backward, merge and parameter counts.
+* ``oracle.linear`` -- forward, backward (adapter scale, dropout), merge and
+  parameter counts.
+* ``oracle.adam``   -- the Adam / AdamW step on the adapters.
+* ``oracle.loftq``  -- merge -> re-quantise round trip and the SVD initialisation.
+* ``oracle.intq``   -- the symmetric uniform INT quantiser with one scale per 16
+  weights (2-bit ternary, 3 and 4 bits).
 
 Every function is pinned by a ``-m "not gpu"`` test in ``tests/test_oracle_*.py``
 against something other than itself (printed values, closed forms, brute force,
