@@ -131,6 +131,31 @@ QLORA_API qlora_status qlora_quantize_nf4_ex(const float* W0, int64_t in, int64_
                                              uint8_t* dq_codes, float* dq_scales, int dq_format, void* stream);
 
 /*
+ * The second base quantiser, of the pages' simulation ("QLoRA (low-rank adapters
+ * on a quantized model)", "The code, line by line": symmetric uniform integers,
+ * one scale per 16 consecutive entries of the flattened (in, out) matrix; no NF4
+ * and no double quantisation; "What the simulations show": 2, 3 and 4 bits, 2-bit
+ * being ternary {-s, 0, s}).  Per group of 16 weights, Q = 2^(bits-1) - 1:
+ *   s = fl32(max |w| / Q),  q = clamp(rint(fl32(w / s)), -Q, Q) (ties to even;
+ *   0 when s = 0),  stored as the nibble q + 8 (packing as for NF4);
+ *   w' = fl32(q s).
+ *   W0      [device] fp32 (in, out).
+ *   bits    2, 3 or 4, else QLORA_ERR_INVALID_ARG.
+ *   codes   [device] out: uint8[in*out/2].
+ *   scales  [device] out: fp32[in*out/16].
+ *   All pointers 16-byte aligned (QLORA_ERR_ALIGNMENT otherwise).
+ * Requires in*out % 16 == 0.  Bit-exact.  (The adapted-layer calls take NF4
+ * weights only; this format is quantised and dequantised here.)
+ */
+QLORA_API qlora_status qlora_quantize_int(const float* W0, int64_t in, int64_t out, int bits, uint8_t* codes,
+                                          float* scales, void* stream);
+
+/* Dense w' (QLORA_F32) or bf16(w') (QLORA_BF16), (in, out), of a weight quantised
+ * by qlora_quantize_int.  Bit-exact. */
+QLORA_API qlora_status qlora_dequantize_int(const uint8_t* codes, const float* scales, int64_t in, int64_t out,
+                                            void* W_out, int out_dtype, void* stream);
+
+/*
  * Dequantise the frozen weight to a dense (in, out) matrix: W_out[k][n] = w'
  * (QLORA_F32) or bf16(w') (QLORA_BF16).  Bit-exact.
  *   w      [host] descriptor of [device] tensors.

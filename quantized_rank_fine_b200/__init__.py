@@ -36,7 +36,7 @@ EXPORTS = (
     "qlora_workspace_bytes", "qlora_ws_init", "qlora_ws_status", "qlora_nf4_codebook",
     "qlora_adapter_params", "qlora_status_string", "qlora_time_kernel", "qlora_launch_count",
     "qlora_linear_fwd_static_ws", "qlora_linear_bwd_adam", "qlora_linear_fwd_ex", "qlora_linear_bwd_ex",
-    "qlora_gemm_set_ctas", "qlora_quantize_nf4_ex",
+    "qlora_gemm_set_ctas", "qlora_quantize_nf4_ex", "qlora_quantize_int", "qlora_dequantize_int",
 )
 
 # Formats of the absmax codes (NF4Weight.dq_format).
@@ -103,6 +103,8 @@ def lib() -> ctypes.CDLL:
             "qlora_launch_count": (ctypes.c_uint64, []),
             "qlora_gemm_set_ctas": (i32, [i32]),
             "qlora_quantize_nf4_ex": (i32, [vp, i64, i64, vp, vp, vp, i32, vp]),
+            "qlora_quantize_int": (i32, [vp, i64, i64, i32, vp, vp, vp]),
+            "qlora_dequantize_int": (i32, [vp, vp, i64, i64, vp, i32, vp]),
             "qlora_linear_fwd_static_ws": (i32, [wp, vp, i64, vp, vp, i32, vp, vp, vp]),
             "qlora_linear_bwd_adam": (i32, [wp, vp, vp, vp, i64, vp, vp, i32, vp, ctypes.POINTER(_AdamState),
                                             ctypes.POINTER(_AdamHparams), ctypes.POINTER(_LinearOpts), vp, sz,
@@ -247,6 +249,30 @@ def qlora_quantize_nf4(W0: torch.Tensor, stream=None, out: NF4Weight | None = No
         _check(lib().qlora_quantize_nf4_ex(_ptr(W0), n_in, n_out, _ptr(out.codes), _ptr(out.dq_codes),
                                            _ptr(out.dq_scales), out.dq_format, _stream(stream)),
                "qlora_quantize_nf4_ex")
+    return out
+
+
+def qlora_quantize_int(W0: torch.Tensor, bits: int, stream=None):
+    """Symmetric uniform INT quantisation with one scale per 16 weights (bits 2,
+    3 or 4; 2 is ternary): W0 fp32 (in, out) on the GPU -> (codes uint8
+    [in*out/2], scales fp32 [in*out/16])."""
+    n_in, n_out = W0.shape
+    n = n_in * n_out
+    codes = torch.empty(n // 2, dtype=torch.uint8, device=W0.device)
+    scales = torch.empty(n // 16, dtype=torch.float32, device=W0.device)
+    _check(lib().qlora_quantize_int(_ptr(W0), n_in, n_out, bits, _ptr(codes), _ptr(scales), _stream(stream)),
+           "qlora_quantize_int")
+    return codes, scales
+
+
+def qlora_dequantize_int(codes: torch.Tensor, scales: torch.Tensor, n_in: int, n_out: int,
+                         dtype=torch.float32, stream=None, out=None) -> torch.Tensor:
+    """Dense w' (fp32) or bf16(w') of a weight from qlora_quantize_int."""
+    code = QLORA_BF16 if dtype == torch.bfloat16 else QLORA_F32
+    if out is None:
+        out = torch.empty((n_in, n_out), dtype=dtype, device=codes.device)
+    _check(lib().qlora_dequantize_int(_ptr(codes), _ptr(scales), n_in, n_out, _ptr(out), code, _stream(stream)),
+           "qlora_dequantize_int")
     return out
 
 

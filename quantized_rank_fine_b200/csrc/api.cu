@@ -266,6 +266,36 @@ qlora_status qlora_quantize_nf4_ex(const float* W0, int64_t in, int64_t out, uin
   return QLORA_OK;
 }
 
+static bool int_shape_ok(int64_t in, int64_t out) {
+  return in >= 1 && out >= 1 && in <= (int64_t(1) << 40) / out && (in * out) % 16 == 0;
+}
+
+qlora_status qlora_quantize_int(const float* W0, int64_t in, int64_t out, int bits, uint8_t* codes, float* scales,
+                                void* stream) {
+  if (!W0 || !codes || !scales || bits < 2 || bits > 4) return QLORA_ERR_INVALID_ARG;
+  if (!int_shape_ok(in, out)) return QLORA_ERR_SHAPE;
+  QLORA_TRY(check_device());
+  QLORA_TRY(check_ptr(W0));
+  QLORA_TRY(check_ptr(codes));
+  QLORA_TRY(check_ptr(scales));
+  QLORA_CUDA(qlora::launch_int_quantize(W0, in * out, bits, codes, scales, static_cast<cudaStream_t>(stream)));
+  return QLORA_OK;
+}
+
+qlora_status qlora_dequantize_int(const uint8_t* codes, const float* scales, int64_t in, int64_t out, void* W_out,
+                                  int out_dtype, void* stream) {
+  if (!codes || !scales || !W_out || (out_dtype != QLORA_F32 && out_dtype != QLORA_BF16))
+    return QLORA_ERR_INVALID_ARG;
+  if (!int_shape_ok(in, out)) return QLORA_ERR_SHAPE;
+  QLORA_TRY(check_device());
+  QLORA_TRY(check_ptr(codes));
+  QLORA_TRY(check_ptr(scales));
+  QLORA_TRY(check_ptr(W_out));
+  QLORA_CUDA(qlora::launch_int_dequantize(codes, scales, in * out, out_dtype == QLORA_BF16, W_out,
+                                          static_cast<cudaStream_t>(stream)));
+  return QLORA_OK;
+}
+
 qlora_status qlora_dequantize(const qlora_nf4_weight* w, void* W_out, int out_dtype, void* stream) {
   if (out_dtype != QLORA_F32 && out_dtype != QLORA_BF16 || !W_out) return QLORA_ERR_INVALID_ARG;
   QLORA_TRY(check_weight_shape(w));

@@ -45,6 +45,14 @@ cudaError_t launch_merge(const uint8_t* codes, const uint8_t* dq_codes, const fl
                          const uint16_t* A, const uint16_t* B, int r, int64_t n_in, int64_t n_out,
                          bool bf16, void* out, cudaStream_t stream, bool u8 = false);
 
+// Symmetric uniform INT quantisation, one scale per 16 weights (bits 2..4),
+// and its dense dequantisation.  n is a multiple of 16; W0, codes, scales and
+// out 16-byte aligned (8-byte for codes).
+cudaError_t launch_int_quantize(const float* W0, int64_t n, int bits, uint8_t* codes, float* scales,
+                                cudaStream_t stream);
+cudaError_t launch_int_dequantize(const uint8_t* codes, const float* scales, int64_t n, bool bf16, void* out,
+                                  cudaStream_t stream);
+
 // One Adam step fused into a gradient's final store (see qlora_linear_bwd_adam):
 // the element g of parameter index i updates theta[i], m[i], v[i] and p16[i].
 struct AdamParams {

@@ -164,3 +164,14 @@ def test_no_gpu_means_loud_error_not_fallback(L):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert L.qlora_quantize_nf4(FAKE, 64, 64, FAKE, FAKE, FAKE, None) in (5, 6)
+
+
+def test_int_quantiser_rejects_before_launch(L):
+    """The INT group-16 quantiser refuses bad bit widths, shapes and dtypes on
+    the host."""
+    for bits in (1, 5, 8):
+        assert L.qlora_quantize_int(FAKE, 16, 16, bits, FAKE, FAKE, None) == 1
+    assert L.qlora_quantize_int(FAKE, 3, 5, 4, FAKE, FAKE, None) == 2          # in*out % 16
+    assert L.qlora_quantize_int(None, 16, 16, 4, FAKE, FAKE, None) == 1
+    assert L.qlora_dequantize_int(FAKE, FAKE, 16, 16, FAKE, 7, None) == 1      # dtype
+    assert L.qlora_dequantize_int(FAKE, FAKE, 0, 16, FAKE, 0, None) == 2
