@@ -1,0 +1,112 @@
+"""Host-side logic of bench.py on the CPU: the multi-rank plumbing over gloo
+(world size 2), the reference arm's JSON line (the float64 oracle, launched as
+the driver launches it), and the workload bookkeeping.  No GPU is used."""
+
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    import datetime
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    try:
+        bench.barrier(world)
+        got = bench.max_over_ranks(float(10 * rank + 1), world)
+        with open(os.path.join(out_dir, f"r{rank}.txt"), "w") as f:
+            f.write(repr(got))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_world2(tmp_path):
+    """Every rank gets the largest per-rank time (the slowest rank's), after a
+    barrier, on two gloo processes."""
+    port = _free_port()
+    mp.start_processes(_rank_main, args=(2, port, str(tmp_path)), nprocs=2, start_method="spawn", join=True)
+    vals = [float(open(tmp_path / f"r{r}.txt").read()) for r in range(2)]
+    assert vals == [11.0, 11.0]
+
+
+def test_max_over_ranks_single_rank_is_identity():
+    assert bench.max_over_ranks(3.5, 1) == 3.5
+
+
+def _check_reference_line(d, workload, steps, warmup, world):
+    assert d["impl"] == "reference" and d["metric"] == "QLoRA linear fwd+bwd tokens/s"
+    assert d["unit"] == "tokens/s" and d["value"] > 0 and d["higher_is_better"] is True
+    assert d["n_gpus"] == world and d["steps"] == steps and d["warmup"] == warmup
+    assert d["dtype"] == "f64" and d["vs_baseline"] is None and d["scaling"] == "weak"
+    assert d["config"]["workload"] == workload
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    e = d["e2e"]
+    assert e["value"] == d["value"] and e["unit"] == d["unit"]
+    assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_in_process():
+    """The reference arm times the oracle on a bounded sample and fills every key
+    of the contract."""
+    args = bench.argparse.Namespace(workload="linear256_m64_r8", steps=2, warmup=1, gpus=1)
+    d = bench.arm_reference(args, 1, 0)
+    _check_reference_line(d, "linear256_m64_r8", 2, 1, 1)
+    assert bench.arm_reference(args, 2, 1) is None          # only rank 0 runs it
+
+
+def test_reference_arm_torchrun_world2():
+    """Launched as the driver launches N > 1 (torch.distributed.run, 127.0.0.1):
+    exactly one JSON line, from rank 0, and every rank exits 0."""
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py", "--impl", "reference",
+           "--gpus", "2", "--workload", "linear256_m64_r8", "--steps", "1", "--warmup", "0"]
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    p = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [ln for ln in p.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, p.stdout
+    _check_reference_line(json.loads(lines[0]), "linear256_m64_r8", 1, 0, 2)
+
+
+def test_workload_defaults_and_bytes(monkeypatch):
+    """Per-workload defaults, and the stack's activation bytes counting each
+    shared X once (q, k, v share one input, gate and up another)."""
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--workload", "llama7b_stack_m2048_r16"])
+    a = bench.parse()
+    assert (a.steps, a.warmup, a.rows) == (20, 3, "")
+    monkeypatch.setattr(sys, "argv", ["bench.py"])
+    a = bench.parse()
+    assert (a.steps, a.warmup, a.rows, a.workload) == (2000, 10, "all", "attn4096_m4096_r16")
+    wl = bench.WORKLOADS["llama7b_stack_m2048_r16"]
+    assert len(wl["shapes"]) == 224
+    M = wl["M"]
+    unshared = dict(wl)
+    unshared.pop("layer")
+    # q, k, v share one 4096-wide X and gate, up another: 3 + 1 fewer X reads per layer
+    saved = 2 * M * 4096 * (2 + 1) * wl["layers"]
+    assert bench.set_bytes(unshared) - bench.set_bytes(wl) == saved
+
+
+@pytest.mark.parametrize("name", sorted(bench.WORKLOADS))
+def test_workload_config_names_the_workload(name):
+    c = bench.workload_config(name)
+    assert c["workload"] == name and c["M"] == bench.WORKLOADS[name]["M"]
