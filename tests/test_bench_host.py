@@ -101,7 +101,7 @@ def test_workload_defaults_and_bytes(monkeypatch):
     M = wl["M"]
     unshared = dict(wl)
     unshared.pop("layer")
-    # q, k, v share one 4096-wide X and gate, up another: 3 + 1 fewer X reads per layer
+    # k and v read q's X and up reads gate's: three fewer 4096-wide X reads per layer
     saved = 2 * M * 4096 * (2 + 1) * wl["layers"]
     assert bench.set_bytes(unshared) - bench.set_bytes(wl) == saved
 
