@@ -73,9 +73,11 @@ typedef enum qlora_op { QLORA_OP_FWD = 1, QLORA_OP_BWD = 2 } qlora_op;
 #define QLORA_BLOCK 64   /* weights per absmax block */
 #define QLORA_GROUP 256  /* absmax values per double-quantisation fp32 scale */
 
-/* Formats of the 8-bit absmax codes (qlora_nf4_weight.dq_format). */
-#define QLORA_DQ_E4M3 0  /* OCP FP8 E4M3, s = max / 448 ("LoRA & QLoRA": an 8-bit float) */
-#define QLORA_DQ_U8 1    /* linear unsigned integer, s = max / 255 ("8 bits", pigeon guide) */
+/* Weight formats (qlora_nf4_weight.dq_format). */
+#define QLORA_DQ_E4M3 0   /* NF4, absmax codes OCP FP8 E4M3, s = max / 448 ("LoRA & QLoRA": an 8-bit float) */
+#define QLORA_DQ_U8 1     /* NF4, absmax codes linear unsigned integers, s = max / 255 ("8 bits", pigeon guide) */
+#define QLORA_FMT_INT16 2 /* symmetric integers from qlora_quantize_int: level = code - 8, one fp32
+                             scale per 16 weights in dq_scales, no absmax codes (dq_codes unused) */
 
 /*
  * The frozen, quantised weight (non-owning view; all pointers [device]).
@@ -85,8 +87,13 @@ typedef enum qlora_op { QLORA_OP_FWD = 1, QLORA_OP_BWD = 2 } qlora_op;
  *               64b .. 64b+63 of the flattened W0), in the format dq_format.
  *   dq_scales : fp32[ceil(in*out/64/256)] scale of each group of 256 consecutive blocks.
  *   in, out   : matrix shape.
- *   dq_format : QLORA_DQ_E4M3 (0, what a zero-initialised descriptor holds) or
- *               QLORA_DQ_U8; anything else is QLORA_ERR_INVALID_ARG.
+ *   dq_format : QLORA_DQ_E4M3 (0, what a zero-initialised descriptor holds),
+ *               QLORA_DQ_U8, or QLORA_FMT_INT16 for a weight from qlora_quantize_int
+ *               (then dq_codes may be NULL and dq_scales holds fp32[in*out/16];
+ *               w' = fl32((code - 8) * dq_scales[e/16]) for element e); anything
+ *               else is QLORA_ERR_INVALID_ARG.  Every call taking a descriptor
+ *               accepts all three; an INT16 weight's forward always takes the
+ *               fused GEMM (the small-M path is NF4 only).
  * Dequantised weight ("What QLoRA adds over LoRA"; "LLMs · QLoRA" levels[idx]*scale):
  *   absmax'_b = fl32(e4m3(dq_codes[b]) * dq_scales[b/256])   (E4M3)
  *             = fl32(dq_codes[b] * dq_scales[b/256])         (U8)
@@ -144,8 +151,9 @@ QLORA_API qlora_status qlora_quantize_nf4_ex(const float* W0, int64_t in, int64_
  *   codes   [device] out: uint8[in*out/2].
  *   scales  [device] out: fp32[in*out/16].
  *   All pointers 16-byte aligned (QLORA_ERR_ALIGNMENT otherwise).
- * Requires in*out % 16 == 0.  Bit-exact.  (The adapted-layer calls take NF4
- * weights only; this format is quantised and dequantised here.)
+ * Requires in*out % 16 == 0.  Bit-exact.  The result can be used by every call
+ * that takes a qlora_nf4_weight, with dq_format = QLORA_FMT_INT16 (in*out must
+ * then be a multiple of 64, as for NF4).
  */
 QLORA_API qlora_status qlora_quantize_int(const float* W0, int64_t in, int64_t out, int bits, uint8_t* codes,
                                           float* scales, void* stream);

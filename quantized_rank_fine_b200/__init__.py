@@ -39,8 +39,9 @@ EXPORTS = (
     "qlora_gemm_set_ctas", "qlora_quantize_nf4_ex", "qlora_quantize_int", "qlora_dequantize_int",
 )
 
-# Formats of the absmax codes (NF4Weight.dq_format).
-QLORA_DQ_E4M3, QLORA_DQ_U8 = 0, 1
+# Weight formats (NF4Weight.dq_format): NF4 with E4M3 or linear uint8 absmax
+# codes, or the symmetric INT format of qlora_quantize_int (one scale per 16).
+QLORA_DQ_E4M3, QLORA_DQ_U8, QLORA_FMT_INT16 = 0, 1, 2
 
 # Flag of qlora_linear_opts.flags.
 QLORA_ACCUMULATE_GRADS = 1
@@ -263,6 +264,12 @@ def qlora_quantize_int(W0: torch.Tensor, bits: int, stream=None):
     _check(lib().qlora_quantize_int(_ptr(W0), n_in, n_out, bits, _ptr(codes), _ptr(scales), _stream(stream)),
            "qlora_quantize_int")
     return codes, scales
+
+
+def int_weight(codes: torch.Tensor, scales: torch.Tensor, n_in: int, n_out: int) -> "NF4Weight":
+    """The weight descriptor of a qlora_quantize_int result, for the layer calls
+    (forward, backward, dequantize, merge)."""
+    return NF4Weight(codes, None, scales, n_in, n_out, QLORA_FMT_INT16)
 
 
 def qlora_dequantize_int(codes: torch.Tensor, scales: torch.Tensor, n_in: int, n_out: int,

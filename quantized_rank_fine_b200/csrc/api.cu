@@ -71,8 +71,10 @@ bool linear_shape_ok(int64_t M, int64_t in, int64_t out, int r) {
 }
 
 qlora_status check_weight_shape(const qlora_nf4_weight* w) {
-  if (!w || !w->codes || !w->dq_codes || !w->dq_scales) return QLORA_ERR_INVALID_ARG;
-  if (w->dq_format != QLORA_DQ_E4M3 && w->dq_format != QLORA_DQ_U8) return QLORA_ERR_INVALID_ARG;
+  if (!w || !w->codes || !w->dq_scales) return QLORA_ERR_INVALID_ARG;
+  if (w->dq_format != QLORA_DQ_E4M3 && w->dq_format != QLORA_DQ_U8 && w->dq_format != QLORA_FMT_INT16)
+    return QLORA_ERR_INVALID_ARG;
+  if (w->dq_format != QLORA_FMT_INT16 && !w->dq_codes) return QLORA_ERR_INVALID_ARG;
   if (w->in < 1 || w->out < 1 || w->in > (int64_t(1) << 40) / w->out || (w->in * w->out) % QLORA_BLOCK != 0)
     return QLORA_ERR_SHAPE;
   return QLORA_OK;
@@ -81,13 +83,13 @@ qlora_status check_weight_shape(const qlora_nf4_weight* w) {
 qlora_status check_weight(const qlora_nf4_weight* w) {
   QLORA_TRY(check_weight_shape(w));
   QLORA_TRY(check_ptr(w->codes));
-  QLORA_TRY(check_ptr(w->dq_codes));
+  QLORA_TRY(check_ptr(w->dq_codes, w->dq_format != QLORA_FMT_INT16));
   QLORA_TRY(check_ptr(w->dq_scales));
   return QLORA_OK;
 }
 
 WeightView view(const qlora_nf4_weight* w) {
-  return WeightView{w->codes, w->dq_codes, w->dq_scales, w->in, w->out, w->dq_format == QLORA_DQ_U8};
+  return WeightView{w->codes, w->dq_codes, w->dq_scales, w->in, w->out, w->dq_format};
 }
 
 // Workspace layout (byte offsets), shared by the size query and the calls:
@@ -303,7 +305,7 @@ qlora_status qlora_dequantize(const qlora_nf4_weight* w, void* W_out, int out_dt
   QLORA_TRY(check_weight(w));
   QLORA_TRY(check_ptr(W_out));
   QLORA_CUDA(qlora::launch_dequantize(w->codes, w->dq_codes, w->dq_scales, w->in * w->out, out_dtype == QLORA_BF16,
-                                      W_out, static_cast<cudaStream_t>(stream), w->dq_format == QLORA_DQ_U8));
+                                      W_out, static_cast<cudaStream_t>(stream), w->dq_format));
   return QLORA_OK;
 }
 
@@ -318,8 +320,7 @@ qlora_status qlora_merge(const qlora_nf4_weight* w, const uint16_t* A, const uin
   QLORA_TRY(check_ptr(B));
   QLORA_TRY(check_ptr(W_out));
   QLORA_CUDA(qlora::launch_merge(w->codes, w->dq_codes, w->dq_scales, A, B, r, w->in, w->out,
-                                 out_dtype == QLORA_BF16, W_out, static_cast<cudaStream_t>(stream),
-                                 w->dq_format == QLORA_DQ_U8));
+                                 out_dtype == QLORA_BF16, W_out, static_cast<cudaStream_t>(stream), w->dq_format));
   return QLORA_OK;
 }
 
@@ -368,7 +369,7 @@ static qlora_status fwd_impl(const qlora_nf4_weight* w, const uint16_t* X, int64
   uint32_t* status = reinterpret_cast<uint32_t*>(base);
   uint16_t* V = V_save ? V_save : reinterpret_cast<uint16_t*>(base + L.v_off);
   const WeightView wv = view(w);
-  if (qlora::gemv_supported(M, w->in, w->out)) {
+  if (w->dq_format != QLORA_FMT_INT16 && qlora::gemv_supported(M, w->in, w->out)) {
     QLORA_CUDA(qlora::launch_xa_small(X, A, M, w->in, r, V, s, lo.scale, lo.drop));
     QLORA_CUDA(qlora::launch_gemv(wv, X, V, B, M, r, Y, status, s));
   } else {

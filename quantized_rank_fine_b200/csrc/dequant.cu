@@ -3,7 +3,8 @@
 // dequantize ("LLMs · QLoRA": levels[idx] * scale; "What QLoRA adds over LoRA":
 // absmax quantised to 8 bits, weights dequantised to bf16):
 //   a'_b = fl32(e4m3(dq_code_b) * s_g) (or fl32(dq_code_b * s_g) for linear
-//   uint8 absmax codes),  w' = fl32(level[code] * a'_b),
+//   uint8 absmax codes),  w' = fl32(level[code] * a'_b); for the INT16 format
+//   (qlora_quantize_int) w' = fl32((code - 8) * s) with one scale per 16 weights,
 //   written as fp32 or as bf16(w').  Plain binary32 products, no FMA contraction,
 //   so the result is bit-exact.
 // merge ("QLoRA (low-rank adapters on a quantized model)", "How it works" step 5):
@@ -24,14 +25,16 @@ constexpr int kDqThreads = 256;
 template <bool kBf16>
 __global__ void __launch_bounds__(kDqThreads)
 dequantize_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ dq_codes,
-                  const float* __restrict__ dq_scales, int64_t n16, void* __restrict__ out, bool u8) {
+                  const float* __restrict__ dq_scales, int64_t n16, void* __restrict__ out, int fmt) {
   __shared__ float lv[16];
-  if (threadIdx.x < 16) lv[threadIdx.x] = nf4_level(threadIdx.x);
+  if (threadIdx.x < 16) lv[threadIdx.x] = fmt == kFmtInt16 ? static_cast<float>(static_cast<int>(threadIdx.x) - 8)
+                                                           : nf4_level(threadIdx.x);
   __syncthreads();
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kDqThreads + threadIdx.x;
   if (t >= n16) return;
   const int64_t blk = t >> 2;                       // 4 threads per 64-weight block
-  const float a = absmax_deq(dq_codes[blk], dq_scales[blk / kGroup], u8);
+  const float a = fmt == kFmtInt16 ? dq_scales[t]   // one scale per 16 weights
+                                   : absmax_deq(dq_codes[blk], dq_scales[blk / kGroup], fmt == kFmtU8);
   const uint2 c = __ldcs(reinterpret_cast<const uint2*>(codes) + t);
   float w[16];
 #pragma unroll
@@ -68,12 +71,12 @@ __global__ void __launch_bounds__(256)
 merge_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ dq_codes,
              const float* __restrict__ dq_scales, const __nv_bfloat16* __restrict__ A,
              const __nv_bfloat16* __restrict__ B, int r, int64_t n_in, int64_t n_out,
-             void* __restrict__ out, bool u8) {
+             void* __restrict__ out, int fmt) {
   __shared__ float sA[kMgRows][kMgR + 1];
   __shared__ __align__(16) float sB[kMgR][kMgCols];
   __shared__ float lv[16];
   const int tid = threadIdx.x, tx = tid & 31, ty = tid >> 5;
-  if (tid < 16) lv[tid] = nf4_level(tid);
+  if (tid < 16) lv[tid] = fmt == kFmtInt16 ? static_cast<float>(tid - 8) : nf4_level(tid);
   const int64_t row0 = static_cast<int64_t>(blockIdx.y) * kMgRows;
   const int64_t col0 = static_cast<int64_t>(blockIdx.x) * kMgCols;
 
@@ -120,7 +123,8 @@ merge_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ dq_c
     if (row >= n_in) continue;
     const int64_t e0 = row * n_out + col;                 // multiple of 8
     const int64_t blk = e0 / kBlock;
-    const float a = absmax_deq(dq_codes[blk], dq_scales[blk / kGroup], u8);
+    const float a = fmt == kFmtInt16 ? dq_scales[e0 / 16]
+                                     : absmax_deq(dq_codes[blk], dq_scales[blk / kGroup], fmt == kFmtU8);
     const uint32_t c = *reinterpret_cast<const uint32_t*>(codes + e0 / 2);
     float w[8];
 #pragma unroll
@@ -142,15 +146,15 @@ merge_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ dq_c
 
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* dq_codes,
                               const float* dq_scales, int64_t n, bool bf16, void* out,
-                              cudaStream_t stream, bool u8) {
+                              cudaStream_t stream, int fmt) {
   const int64_t n16 = n / 16;
   if (n16 == 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>((n16 + kDqThreads - 1) / kDqThreads);
   timing_before(QLORA_KERNEL_DEQUANTIZE, stream);
   if (bf16)
-    dequantize_kernel<true><<<grid, kDqThreads, 0, stream>>>(codes, dq_codes, dq_scales, n16, out, u8);
+    dequantize_kernel<true><<<grid, kDqThreads, 0, stream>>>(codes, dq_codes, dq_scales, n16, out, fmt);
   else
-    dequantize_kernel<false><<<grid, kDqThreads, 0, stream>>>(codes, dq_codes, dq_scales, n16, out, u8);
+    dequantize_kernel<false><<<grid, kDqThreads, 0, stream>>>(codes, dq_codes, dq_scales, n16, out, fmt);
   timing_after(QLORA_KERNEL_DEQUANTIZE, stream);
   count_launch();
   return cudaGetLastError();
@@ -158,16 +162,16 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* dq_codes,
 
 cudaError_t launch_merge(const uint8_t* codes, const uint8_t* dq_codes, const float* dq_scales,
                          const uint16_t* A, const uint16_t* B, int r, int64_t n_in,
-                         int64_t n_out, bool bf16, void* out, cudaStream_t stream, bool u8) {
+                         int64_t n_out, bool bf16, void* out, cudaStream_t stream, int fmt) {
   dim3 grid(static_cast<unsigned>((n_out + kMgCols - 1) / kMgCols),
             static_cast<unsigned>((n_in + kMgRows - 1) / kMgRows));
   const auto* a = reinterpret_cast<const __nv_bfloat16*>(A);
   const auto* b = reinterpret_cast<const __nv_bfloat16*>(B);
   timing_before(QLORA_KERNEL_MERGE, stream);
   if (bf16)
-    merge_kernel<true><<<grid, 256, 0, stream>>>(codes, dq_codes, dq_scales, a, b, r, n_in, n_out, out, u8);
+    merge_kernel<true><<<grid, 256, 0, stream>>>(codes, dq_codes, dq_scales, a, b, r, n_in, n_out, out, fmt);
   else
-    merge_kernel<false><<<grid, 256, 0, stream>>>(codes, dq_codes, dq_scales, a, b, r, n_in, n_out, out, u8);
+    merge_kernel<false><<<grid, 256, 0, stream>>>(codes, dq_codes, dq_scales, a, b, r, n_in, n_out, out, fmt);
   timing_after(QLORA_KERNEL_MERGE, stream);
   count_launch();
   return cudaGetLastError();

@@ -146,11 +146,19 @@ struct BlockLut {
   uint32_t lo[4], hi[4];
 };
 
+// Level j of the weight format: the NF4 level, or the integer j - 8 of the
+// symmetric INT format (qlora_quantize_int).
+template <bool kInt>
+__device__ __forceinline__ constexpr float format_level(int j) {
+  return kInt ? static_cast<float>(j - 8) : nf4_level(j);
+}
+
+template <bool kInt>
 __device__ __forceinline__ BlockLut make_lut(float a) {
   uint32_t pr[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
-    pr[i] = pack_bf16x2(mul_rn(nf4_level(2 * i), a), mul_rn(nf4_level(2 * i + 1), a));
+    pr[i] = pack_bf16x2(mul_rn(format_level<kInt>(2 * i), a), mul_rn(format_level<kInt>(2 * i + 1), a));
   BlockLut t;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
@@ -177,7 +185,20 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
-template <bool kDX>
+// Scale data of one K-step for a dequant thread: the absmax code and group
+// scale of its 64-weight NF4 block, or the four fp32 scales of its four
+// 16-weight groups (INT16 format).
+template <bool kInt>
+struct ScaleSlot {
+  uint8_t c = 0;
+  float s = 0.0f;
+};
+template <>
+struct ScaleSlot<true> {
+  float4 s = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+};
+
+template <bool kDX, bool kInt>
 __global__ void __launch_bounds__(kThreads, 1)
 nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_ext_a,
                 const __grid_constant__ CUtensorMap tm_ext_b, const __grid_constant__ CUtensorMap tm_codes,
@@ -384,24 +405,25 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
       const int g0 = g;
       const int kb_first = w.kb0 + ((group - g0) & 1);
       g += w.kb1 - w.kb0;
-      // Absmax code and scale of the group's next K-steps, loaded two of its
-      // steps ahead into one of two register slots; the loop is unrolled by two
-      // so that a slot is consumed and refilled in place (moving a pending
-      // load's register to another would wait for the load one step early).
-      uint8_t dqcA = 0, dqcB = 0;
-      float dqsA = 0.0f, dqsB = 0.0f;
-      if (valid && kb_first < nkb_w) {
-        const int64_t b0 = blk + kb_first * blk_step;
-        dqcA = __ldg(p.dq_codes + b0);
-        dqsA = __ldg(p.dq_scales + b0 / kGroup);
-      }
-      if (valid && kb_first + 2 < nkb_w) {
-        const int64_t b1 = blk + (kb_first + 2) * blk_step;
-        dqcB = __ldg(p.dq_codes + b1);
-        dqsB = __ldg(p.dq_scales + b1 / kGroup);
-      }
-      // one K-step with the absmax in (dqc, dqs); refills them for kb + 4
-      auto step = [&](int kb, uint8_t& dqc, float& dqs) -> bool {
+      // Scale data of the group's next K-steps, loaded two of its steps ahead
+      // into one of two register slots; the loop is unrolled by two so that a
+      // slot is consumed and refilled in place (moving a pending load's
+      // register to another would wait for the load one step early).
+      auto load_slot = [&](int kb, ScaleSlot<kInt>& sl) {
+        if (!valid || kb >= nkb_w) return;
+        const int64_t b = blk + kb * blk_step;
+        if constexpr (kInt) {
+          sl.s = __ldg(reinterpret_cast<const float4*>(p.dq_scales) + b);
+        } else {
+          sl.c = __ldg(p.dq_codes + b);
+          sl.s = __ldg(p.dq_scales + b / kGroup);
+        }
+      };
+      ScaleSlot<kInt> slotA, slotB;
+      load_slot(kb_first, slotA);
+      load_slot(kb_first + 2, slotB);
+      // one K-step with its scale data in `sl`; refills it for kb + 4
+      auto step = [&](int kb, ScaleSlot<kInt>& sl) -> bool {
         const int gg = g0 + (kb - w.kb0);
         const int s = gg % kStages;
         const uint32_t ph = (gg / kStages) & 1;
@@ -417,17 +439,23 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
                        : "=r"(wd[0]), "=r"(wd[1]), "=r"(wd[2]), "=r"(wd[3]) : "r"(csrc + code_off0));
           asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                        : "=r"(wd[4]), "=r"(wd[5]), "=r"(wd[6]), "=r"(wd[7]) : "r"(csrc + code_off1));
-          const BlockLut lut = make_lut(valid ? absmax_deq(dqc, dqs, p.dq_u8 != 0) : 0.0f);
-          if (valid && kb + 4 < nkb_w) {
-            const int64_t nb = blk + (kb + 4) * blk_step;
-            dqc = __ldg(p.dq_codes + nb);
-            dqs = __ldg(p.dq_scales + nb / kGroup);
+          // one table per block (NF4) or per 16-weight group (INT16, words 2q, 2q+1)
+          BlockLut lut[kInt ? 4 : 1];
+          if constexpr (kInt) {
+            lut[0] = make_lut<true>(valid ? sl.s.x : 0.0f);
+            lut[1] = make_lut<true>(valid ? sl.s.y : 0.0f);
+            lut[2] = make_lut<true>(valid ? sl.s.z : 0.0f);
+            lut[3] = make_lut<true>(valid ? sl.s.w : 0.0f);
+          } else {
+            lut[0] = make_lut<false>(valid ? absmax_deq(sl.c, sl.s, p.dq_u8 != 0) : 0.0f);
           }
+          load_slot(kb + 4, sl);
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
+            const BlockLut& L = lut[kInt ? c >> 1 : 0];
             uint32_t o0, o1, o2, o3;
-            lut4(lut, wd[c] & 0xFFFFu, o0, o1);
-            lut4(lut, wd[c] >> 16, o2, o3);
+            lut4(L, wd[c] & 0xFFFFu, o0, o1);
+            lut4(L, wd[c] >> 16, o2, o3);
             st_shared_v4(dst + ((c ^ swz) << 4), o0, o1, o2, o3);
           }
           fence_proxy_async_smem();
@@ -437,7 +465,7 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
         return true;
       };
       for (int kb = kb_first; kb < w.kb1; kb += 4) {
-        if (!step(kb, dqcA, dqsA) || (kb + 2 < w.kb1 && !step(kb + 2, dqcB, dqsB))) {
+        if (!step(kb, slotA) || (kb + 2 < w.kb1 && !step(kb + 2, slotB))) {
           alive = false;
           break;
         }
@@ -578,13 +606,13 @@ struct GemmPlan {
   int pairs, tiles_n, dp_tiles, sk_tiles;
 };
 
-template <bool kDX>
+template <bool kDX, bool kInt>
 cudaError_t prepare_kernel() {
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && attr_set[dev]) return cudaSuccess;
-  const cudaError_t e = cudaFuncSetAttribute(nf4_gemm_kernel<kDX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const cudaError_t e = cudaFuncSetAttribute(nf4_gemm_kernel<kDX, kInt>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(kSmemBytes));
   if (e == cudaSuccess && dev >= 0 && dev < 64) attr_set[dev] = true;
   return e;
@@ -612,8 +640,8 @@ int device_pairs() {
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    if (prepare_kernel<false>() != cudaSuccess ||
-        cudaOccupancyMaxActiveClusters(&n, nf4_gemm_kernel<false>, &cfg) != cudaSuccess || n <= 0) {
+    if (prepare_kernel<false, false>() != cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&n, nf4_gemm_kernel<false, false>, &cfg) != cudaSuccess || n <= 0) {
       cudaGetLastError();
       return 1;
     }
@@ -650,11 +678,11 @@ size_t plan_ws_bytes(const GemmPlan& P) {
   return P.sk_tiles > 0 ? static_cast<size_t>(2 * P.pairs) * kSlotFloats * 4 : 0;
 }
 
-template <bool kDX>
+template <bool kDX, bool kInt>
 cudaError_t launch_gemm(const CUtensorMap& act, const CUtensorMap& ea, const CUtensorMap& eb, const CUtensorMap& cm,
                         GemmArgs a, uint32_t* counters, void* partials, size_t partial_bytes,
                         cudaStream_t stream) {
-  const cudaError_t pe = prepare_kernel<kDX>();
+  const cudaError_t pe = prepare_kernel<kDX, kInt>();
   if (pe != cudaSuccess) return pe;
   GemmPlan P = plan_gemm(a.M, a.N, a.K, a.r, partials != nullptr && counters != nullptr);
   if (P.sk_tiles > 0 && partial_bytes < plan_ws_bytes(P)) P = plan_gemm(a.M, a.N, a.K, a.r, false);
@@ -679,7 +707,7 @@ cudaError_t launch_gemm(const CUtensorMap& act, const CUtensorMap& ea, const CUt
   cfg.numAttrs = 2;
   const int which = kDX ? QLORA_KERNEL_DX_GEMM : QLORA_KERNEL_FWD_GEMM;
   timing_before(which, stream);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, nf4_gemm_kernel<kDX>, act, ea, eb, cm, a);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, nf4_gemm_kernel<kDX, kInt>, act, ea, eb, cm, a);
   timing_after(which, stream);
   count_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
@@ -698,9 +726,10 @@ cudaError_t launch_fwd_gemm(const WeightView& w, const uint16_t* X, const uint16
       !make_map(&eb, B, r, w.out, 64, 64) ||
       !make_map_t(&cm, w.codes, w.in, w.out / 2, 64, 64, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
-  GemmArgs a{w.codes, w.dq_codes, w.dq_scales, w.out, M, w.out, w.in, r, Y, status, w.dq_u8 ? 1 : 0,
+  GemmArgs a{w.codes, w.dq_codes, w.dq_scales, w.out, M, w.out, w.in, r, Y, status, w.fmt == kFmtU8 ? 1 : 0,
              0, 0, 0, nullptr, nullptr};
-  return launch_gemm<false>(act, ea, eb, cm, a, counters, partials, partial_bytes, stream);
+  return w.fmt == kFmtInt16 ? launch_gemm<false, true>(act, ea, eb, cm, a, counters, partials, partial_bytes, stream)
+                            : launch_gemm<false, false>(act, ea, eb, cm, a, counters, partials, partial_bytes, stream);
 }
 
 // dX = dY deq(W)^T + U A^T.
@@ -714,9 +743,10 @@ cudaError_t launch_dx_gemm(const WeightView& w, const uint16_t* dY, const uint16
       !make_map(&eb, A, w.in, r, 64, 128) ||
       !make_map_t(&cm, w.codes, w.in, w.out / 2, 32, 128, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, CU_TENSOR_MAP_SWIZZLE_32B))
     return cudaErrorInvalidValue;
-  GemmArgs a{w.codes, w.dq_codes, w.dq_scales, w.out, M, w.in, w.out, r, dX, status, w.dq_u8 ? 1 : 0,
+  GemmArgs a{w.codes, w.dq_codes, w.dq_scales, w.out, M, w.in, w.out, r, dX, status, w.fmt == kFmtU8 ? 1 : 0,
              0, 0, 0, nullptr, nullptr};
-  return launch_gemm<true>(act, ea, eb, cm, a, counters, partials, partial_bytes, stream);
+  return w.fmt == kFmtInt16 ? launch_gemm<true, true>(act, ea, eb, cm, a, counters, partials, partial_bytes, stream)
+                            : launch_gemm<true, false>(act, ea, eb, cm, a, counters, partials, partial_bytes, stream);
 }
 
 size_t fwd_gemm_split_bytes(int64_t M, int64_t n_in, int64_t n_out, int r) {

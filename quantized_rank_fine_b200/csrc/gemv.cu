@@ -487,7 +487,8 @@ bool gemv_supported(int64_t M, int64_t K, int64_t N) {
 cudaError_t launch_gemv(const WeightView& w, const uint16_t* X, const uint16_t* V, const uint16_t* B, int64_t M,
                         int r, uint16_t* Y, uint32_t* status, cudaStream_t stream) {
   int S, Kc;
-  if (M < 1 || M > kGemvMaxTokens || !gemv_plan(w.in, w.out, cluster_fit(), S, Kc)) return cudaErrorInvalidValue;
+  if (w.fmt == kFmtInt16 || M < 1 || M > kGemvMaxTokens || !gemv_plan(w.in, w.out, cluster_fit(), S, Kc))
+    return cudaErrorInvalidValue;   // NF4 weights only
   auto enc = gemv_encoder();
   if (!enc) return cudaErrorInvalidValue;
   // codes as an (in x out/2) byte matrix; box = one 256-column tile (128 bytes) x 64 rows
@@ -527,7 +528,7 @@ cudaError_t launch_gemv(const WeightView& w, const uint16_t* X, const uint16_t* 
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  GemvArgs a{w.dq_codes, w.dq_scales, w.in, w.out, static_cast<int>(M), r, Y, Kc, status, w.dq_u8 ? 1 : 0};
+  GemvArgs a{w.dq_codes, w.dq_scales, w.in, w.out, static_cast<int>(M), r, Y, Kc, status, w.fmt == kFmtU8 ? 1 : 0};
 
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>((w.out + kTileCols - 1) / kTileCols), static_cast<unsigned>(S));

@@ -33,17 +33,22 @@ struct WeightView {
   const uint8_t* dq_codes;
   const float* dq_scales;
   int64_t in, out;
-  bool dq_u8;         // absmax codes are linear uint8 (else E4M3)
+  int fmt;            // kFmtE4M3, kFmtU8 or kFmtInt16
 };
+
+// Weight formats (the values of qlora_nf4_weight.dq_format): NF4 with E4M3 or
+// linear uint8 absmax codes, or symmetric integers (level = code - 8) with one
+// fp32 scale per 16 weights in dq_scales.
+constexpr int kFmtE4M3 = 0, kFmtU8 = 1, kFmtInt16 = 2;
 
 // dq_u8 / u8: the absmax codes are linear uint8 (s = max / 255) instead of E4M3.
 cudaError_t launch_quantize_nf4(const float* W0, int64_t n, uint8_t* codes, uint8_t* dq_codes,
                                 float* dq_scales, cudaStream_t stream, bool dq_u8 = false);
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* dq_codes, const float* dq_scales,
-                              int64_t n, bool bf16, void* out, cudaStream_t stream, bool u8 = false);
+                              int64_t n, bool bf16, void* out, cudaStream_t stream, int fmt = kFmtE4M3);
 cudaError_t launch_merge(const uint8_t* codes, const uint8_t* dq_codes, const float* dq_scales,
                          const uint16_t* A, const uint16_t* B, int r, int64_t n_in, int64_t n_out,
-                         bool bf16, void* out, cudaStream_t stream, bool u8 = false);
+                         bool bf16, void* out, cudaStream_t stream, int fmt = kFmtE4M3);
 
 // Symmetric uniform INT quantisation, one scale per 16 weights (bits 2..4),
 // and its dense dequantisation.  n is a multiple of 16; W0, codes, scales and

@@ -175,3 +175,12 @@ def test_int_quantiser_rejects_before_launch(L):
     assert L.qlora_quantize_int(None, 16, 16, 4, FAKE, FAKE, None) == 1
     assert L.qlora_dequantize_int(FAKE, FAKE, 16, 16, FAKE, 7, None) == 1      # dtype
     assert L.qlora_dequantize_int(FAKE, FAKE, 0, 16, FAKE, 0, None) == 2
+
+
+def test_int16_weight_descriptor_checks(L):
+    """An INT16 weight needs no absmax codes (NULL passes the argument checks and
+    fails only for lack of a device); an NF4 weight without them is refused."""
+    w_int = q._Weight(0x10000, 0, 0x10000, 256, 256, q.QLORA_FMT_INT16)
+    assert L.qlora_dequantize(ctypes.byref(w_int), FAKE, 0, None) != 1
+    w_nf4 = q._Weight(0x10000, 0, 0x10000, 256, 256, q.QLORA_DQ_E4M3)
+    assert L.qlora_dequantize(ctypes.byref(w_nf4), FAKE, 0, None) == 1

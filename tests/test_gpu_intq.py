@@ -8,8 +8,8 @@ import torch
 
 import quantized_rank_fine_b200 as q
 import synth
-from oracle import intq, nf4
-from tests.helpers import require_gpu
+from oracle import intq, linear, nf4
+from tests.helpers import assert_close, require_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -65,3 +65,45 @@ def test_int_quantize_edge_cases(bits):
     G[11] = np.asarray(rng.normal(0, 1, 16), dtype=np.float32) * np.float32(1e-41)
     G[12] = -np.abs(G[12])
     _check(G.reshape(16, 64), bits)
+
+
+def _int_layer(n_in, n_out, M, r, bits, tag):
+    t = synth.layer_inputs(n_in, n_out, M, r, device="cuda", tag=tag)
+    codes, scales = q.qlora_quantize_int(t["W0"], bits)
+    return t, q.int_weight(codes, scales, n_in, n_out)
+
+
+def _int_oracle_weight(w):
+    return nf4.round_bf16(intq.dequantize_int(w.codes.cpu().numpy(), w.dq_scales.cpu().numpy(), w.n_in, w.n_out))
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_int_weight_dequantize_and_merge(bits):
+    """The INT weight through the layer's descriptor: qlora_dequantize equals
+    qlora_dequantize_int bit for bit, and the merge matches the oracle's."""
+    t, w = _int_layer(320, 192, 1, 24, bits, "intm")
+    a = q.qlora_dequantize(w, torch.float32)
+    b = q.qlora_dequantize_int(w.codes, w.dq_scales, 320, 192, torch.float32)
+    assert torch.equal(a, b)
+    ref = linear.merge(intq.dequantize_int(w.codes.cpu().numpy(), w.dq_scales.cpu().numpy(), 320, 192),
+                       t["A"], t["B"])
+    assert_close(q.qlora_merge(w, t["A"], t["B"], torch.float32), ref, "merge int", rel_fro=1e-6, max_abs=1e-5)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("M,n_in,n_out,r", [(300, 320, 192, 24), (8, 512, 768, 16), (1100, 2048, 1536, 40)])
+def test_linear_int_weight(bits, M, n_in, n_out, r):
+    """Forward and backward of the adapted layer on an INT (group 16) base,
+    through the fused GEMMs (small M included), against the oracle."""
+    t, w = _int_layer(n_in, n_out, M, r, bits, "intlin")
+    ws = q.Workspace()
+    Y, V = q.qlora_linear_fwd(w, t["X"], t["A"], t["B"], ws)
+    dX, dA, dB = q.qlora_linear_bwd(w, t["X"], V, t["dY"], t["A"], t["B"], ws)
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+    Wq = _int_oracle_weight(w)
+    Yr, Vr = linear.forward(t["X"], t["A"], t["B"], Wq)
+    g = linear.backward(t["X"], t["A"], t["B"], Wq, t["dY"])
+    for name, got, ref in (("Y", Y, Yr), ("V", V, Vr), ("dX", dX, g["dX"]), ("dA", dA, g["dA"]),
+                           ("dB", dB, g["dB"])):
+        assert_close(got, ref, name)
