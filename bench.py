@@ -123,11 +123,37 @@ def flops_fwd_gemm(n_in, n_out, M, r):
 GEMM_SOURCES = ("gemm.cu", "sm100.cuh", "common.cuh")
 
 
+def code_tokens(text: str) -> str:
+    """C/C++/CUDA source with its comments removed and whitespace collapsed: what
+    the compiler sees, so that a comment edit does not count as a kernel change."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":                          # string or character literal, kept whole
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def src_hash(*names):
+    """Hash of the code (comments and whitespace aside) of the GEMM's sources."""
     h = hashlib.sha1()
     for n in names:
-        with open(os.path.join(ROOT, "quantized_rank_fine_b200", "csrc", n), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "quantized_rank_fine_b200", "csrc", n), encoding="utf-8") as f:
+            h.update(code_tokens(f.read()).encode())
     return h.hexdigest()[:12]
 
 

@@ -1,4 +1,6 @@
-// Fused NF4-dequant GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM).
+// Fused dequant GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM), for
+// NF4 weights (one absmax per 64 weights, E4M3 or linear uint8 codes) and for the
+// symmetric INT weights of qlora_quantize_int (one fp32 scale per 16 weights).
 //
 //   forward  Y  = [X | V] . [deq(Wq) ; B]      (M x out, K = in + r)
 //   dX       dX = [dY | U] . [deq(Wq)^T ; A^T] (M x in,  K = out + r)
@@ -24,15 +26,18 @@
 //              the CTA's half of the B / A^T tile instead.
 //   warp 1     TMEM allocation (both CTAs, pair form); in the even CTA of the
 //              pair the single thread that issues the MMAs for both.
-//   warps 2-9  dequant producers (one thread per 32 weights per K-step): codes
-//              from shared memory -> per-block 16-entry bf16 table ->
-//              byte-permute lookup -> 16-byte stores in the UMMA canonical
-//              layout; then the epilogue (TMEM -> registers -> global).
+//   warps 2-9  dequant producers, two groups of 4 warps taking alternate
+//              K-steps (one thread per 64 weights per step): codes from shared
+//              memory -> 16-entry bf16 table per 64-weight block (NF4) or per
+//              16-weight group (INT) -> byte-permute lookup -> 16-byte stores in
+//              the UMMA canonical layout; then the epilogue (TMEM -> registers
+//              -> global), all 8 warps.
 // Barriers per stage: `loaded` (this CTA's TMA bytes), `ready` (in the even CTA:
-// the 16 dequant warps of both CTAs, each after its CTA's stage has landed and
-// its weight half is written) and `free` (the pair MMAs' commit, multicast to
-// both CTAs); per work item `tmem_full` (the last MMA's commit, multicast) and
-// `tmem_empty` (in the even CTA: both CTAs' epilogue warps have read their TMEM).
+// the 4 dequant warps of each CTA that took the stage, each after its CTA's
+// stage has landed and its weight half is written) and `free` (the pair MMAs'
+// commit, multicast to both CTAs); per work item `tmem_full` (the last MMA's
+// commit, multicast) and `tmem_empty` (in the even CTA: the 8 epilogue warps of
+// each CTA have read their TMEM).
 // The weight tile is written MN-major for the forward (N contiguous in W) and
 // K-major for dX (K contiguous in W), so the dequant never transposes.
 //

@@ -110,3 +110,14 @@ def test_workload_defaults_and_bytes(monkeypatch):
 def test_workload_config_names_the_workload(name):
     c = bench.workload_config(name)
     assert c["workload"] == name and c["M"] == bench.WORKLOADS[name]["M"]
+
+
+def test_code_hash_ignores_comments_not_code():
+    """The traffic record's source hash: comments and whitespace do not change
+    it, code (including string literals that contain comment markers) does."""
+    a = 'int f(int x) {  // add one\n  return x + 1; /* done */ }\nconst char* s = "a // b";\n'
+    b = 'int f(int x) { return x + 1; }\n/* header */ const char* s = "a // b";'
+    c = 'int f(int x) { return x + 2; }\nconst char* s = "a // b";'
+    assert bench.code_tokens(a) == bench.code_tokens(b)
+    assert bench.code_tokens(a) != bench.code_tokens(c)
+    assert '"a // b"' in bench.code_tokens(a)
