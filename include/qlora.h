@@ -176,8 +176,9 @@ QLORA_API qlora_status qlora_dequantize(const qlora_nf4_weight* w, void* W_out, 
  * Forward of the adapted layer ("How it works" steps 2-3; "LoRA & QLoRA"
  * Mathematical Formulation h = W0 x + B(A x)):
  *   V = bf16(X A)  (fp32 accumulation),   Y = bf16(X bf16(w') + V B)  (fp32 accumulation).
- * For M <= 16 a dequant-GEMV computes the base term as sum_k bf16(x_k a'_k) bf16(l_k)
- * (the block absmax folded into the activation; the same sum in exact arithmetic).
+ * For M <= 16 and an NF4 weight a dequant-GEMV computes the base term as
+ * sum_k bf16(x_k a'_k) bf16(l_k) (the block absmax folded into the activation; the
+ * same sum in exact arithmetic); otherwise the fused dequant GEMM runs.
  *   w      [host] descriptor of [device] tensors.
  *   X      [device] bf16 (M, in).
  *   A      [device] bf16 (in, r).          B [device] bf16 (r, out).
