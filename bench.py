@@ -73,7 +73,7 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-rows", action="store_true", help="skip the per-kernel row measurements")
     p.add_argument("--rows", default=None,
-                   help="comma-separated subset of the rows: quantize, dequantize, merge, gemv, train_step "
+                   help="comma-separated subset of the rows: quantize, dequantize, merge, gemv, train_step, int16 "
                         "(default: all of them; none for the stack, whose quantize pass is always measured)")
     p.add_argument("--rows-only", action="store_true",
                    help="measure only the rows (no headline step); prints {'rows': ...}")
@@ -345,7 +345,7 @@ def run_step(layers, ws):
         q.qlora_linear_bwd(w, t["X"], o["V"], t["dY"], t["A"], t["B"], ws, dX=o["dX"], dA=o["dA"], dB=o["dB"])
 
 
-ROW_NAMES = ("quantize", "dequantize", "merge", "gemv", "train_step")
+ROW_NAMES = ("quantize", "dequantize", "merge", "gemv", "train_step", "int16")
 
 
 def time_rows(wl, pk, which="all"):
@@ -364,6 +364,11 @@ def time_rows(wl, pk, which="all"):
         rows["gemv"] = time_gemv(pk)
     if "train_step" in want:
         rows["train_step_adam"] = time_train_step(wl)
+    if "int16" in want:
+        try:
+            rows["int16"] = time_int16_rows(wl, pk)
+        except Exception as e:   # a secondary row never takes the headline down
+            rows["int16"] = {"error": f"{type(e).__name__}: {e}"}
     return rows
 
 
@@ -409,6 +414,55 @@ def time_weight_rows(wl, pk, want):
     del W0s, ws_
     torch.cuda.synchronize()
     return rows
+
+
+def time_int16_rows(wl, pk):
+    """The INT base of the pages' simulation (qlora_quantize_int: symmetric
+    integers, one fp32 scale per 16 weights), 4 bits, on the workload's first
+    weight shape: quantize and dequantize (GB/s against HBM), and the fused
+    forward GEMM on that weight at the workload's M (TFLOP/s), next to the NF4
+    weight's forward GEMM measured the same way."""
+    import torch
+    import quantized_rank_fine_b200 as q
+    import synth
+    n_in, n_out = wl["shapes"][0]
+    M, r = wl["M"], wl["r"]
+    n = n_in * n_out
+    reps = max(3, math.ceil(3 * L2_BYTES / (4 * n)))
+    W0s = [synth.normal(f"intW{i}", (n_in, n_out), 0.02, device="cuda") for i in range(reps)]
+    ints = [q.qlora_quantize_int(W, 4) for W in W0s]
+    torch.cuda.synchronize()
+    hbm = pk["hbm_gbs"]
+    out = {"bits": 4, "shape": [n_in, n_out]}
+    t = graph_timed(lambda i: q.qlora_quantize_int(W0s[i % reps], 4, out=ints[i % reps]), q.KERNEL_QUANTIZE, 30)
+    b = n * (4 + 0.5 + 0.25)
+    out["quantize"] = {"ms": t, "gbs": b / t / 1e6, "frac_hbm": b / t / 1e6 / hbm, "bytes_per_weight": 4.75}
+    dq = [torch.empty((n_in, n_out), dtype=torch.bfloat16, device="cuda") for _ in range(reps)]
+    t = graph_timed(lambda i: q.qlora_dequantize_int(*ints[i % reps], n_in, n_out, torch.bfloat16, out=dq[i % reps]),
+                    q.KERNEL_DEQUANTIZE, 30)
+    b = n * (0.5 + 0.25 + 2)
+    out["dequantize_bf16"] = {"ms": t, "gbs": b / t / 1e6, "frac_hbm": b / t / 1e6 / hbm}
+    del dq
+    # forward GEMM: INT16 weights against NF4 weights of the same W0, inputs rotated
+    wts_int = [q.int_weight(c, s, n_in, n_out) for c, s in ints]
+    wts_nf4 = [q.qlora_quantize_nf4(W) for W in W0s]
+    del W0s
+    X = [synth.normal(f"intX{i}", (M, n_in), 1.0, torch.bfloat16, "cuda") for i in range(2)]
+    A = synth.normal("intA", (n_in, r), 1 / math.sqrt(n_in), torch.bfloat16, "cuda")
+    B = synth.normal("intB", (r, n_out), 0.01, torch.bfloat16, "cuda")
+    Y = torch.empty((M, n_out), dtype=torch.bfloat16, device="cuda")
+    V = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+    ws = q.Workspace()
+    fl = flops_fwd_gemm(n_in, n_out, M, r)
+    for name, wts in (("fwd_gemm_int16", wts_int), ("fwd_gemm_nf4", wts_nf4)):
+        t = graph_timed(lambda i: q.qlora_linear_fwd(wts[i % reps], X[i % 2], A, B, ws, Y=Y, V=V),
+                        q.KERNEL_FWD_GEMM, 20)
+        out[name] = {"ms": t, "tflops": fl / t / 1e9}
+    if ws.status() != 0:
+        raise RuntimeError("a kernel wait timed out in the INT rows")
+    del ints, wts_int, wts_nf4
+    torch.cuda.synchronize()
+    return out
 
 
 def time_train_step(wl):

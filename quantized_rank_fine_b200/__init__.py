@@ -253,14 +253,17 @@ def qlora_quantize_nf4(W0: torch.Tensor, stream=None, out: NF4Weight | None = No
     return out
 
 
-def qlora_quantize_int(W0: torch.Tensor, bits: int, stream=None):
+def qlora_quantize_int(W0: torch.Tensor, bits: int, stream=None, out=None):
     """Symmetric uniform INT quantisation with one scale per 16 weights (bits 2,
     3 or 4; 2 is ternary): W0 fp32 (in, out) on the GPU -> (codes uint8
-    [in*out/2], scales fp32 [in*out/16])."""
+    [in*out/2], scales fp32 [in*out/16]), allocated unless `out` gives them."""
     n_in, n_out = W0.shape
     n = n_in * n_out
-    codes = torch.empty(n // 2, dtype=torch.uint8, device=W0.device)
-    scales = torch.empty(n // 16, dtype=torch.float32, device=W0.device)
+    if out is None:
+        codes = torch.empty(n // 2, dtype=torch.uint8, device=W0.device)
+        scales = torch.empty(n // 16, dtype=torch.float32, device=W0.device)
+    else:
+        codes, scales = out
     _check(lib().qlora_quantize_int(_ptr(W0), n_in, n_out, bits, _ptr(codes), _ptr(scales), _stream(stream)),
            "qlora_quantize_int")
     return codes, scales
