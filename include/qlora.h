@@ -3,9 +3,10 @@
  *
  * A linear layer whose frozen weight W0 (in x out, stored row-major as (in, out))
  * is kept as 4-bit NormalFloat (NF4) codes with one absmax per 64 consecutive
- * weights, the absmax values themselves double-quantised to 8-bit E4M3 codes with
- * one fp32 scale per 256 absmax values, plus trainable low-rank adapters
- * A (in x r) and B (r x out):
+ * weights, the absmax values themselves double-quantised to 8-bit codes (E4M3, or
+ * linear uint8) with one fp32 scale per 256 absmax values -- or, the pages' second
+ * base quantiser, as symmetric 2-4 bit integers with one fp32 scale per 16
+ * weights -- plus trainable low-rank adapters A (in x r) and B (r x out):
  *
  *     forward   Y  = X deq(Wq) + (X A) B
  *     backward  dX = dY deq(Wq)^T + (dY B^T) A^T
@@ -57,7 +58,8 @@ typedef enum qlora_status {
   QLORA_ERR_INVALID_ARG = 1,        /* NULL where a tensor is required, bad enum, host pointer */
   QLORA_ERR_SHAPE = 2,              /* a size constraint of the call is violated */
   QLORA_ERR_ALIGNMENT = 3,          /* a tensor pointer is not 16-byte aligned */
-  QLORA_ERR_WORKSPACE = 4,          /* workspace NULL or smaller than qlora_workspace_bytes() */
+  QLORA_ERR_WORKSPACE = 4,          /* workspace NULL or smaller than the call's minimum (see
+                                       qlora_workspace_bytes) */
   QLORA_ERR_UNSUPPORTED_DEVICE = 5, /* current device is not sm_100 */
   QLORA_ERR_CUDA = 6,               /* a CUDA runtime call or kernel launch failed */
   QLORA_ERR_TIMEOUT = 7             /* a bounded wait inside a kernel gave up (qlora_ws_status) */
