@@ -7,7 +7,10 @@ A step is one forward + backward pass of the adapted linear layer(s) of the
 workload over one batch of M tokens: dequantisation of the frozen NF4 weight
 inside the GEMMs, V = X A, Y, U = dY B^T, dX, dA, dB.  Quantisation and merge
 are one-time operations of the method ("How it works" steps 1 and 5) and are
-timed separately under "rows", with the small-M forward.
+timed separately under "rows", with the small-M forward, the training step with
+the fused Adam update, and the INT (one scale per 16 weights) base quantiser.
+The Llama-7B stack workload (--workload llama7b_stack_m2048_r16) runs all 224
+linears of the model per step and times the quantise pass over all of them.
 
 Timing: W untimed warm-up steps, then exactly K steps between a barrier +
 synchronize on both sides, CUDA events on the launching stream, max over ranks.
