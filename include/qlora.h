@@ -394,11 +394,11 @@ typedef enum qlora_kernel {
  * Returns QLORA_ERR_INVALID_ARG for an unknown kernel or NULL arrays with n > 0. */
 QLORA_API qlora_status qlora_time_kernel(int which, void* const* starts, void* const* stops, int n);
 
-/* Most CTAs the fused dequant GEMMs use (0, the default: one per SM; larger
- * values are capped at the SM count).  A testing and tuning knob: a small count
- * makes small layers exercise the shared-K-step schedule.  Process-wide; takes
- * effect for calls (and workspace sizes) after it.  QLORA_ERR_INVALID_ARG if
- * ctas < 0. */
+/* Most CTAs the fused dequant GEMMs use (0, the default: every SM, as CTA pairs
+ * on the two SMs of a TPC; a count c gives max(1, c / 2) pairs, capped at the
+ * pairs the device holds at once).  A testing and tuning knob: a small count makes
+ * small layers exercise the shared-K-step schedule.  Process-wide; takes effect
+ * for calls (and workspace sizes) after it.  QLORA_ERR_INVALID_ARG if ctas < 0. */
 QLORA_API qlora_status qlora_gemm_set_ctas(int ctas);
 
 /* Number of kernel launches libqlora has issued in this process. */
