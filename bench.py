@@ -62,9 +62,13 @@ WORKLOADS = {
     "llama7b_stack_m2048_r16": dict(shapes=[(a, b) for _, a, b, _ in LLAMA7B_LAYER] * 32, M=2048, r=16,
                                     layer=LLAMA7B_LAYER, layers=32, steps=20, warmup=3),
 }
-DEFAULT_WORKLOAD = "attn4096_m4096_r16"
+DEFAULT_WORKLOAD = "llama7b_stack_m2048_r16"
 L2_BYTES = 126 * 2 ** 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# B200 datasheet figures, reported beside the measured ones: dense bf16 tensor
+# throughput and HBM3e bandwidth
+SPEC_BF16_TFLOPS = 2250.0
+SPEC_HBM_GBS = 8000.0
 
 
 def parse():
@@ -88,7 +92,7 @@ def parse():
     if a.warmup is None:
         a.warmup = wl.get("warmup", 10)
     if a.rows is None:
-        a.rows = "" if "layer" in wl else "all"
+        a.rows = "all"
     return a
 
 
@@ -163,31 +167,89 @@ def src_hash(*names):
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 100 ms while running."""
+    """SM clock and clock-event reasons of one GPU, sampled every ~2 ms by a thread
+    polling NVML (read-only queries) while the timed region runs; `nvidia-smi`
+    every 100 ms when NVML cannot be loaded.  A median needs samples inside the
+    region, which for a short region only an in-process poll provides."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_S = 0.002
 
-    def __init__(self, index):
-        self.index = index
+    def __init__(self, index, uuid=None, pci_bus_id=None):
+        self.index = index          # nvidia-smi index (fallback path)
+        self.uuid = uuid            # CUDA device UUID, for NVML
+        self.pci_bus_id = pci_bus_id
         self.proc = None
+        self.thread = None
+        self.samples = []           # (sm_mhz, reasons bitmask)
+        self.sm_max = None
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        for how, key in ((pynvml.nvmlDeviceGetHandleByUUID, self.uuid),
+                         (pynvml.nvmlDeviceGetHandleByPciBusId, self.pci_bus_id)):
+            if key:
+                try:
+                    return pynvml, how(key)
+                except Exception:
+                    pass
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(int(self.index))
 
     def start(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            nv, h = self._nvml_handle()
+            self.sm_max = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        except Exception:
+            nv = None
+        if nv is None:
+            self.source = "nvidia-smi"
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                     "--format=csv,noheader,nounits", "-lms", "100"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except OSError:
+                self.proc = None
+            return
+        self.source = "nvml"
+        self._stop = threading.Event()
+
+        def poll():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                         int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))))
+                except Exception:
+                    pass
+                time.sleep(self.PERIOD_S)
+
+        self.thread = threading.Thread(target=poll, daemon=True)
+        self.thread.start()
 
     def stop(self):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        if self.thread is not None:
+            import pynvml as nv
+            self._stop.set()
+            self.thread.join(timeout=5)
+            bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+            sm = [s for s, _ in self.samples]
+            reasons = sorted(n for n in names if any(r & bits[n] for _, r in self.samples))
+            return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.sm_max,
+                    "reasons": reasons, "samples": len(sm), "source": "nvml, 2 ms poll"}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
         self.proc.terminate()
         out, _ = self.proc.communicate(timeout=10)
         sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in out.strip().splitlines():
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
@@ -201,7 +263,23 @@ class ClockSampler:
                 if v.lower() == "active":
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi, 100 ms"}
+
+
+def clock_sampler(local):
+    """The sampler for this rank's GPU (NVML by the CUDA device's UUID)."""
+    import torch
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    smi_id = vis.split(",")[local] if vis and len(vis.split(",")) > local else str(local)
+    uuid = pci = None
+    try:
+        p = torch.cuda.get_device_properties(local)
+        u = str(p.uuid)
+        uuid = u if u.startswith("GPU-") else "GPU-" + u
+        pci = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except Exception:
+        pass
+    return ClockSampler(smi_id, uuid, pci)
 
 
 # ------------------------------------------------------------------ distributed plumbing
@@ -267,6 +345,30 @@ def build_sets(wl, nsets, seed_base):
     return sets
 
 
+def stack_weight(li, name, n_in, n_out, seed, device="cuda"):
+    """W0 of projection `name` of layer li of the stack (fp32 0.02 N(0, 1))."""
+    import torch
+    import synth
+    return synth.normal(f"stack{li}.{name}:W0", (n_in, n_out), 0.02, torch.float32, device, seed)
+
+
+def stack_linear(li, name, n_in, n_out, x_key, M, r, seed, acts, device="cuda"):
+    """W0 and the inputs of one linear of the stack, drawn on the device: its own
+    adapters A, B and output gradient dY, and the input X of its key, drawn once
+    per layer and key (`acts` holds the layer's drawn inputs)."""
+    import torch
+    import synth
+    p = f"stack{li}.{name}:"
+    W0 = stack_weight(li, name, n_in, n_out, seed, device)
+    if x_key not in acts:
+        acts[x_key] = synth.normal(f"stack{li}.{x_key}:X", (M, n_in), 1.0, torch.bfloat16, device, seed)
+    t = {"X": acts[x_key],
+         "A": synth.normal(p + "A", (n_in, r), 1.0 / math.sqrt(n_in), torch.bfloat16, device, seed),
+         "B": synth.normal(p + "B", (r, n_out), 0.01, torch.bfloat16, device, seed),
+         "dY": synth.normal(p + "dY", (M, n_out), 1.0, torch.bfloat16, device, seed)}
+    return W0, t
+
+
 def build_stack(wl, seed, pk):
     """The Llama-7B linear stack as one input set, and its quantize pass.
 
@@ -283,14 +385,8 @@ def build_stack(wl, seed, pk):
     for li in range(wl["layers"]):
         acts = {}
         for name, n_in, n_out, x_key in wl["layer"]:
-            p = f"stack{li}.{name}:"
-            W0s.append(synth.normal(p + "W0", (n_in, n_out), 0.02, torch.float32, "cuda", seed))
-            if x_key not in acts:
-                acts[x_key] = synth.normal(f"stack{li}.{x_key}:X", (M, n_in), 1.0, torch.bfloat16, "cuda", seed)
-            t = {"X": acts[x_key],
-                 "A": synth.normal(p + "A", (n_in, r), 1.0 / math.sqrt(n_in), torch.bfloat16, "cuda", seed),
-                 "B": synth.normal(p + "B", (r, n_out), 0.01, torch.bfloat16, "cuda", seed),
-                 "dY": synth.normal(p + "dY", (M, n_out), 1.0, torch.bfloat16, "cuda", seed)}
+            W0, t = stack_linear(li, name, n_in, n_out, x_key, M, r, seed, acts)
+            W0s.append(W0)
             out = {
                 "Y": torch.empty((M, n_out), dtype=torch.bfloat16, device="cuda"),
                 "V": torch.empty((M, r), dtype=torch.bfloat16, device="cuda"),
@@ -315,8 +411,7 @@ def build_stack(wl, seed, pk):
     torch.cuda.empty_cache()
     ms = min(times)
     b = sum(a * o * (4 + 0.5 + 1 / 64) + 4 * math.ceil(a * o / 64 / 256) for a, o in wl["shapes"])
-    row = {"ms": ms, "weights": n, "launches": len(weights), "gbs": b / ms / 1e6,
-           "frac_hbm": b / ms / 1e6 / pk["hbm_gbs"],
+    row = {"ms": ms, "weights": n, "launches": len(weights), **hbm_fracs(b, ms, pk),
            "note": "all 224 W0 of the stack quantised back to back (fp32 in, NF4 codes + absmax codes + "
                    "scales out); the better of two timed passes"}
     layers = [(w, t, o) for w, (t, o) in zip(weights, plan)]
@@ -348,7 +443,7 @@ def run_step(layers, ws):
         q.qlora_linear_bwd(w, t["X"], o["V"], t["dY"], t["A"], t["B"], ws, dX=o["dX"], dA=o["dA"], dB=o["dB"])
 
 
-ROW_NAMES = ("quantize", "dequantize", "merge", "gemv", "train_step", "int16")
+ROW_NAMES = ("quantize", "dequantize", "merge", "gemv", "train_step", "int16", "mlp_m8192")
 
 
 def time_rows(wl, pk, which="all"):
@@ -366,7 +461,11 @@ def time_rows(wl, pk, which="all"):
     if "gemv" in want:
         rows["gemv"] = time_gemv(pk)
     if "train_step" in want:
-        rows["train_step_adam"] = time_train_step(wl)
+        # the stack's layers are too many for graph-captured sets: its training-step
+        # row runs the attention projection (4096 x 4096, r = 16, M = 4096)
+        rows["train_step_adam"] = time_train_step(WORKLOADS["attn4096_m4096_r16"] if "layer" in wl else wl)
+    if "mlp_m8192" in want:
+        rows["mlp_m8192"] = time_mlp_row(pk)
     if "int16" in want:
         try:
             rows["int16"] = time_int16_rows(wl, pk)
@@ -375,13 +474,26 @@ def time_rows(wl, pk, which="all"):
     return rows
 
 
+def weight_row_shape(wl):
+    """Weight shape of the quantize / dequantize / merge rows: the workload's first
+    shape, or 4096 x 11008 (the largest matrix of a layer) for the stack."""
+    return (4096, 11008) if "layer" in wl else wl["shapes"][0]
+
+
+def hbm_fracs(b, ms, pk):
+    """GB/s of b algorithmic bytes in ms, as fractions of the measured and the
+    datasheet HBM bandwidth."""
+    gbs = b / ms / 1e6
+    return {"gbs": gbs, "frac_hbm": gbs / pk["hbm_gbs"], "frac_hbm_spec": gbs / SPEC_HBM_GBS}
+
+
 def time_weight_rows(wl, pk, want):
-    """Quantize, dequantize and merge on the workload's first weight shape."""
+    """Quantize, dequantize and merge on one weight (weight_row_shape)."""
     import torch
     import quantized_rank_fine_b200 as q
     import synth
     rows = {}
-    n_in, n_out = wl["shapes"][0]
+    n_in, n_out = weight_row_shape(wl)
     n = n_in * n_out
     reps = max(3, math.ceil(3 * L2_BYTES / (4 * n)))
     W0s = [synth.normal(f"rowsW{i}", (n_in, n_out), 0.02, device="cuda") for i in range(reps)]
@@ -391,18 +503,17 @@ def time_weight_rows(wl, pk, want):
     def timed(fn, which, iters):
         return graph_timed(fn, which, iters)
 
-    hbm = pk["hbm_gbs"]
     iters = 30
     if "quantize" in want:
         t = timed(lambda i: q.qlora_quantize_nf4(W0s[i % reps], out=ws_[i % reps]), q.KERNEL_QUANTIZE, iters)
         b = n * (4 + 0.5 + 1 / 64) + 4 * math.ceil(n / 64 / 256)
-        rows["quantize"] = {"ms": t, "gbs": b / t / 1e6, "frac_hbm": b / t / 1e6 / hbm, "bytes_per_weight": 4.516}
+        rows["quantize"] = {"shape": [n_in, n_out], "ms": t, **hbm_fracs(b, t, pk), "bytes_per_weight": 4.516}
     if "dequantize" in want:
         outs = [torch.empty((n_in, n_out), dtype=torch.bfloat16, device="cuda") for _ in range(reps)]
         t = timed(lambda i: q.qlora_dequantize(ws_[i % reps], torch.bfloat16, out=outs[i % reps]),
                   q.KERNEL_DEQUANTIZE, iters)
         b = n * (0.5 + 1 / 64 + 2) + 4 * math.ceil(n / 64 / 256)
-        rows["dequantize_bf16"] = {"ms": t, "gbs": b / t / 1e6, "frac_hbm": b / t / 1e6 / hbm}
+        rows["dequantize_bf16"] = {"shape": [n_in, n_out], "ms": t, **hbm_fracs(b, t, pk)}
         del outs
     if "merge" in want:
         r = wl["r"]
@@ -412,7 +523,7 @@ def time_weight_rows(wl, pk, want):
         t = timed(lambda i: q.qlora_merge(ws_[i % reps], A, B, torch.float32, out=outs32[i % reps]),
                   q.KERNEL_MERGE, iters)
         b = n * (0.5 + 1 / 64 + 4) + 2 * r * (n_in + n_out)
-        rows["merge_f32"] = {"ms": t, "gbs": b / t / 1e6, "frac_hbm": b / t / 1e6 / hbm}
+        rows["merge_f32"] = {"shape": [n_in, n_out], "r": r, "ms": t, **hbm_fracs(b, t, pk)}
         del outs32
     del W0s, ws_
     torch.cuda.synchronize()
@@ -435,16 +546,15 @@ def time_int16_rows(wl, pk):
     W0s = [synth.normal(f"intW{i}", (n_in, n_out), 0.02, device="cuda") for i in range(reps)]
     ints = [q.qlora_quantize_int(W, 4) for W in W0s]
     torch.cuda.synchronize()
-    hbm = pk["hbm_gbs"]
     out = {"bits": 4, "shape": [n_in, n_out]}
     t = graph_timed(lambda i: q.qlora_quantize_int(W0s[i % reps], 4, out=ints[i % reps]), q.KERNEL_QUANTIZE, 30)
     b = n * (4 + 0.5 + 0.25)
-    out["quantize"] = {"ms": t, "gbs": b / t / 1e6, "frac_hbm": b / t / 1e6 / hbm, "bytes_per_weight": 4.75}
+    out["quantize"] = {"ms": t, **hbm_fracs(b, t, pk), "bytes_per_weight": 4.75}
     dq = [torch.empty((n_in, n_out), dtype=torch.bfloat16, device="cuda") for _ in range(reps)]
     t = graph_timed(lambda i: q.qlora_dequantize_int(*ints[i % reps], n_in, n_out, torch.bfloat16, out=dq[i % reps]),
                     q.KERNEL_DEQUANTIZE, 30)
     b = n * (0.5 + 0.25 + 2)
-    out["dequantize_bf16"] = {"ms": t, "gbs": b / t / 1e6, "frac_hbm": b / t / 1e6 / hbm}
+    out["dequantize_bf16"] = {"ms": t, **hbm_fracs(b, t, pk)}
     del dq
     # forward GEMM: INT16 weights against NF4 weights of the same W0, inputs rotated
     wts_int = [q.int_weight(c, s, n_in, n_out) for c, s in ints]
@@ -464,6 +574,88 @@ def time_int16_rows(wl, pk):
     if ws.status() != 0:
         raise RuntimeError("a kernel wait timed out in the INT rows")
     del ints, wts_int, wts_nf4
+    torch.cuda.synchronize()
+    return out
+
+
+def tensor_fracs(flops, ms, pk):
+    """TFLOP/s of `flops` in ms, as fractions of the measured burst and sustained
+    bf16 peaks and of the datasheet's dense bf16 peak."""
+    tf = flops / ms / 1e9
+    return {"tflops": tf, "frac_burst": tf / pk["bf16_tflops"], "frac_sustained": tf / pk["bf16_tflops_sustained"],
+            "frac_spec": tf / SPEC_BF16_TFLOPS}
+
+
+def time_mlp_row(pk):
+    """The Llama-7B MLP projections (4096 -> 11008 and 11008 -> 4096, r = 64) at
+    M = 8192 tokens, the size the fused GEMM's throughput target is stated at.
+    Three CUDA graphs of back-to-back fwd + bwd steps over input sets larger than
+    L2: one with the forward GEMM's launches bracketed by events, one with the dX
+    GEMM's, one plain for the whole step.  Each GEMM is reported per projection
+    shape (mean over its launches) and both together."""
+    import torch
+    import quantized_rank_fine_b200 as q
+    wl = WORKLOADS["mlp4096x11008_m8192_r64"]
+    M, r = wl["M"], wl["r"]
+    shapes = wl["shapes"]
+    nsets = max(2, math.ceil(3 * L2_BYTES / set_bytes(wl)))
+    sets = build_sets(wl, nsets, seed_base=11)
+    ws = q.Workspace()
+    steps = 2 * nsets
+    for i in range(3):
+        run_step(sets[i % nsets], ws)
+    torch.cuda.synchronize()
+
+    def graph(timer):
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side, capture_error_mode="relaxed"):
+                for i in range(steps):
+                    run_step(sets[i % nsets], ws)
+        torch.cuda.current_stream().wait_stream(side)
+        if timer is not None:
+            timer.disarm()
+        return g
+
+    out = {"M": M, "r": r}
+    for name, kind in (("fwd_gemm", q.KERNEL_FWD_GEMM), ("dx_gemm", q.KERNEL_DX_GEMM)):
+        tm = q.KernelTimer(kind, steps * len(shapes))
+        g = graph(tm)
+        g.replay()
+        torch.cuda.synchronize()
+        ts = tm.times_ms()
+        del g
+        per = {}
+        for j, (a, b) in enumerate(shapes):
+            t = statistics.mean(ts[j::len(shapes)])
+            fl = flops_fwd_gemm(a, b, M, r) if name == "fwd_gemm" else flops_fwd_gemm(b, a, M, r)
+            per[f"{a}x{b}"] = {"ms": t, **tensor_fracs(fl, t, pk)}
+        t_all = sum(per[f"{a}x{b}"]["ms"] for a, b in shapes)
+        fl_all = sum(flops_fwd_gemm(a, b, M, r) for a, b in shapes)   # the dX GEMMs have the same total
+        per["both"] = {"ms": t_all, **tensor_fracs(fl_all, t_all, pk)}
+        out[name] = per
+    g = graph(None)
+    g.replay()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) / steps)
+    del g
+    t = statistics.median(times)
+    out["fwd_bwd"] = {"ms_per_step": t, "tokens_per_s": M / (t * 1e-3),
+                      **tensor_fracs(sum(flops_fwd_bwd(a, b, M, r) for a, b in shapes), t, pk)}
+    out["note"] = ("fractions of the measured bf16 burst / sustained peaks (MEASURED_PEAKS.json) and of the "
+                   f"{SPEC_BF16_TFLOPS:.0f} TFLOP/s datasheet peak; fwd + bwd = both projections")
+    if ws.status() != 0:
+        raise RuntimeError("a kernel wait timed out in the MLP row")
+    del sets
     torch.cuda.synchronize()
     return out
 
@@ -600,8 +792,7 @@ def time_gemv(pk):
                 raise RuntimeError("a kernel wait timed out in the small-M forward")
             b = n_in * n_out * (0.5 + 1 / 64) + 4 * math.ceil(n_in * n_out / 16384) + 2 * r * (n_in + n_out) \
                 + 2 * M * (n_in + n_out) + 2 * M * r
-            out[f"{n_in}x{n_out}_m{M}"] = {"us_per_forward": t * 1e3, "gbs": b / t / 1e6,
-                                           "frac_hbm": b / t / 1e6 / pk["hbm_gbs"], "launches": 2}
+            out[f"{n_in}x{n_out}_m{M}"] = {"us_per_forward": t * 1e3, **hbm_fracs(b, t, pk), "launches": 2}
         del wts
         torch.cuda.synchronize()
     return out
@@ -666,9 +857,7 @@ def arm_ours(args, world, rank, local):
             g.replay()
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
-    smi_id = vis.split(",")[local] if vis and len(vis.split(",")) > local else str(local)
-    clocks = ClockSampler(smi_id)
+    clocks = clock_sampler(local)
     barrier(world)
     torch.cuda.synchronize()
     clocks.start()
@@ -728,13 +917,14 @@ def arm_ours(args, world, rank, local):
         "tflops": step_flops * args.steps * world / (ms / 1e3) / 1e12,
         "roofline": {"kernel": "nf4_gemm_kernel<fwd> (fused dequant GEMM, tcgen05)", "bound": "tensor",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "frac_spec": achieved / SPEC_BF16_TFLOPS,
                      "peak_source": f"{pk_src} {'burst' if timed_s < 2.0 else 'sustained'} bf16",
                      "flops_per_launch": gemm_flops[0] if nl == 1 else
                      {f"{a}x{b}": flops_fwd_gemm(a, b, M, r) for a, b in wl["shapes"]},
                      "mean_launch_ms": statistics.mean(gemm_ms), "traffic": traffic},
         "gpu_launches": launches,
         "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"],
-                   "samples": clk["samples"]},
+                   "samples": clk["samples"], "source": clk.get("source")},
     }
 
     # end to end through the public API with host buffers
@@ -746,57 +936,111 @@ def arm_ours(args, world, rank, local):
         # per GPU (each rank quantises its own replica of the stack); slowest rank
         slow = max_over_ranks(quantize_pass["ms"], world) / quantize_pass["ms"]
         quantize_pass.update(ms=quantize_pass["ms"] * slow, gbs=quantize_pass["gbs"] / slow,
-                             frac_hbm=quantize_pass["frac_hbm"] / slow)
+                             frac_hbm=quantize_pass["frac_hbm"] / slow,
+                             frac_hbm_spec=quantize_pass["frac_hbm_spec"] / slow)
         line.setdefault("rows", {})["quantize_pass"] = quantize_pass
     if world == 1 and rank == 0 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(args.workload, budget_s=20.0)
     return line
 
 
+def e2e_slots(sets):
+    """Two device slots of per-step data for the end-to-end leg: slot s holds the
+    inputs X and dY and the gradient outputs dA and dB that step i (with
+    i % 2 = s) uses; weights, adapters and the other outputs are shared.  With
+    one input set (the stack) the second slot gets its own X, dY, dA and dB."""
+    import torch
+    if len(sets) >= 2:
+        return [sets[0], sets[1]]
+    fresh = {}
+
+    def twin(d):
+        if d.data_ptr() not in fresh:
+            fresh[d.data_ptr()] = torch.empty_like(d)
+        return fresh[d.data_ptr()]
+
+    second = []
+    for w, t, o in sets[0]:
+        t2 = dict(t, X=twin(t["X"]), dY=twin(t["dY"]))
+        o2 = dict(o, dA=torch.empty_like(o["dA"]), dB=torch.empty_like(o["dB"]))
+        second.append((w, t2, o2))
+    return [sets[0], second]
+
+
 def e2e(args, sets, ws, wl, world):
-    """Same metric, each step copying X and dY from pinned host memory and the
-    adapter gradients dA, dB back to pinned host memory, on one stream."""
+    """Same metric through the public API from host memory: every step copies its
+    inputs (each distinct X and dY) from pinned host memory to the device and the
+    adapter gradients dA, dB back to pinned host memory.  The copies run on their
+    own streams (host-to-device, device-to-host) and overlap the layer calls of
+    the neighbouring steps; two device slots alternate, and events order each
+    slot's copy-in, layer calls and copy-out."""
     import torch
     M = wl["M"]
-    nsets = len(sets)
-    host = []          # per set: ([(device input, pinned host copy)], [(device gradient, pinned host buffer)])
-    for layers in sets:
-        ins, seen = [], set()
-        for w, t, o in layers:
-            for d in (t["X"], t["dY"]):
-                if d.data_ptr() not in seen:      # the stack's shared activations are copied once
-                    seen.add(d.data_ptr())
-                    ins.append((d, torch.empty(d.shape, dtype=d.dtype, pin_memory=True).copy_(d)))
-        outs = [(o[k], torch.empty(o[k].shape, dtype=torch.float32).pin_memory())
-                for w, t, o in layers for k in ("dA", "dB")]
-        host.append((ins, outs))
-    h2d = sum(d.numel() * d.element_size() for d, _ in host[0][0])
-    d2h = sum(d.numel() * d.element_size() for d, _ in host[0][1])
+    slots = e2e_slots(sets)
+    ins, outs = [], []          # per slot: [(device input, pinned host source)], [(device grad, pinned host dest)]
+    host_src = {}               # one pinned host copy per distinct input of slot 0, the source of both slots
+    for s, layers in enumerate(slots):
+        seen, si = set(), []
+        for j, (w, t, o) in enumerate(layers):
+            for k in ("X", "dY"):
+                d = t[k]
+                if d.data_ptr() in seen:          # the stack's shared activations are copied once
+                    continue
+                seen.add(d.data_ptr())
+                key = (j, k)
+                if key not in host_src:
+                    host_src[key] = torch.empty(d.shape, dtype=d.dtype, pin_memory=True).copy_(slots[0][j][1][k])
+                si.append((d, host_src[key]))
+        ins.append(si)
+        outs.append([(o[k], torch.empty(o[k].shape, dtype=torch.float32).pin_memory())
+                     for w, t, o in layers for k in ("dA", "dB")])
+    h2d = sum(d.numel() * d.element_size() for d, _ in ins[0])
+    d2h = sum(d.numel() * d.element_size() for d, _ in outs[0])
     steps = 10 if "layer" in wl else max(10, args.steps // 4)
+    comp = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
 
-    def step(i):
-        ins, outs = host[i % nsets]
-        for d, h in ins:
-            d.copy_(h, non_blocking=True)
-        run_step(sets[i % nsets], ws)
-        for d, h in outs:
-            h.copy_(d, non_blocking=True)
+    def run(n, e_start=None):
+        ev = lambda: torch.cuda.Event()
+        h_done, c_done, d_done = [], [], []
+        if e_start is not None:
+            up.wait_event(e_start)
+        for i in range(n):
+            s = i % 2
+            if i >= 2:
+                up.wait_event(c_done[i - 2])      # slot s's inputs were read by step i - 2
+            with torch.cuda.stream(up):
+                for d, h in ins[s]:
+                    d.copy_(h, non_blocking=True)
+            h_done.append(ev())
+            h_done[i].record(up)
+            comp.wait_event(h_done[i])
+            if i >= 2:
+                comp.wait_event(d_done[i - 2])    # slot s's gradients were copied out after step i - 2
+            run_step(slots[s], ws)
+            c_done.append(ev())
+            c_done[i].record(comp)
+            down.wait_event(c_done[i])
+            with torch.cuda.stream(down):
+                for d, h in outs[s]:
+                    h.copy_(d, non_blocking=True)
+            d_done.append(ev())
+            d_done[i].record(down)
+        comp.wait_event(d_done[-1])
 
-    for i in range(3):
-        step(i)
+    run(3)
     torch.cuda.synchronize()
-    s = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
-    e0.record(s)
-    for i in range(steps):
-        step(i)
-    e1.record(s)
+    e0.record(comp)
+    run(steps, e0)
+    e1.record(comp)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world)
     return {"value": M * steps * world / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": steps}
+            "d2h_bytes_per_step": d2h, "steps": steps,
+            "overlap": "copy-in, layer calls and copy-out of neighbouring steps on three streams, two device slots"}
 
 
 # ------------------------------------------------------------------ the oracle (CPU baseline / reference arm)

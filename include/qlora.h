@@ -205,18 +205,31 @@ QLORA_API qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16_
  * minus the workspace and uses a fixed array of QLORA_STATIC_WS_BYTES inside the
  * library's own device memory instead (held by every GPU that loads the library
  * until the process exits); it allocates nothing.
- *   Returns QLORA_ERR_WORKSPACE, launching nothing, when the sizes need more than
- *   QLORA_STATIC_WS_BYTES (qlora_workspace_bytes(QLORA_OP_FWD, ...) larger).
- *   The first call on each device looks up the array's device address; make that
- *   first call before any stream capture.  Every call shares the one array and
- *   zeroes its bookkeeping words first; calls whose work overlaps on the GPU
- *   (other streams, other threads) race and must not be issued.  A wait that
- *   times out inside a kernel is not reported by this entry point.
+ *   Returns QLORA_ERR_WORKSPACE, launching nothing, when the smallest forward
+ *   workspace of these sizes (everything but the fused GEMM's split partial
+ *   tiles: the 1280-byte prefix and V, M x r bf16 rounded up to 256 bytes) is
+ *   larger than QLORA_STATIC_WS_BYTES.  The GEMM then always keeps its tiles
+ *   whole, which can cost up to one wave of tiles against qlora_linear_fwd with
+ *   a full-size workspace.
+ *   The array's device address is looked up on every call made outside a stream
+ *   capture and cached per device for calls inside one: a captured call needs an
+ *   earlier uncaptured call on the same device (else QLORA_ERR_INVALID_ARG).
+ *   Every call shares the one array and zeroes its split counters first; calls
+ *   whose work overlaps on the GPU (other streams, other threads) race and must
+ *   not be issued.  A bounded wait that gives up inside a kernel sets the array's
+ *   status word, which stays set until qlora_static_ws_status reads it.
  */
 #define QLORA_STATIC_WS_BYTES (16u << 20)
 QLORA_API qlora_status qlora_linear_fwd_static_ws(const qlora_nf4_weight* w, const uint16_t* X, int64_t M,
                                                   const uint16_t* A, const uint16_t* B, int r, uint16_t* Y,
                                                   uint16_t* V_save, void* stream);
+
+/* qlora_ws_status for the array of qlora_linear_fwd_static_ws on the current
+ * device: synchronise `stream`, then QLORA_ERR_TIMEOUT (and clear the word) if a
+ * bounded wait in a kernel of a static-workspace call gave up since the last
+ * check, else QLORA_OK.  Inside a stream capture it needs an earlier uncaptured
+ * call on the device, like the forward. */
+QLORA_API qlora_status qlora_static_ws_status(void* stream);
 
 /*
  * Backward of the adapted layer ("How it works" step 4; "The code, line by line":
@@ -339,6 +352,37 @@ QLORA_API qlora_status qlora_linear_bwd_adam(const qlora_nf4_weight* w, const ui
 QLORA_API qlora_status qlora_merge(const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B, int r,
                          void* W_out, int out_dtype, void* stream);
 
+/*
+ * LoftQ-style initialisation of the adapters ("QLoRA (low-rank adapters on a
+ * quantized model)", "Going further": start A and B from an SVD of W0 - Q(W0)
+ * instead of B = 0).  Three steps: qlora_loftq_residual below, a rank-r (or
+ * thin) singular value decomposition R = U diag(S) Vh by any library, and
+ * qlora_loftq_split, which splits it symmetrically into A B.
+ *
+ * qlora_loftq_residual: R[k][n] = fl32(W0[k][n] - w'), w' the dequantised weight
+ * of `w` (any format), for a weight quantised from this W0.  Bit-exact.
+ *   W0  [device] fp32 (in, out).   w [host] descriptor of [device] tensors.
+ *   R   [device] out: fp32 (in, out).
+ * Requires in*out % 64 == 0.
+ */
+QLORA_API qlora_status qlora_loftq_residual(const float* W0, const qlora_nf4_weight* w, float* R, void* stream);
+
+/*
+ * qlora_loftq_split: the adapters from the leading r singular triplets,
+ *   s_j = fl32(sqrt(S[j])) (IEEE square root),
+ *   A[i][j] = bf16(fl32(U[i][j] s_j)),  B[j][o] = bf16(fl32(s_j Vh[j][o]))
+ * for i < in, j < r, o < out, so that A B = U_r diag(S_r) Vh_r up to the
+ * roundings (A^T A = B B^T = diag(S_r) in exact arithmetic).  Bit-exact.
+ *   U   [device] fp32, row i at U + i ldu (ldu >= r); columns 0..r-1 are read.
+ *   S   [device] fp32[r] or longer, >= 0 (singular values).
+ *   Vh  [device] fp32, row j at Vh + j ldv (ldv >= out); rows 0..r-1 are read.
+ *   A   [device] out: bf16 (in, r).   B [device] out: bf16 (r, out).
+ *   All pointers 16-byte aligned; QLORA_ERR_SHAPE for r < 1 or short strides.
+ */
+QLORA_API qlora_status qlora_loftq_split(const float* U, int64_t ldu, const float* S, const float* Vh,
+                                         int64_t ldv, int64_t in, int64_t out, int r, uint16_t* A,
+                                         uint16_t* B, void* stream);
+
 /* ---------------------------------------------------------------- helpers */
 
 /* Bytes of workspace qlora_linear_fwd / qlora_linear_bwd use at these sizes on
@@ -366,6 +410,14 @@ QLORA_API qlora_status qlora_ws_init(void* ws, size_t ws_bytes, void* stream);
  * kernel that used this workspace gave up since the last check (and clear it),
  * else QLORA_OK.  Device work of a call that timed out left its outputs undefined. */
 QLORA_API qlora_status qlora_ws_status(void* ws, void* stream);
+
+/* The quantisers take no workspace: a bounded wait inside qlora_quantize_nf4(_ex)
+ * that gives up (its bulk copies of W0 did not land within the limit) sets a
+ * status word of the library on the device instead.  This call synchronises
+ * `stream`, then returns QLORA_ERR_TIMEOUT (and clears the word) if that
+ * happened on the current device since the last check, else QLORA_OK.  The codes
+ * of a quantisation that timed out are undefined. */
+QLORA_API qlora_status qlora_quantize_status(void* stream);
 
 /* The 16 NF4 levels, ascending (code = index) [host]. */
 QLORA_API void qlora_nf4_codebook(float out[16]);
@@ -400,6 +452,21 @@ QLORA_API qlora_status qlora_time_kernel(int which, void* const* starts, void* c
  * small layers exercise the shared-K-step schedule.  Process-wide; takes effect
  * for calls (and workspace sizes) after it.  QLORA_ERR_INVALID_ARG if ctas < 0. */
 QLORA_API qlora_status qlora_gemm_set_ctas(int ctas);
+
+/* Test of the failure path (no counterpart on the pages): one kernel runs a
+ * single bounded wait that nothing can complete -- kind 0 on an mbarrier of its
+ * own with no arrivals, kind 1 on the last of the workspace's GEMM counters
+ * (zero, awaited to reach 1, advanced by nothing) -- with a limit of limit_us
+ * microseconds (1 .. 1,000,000), after which it raises a bit in the workspace's
+ * status word and returns, as every wait in the library's kernels does at its
+ * 2 s limit.  qlora_ws_status then reports QLORA_ERR_TIMEOUT.  The kernel has no
+ * copies or tensor-core work in flight, so the context stays usable.
+ *   ws  [device] a workspace of at least 1280 bytes (the prefix), initialised by
+ *       qlora_ws_init; the counter is left at zero.
+ * QLORA_ERR_INVALID_ARG for another kind or limit, QLORA_ERR_WORKSPACE for a
+ * missing or short workspace. */
+QLORA_API qlora_status qlora_selftest_wait_timeout(void* ws, size_t ws_bytes, int kind, uint32_t limit_us,
+                                                   void* stream);
 
 /* Number of kernel launches libqlora has issued in this process. */
 QLORA_API uint64_t qlora_launch_count(void);

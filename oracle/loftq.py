@@ -14,6 +14,9 @@ TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).
   of W0 - Q(W0) instead of zero.  Reading: the rank-r truncated SVD of the
   residual R = W0 - deq(Q(W0)) = U S V^T, split symmetrically, A = U_r S_r^1/2,
   B = S_r^1/2 V_r^T (the page fixes the product A B, not the split).
+  ``split_adapters`` restates that split in the precision of stored adapters
+  (fp32 square roots and products, bf16 results), the step a GPU kernel takes
+  from a given decomposition.
 """
 
 from __future__ import annotations
@@ -44,6 +47,23 @@ def loftq_init(W0, r: int):
     U, S, Vt = np.linalg.svd(R, full_matrices=False)
     root = np.sqrt(S[:r])
     return U[:, :r] * root[None, :], root[:, None] * Vt[:r, :]
+
+
+def split_adapters(U, S, Vt, r: int):
+    """The symmetric split in the library's precision: each of the r largest
+    singular values is square-rooted in fp32 (s = fl32(sqrt(S_j)), the correctly
+    rounded square root), A[i][j] = bf16(fl32(U[i][j] s_j)) and
+    B[j][o] = bf16(fl32(s_j Vt[j][o])) (adapters are stored in bf16).  U, S, Vt
+    are fp32 values; returns (A, B) as float32 arrays holding bf16 values.  Every
+    fl32 is one exact float64 operation rounded once (exact products of two fp32
+    values; for the square root the float64 double rounding is innocuous)."""
+    U = np.asarray(U, np.float32).astype(np.float64)
+    S = np.asarray(S, np.float32).astype(np.float64)
+    Vt = np.asarray(Vt, np.float32).astype(np.float64)
+    s = nf4.fl32(np.sqrt(S[:r])).astype(np.float64)
+    A = nf4.round_bf16(nf4.fl32(U[:, :r] * s[None, :]))
+    B = nf4.round_bf16(nf4.fl32(s[:, None] * Vt[:r, :]))
+    return A, B
 
 
 def requantize_merged(Wq, A, B):

@@ -13,6 +13,7 @@ from __future__ import annotations
 
 import ctypes
 import os
+from contextlib import nullcontext as _nullcontext
 from dataclasses import dataclass
 
 import torch
@@ -37,6 +38,8 @@ EXPORTS = (
     "qlora_adapter_params", "qlora_status_string", "qlora_time_kernel", "qlora_launch_count",
     "qlora_linear_fwd_static_ws", "qlora_linear_bwd_adam", "qlora_linear_fwd_ex", "qlora_linear_bwd_ex",
     "qlora_gemm_set_ctas", "qlora_quantize_nf4_ex", "qlora_quantize_int", "qlora_dequantize_int",
+    "qlora_static_ws_status", "qlora_quantize_status", "qlora_selftest_wait_timeout",
+    "qlora_loftq_residual", "qlora_loftq_split",
 )
 
 # Weight formats (NF4Weight.dq_format): NF4 with E4M3 or linear uint8 absmax
@@ -107,6 +110,11 @@ def lib() -> ctypes.CDLL:
             "qlora_quantize_int": (i32, [vp, i64, i64, i32, vp, vp, vp]),
             "qlora_dequantize_int": (i32, [vp, vp, i64, i64, vp, i32, vp]),
             "qlora_linear_fwd_static_ws": (i32, [wp, vp, i64, vp, vp, i32, vp, vp, vp]),
+            "qlora_static_ws_status": (i32, [vp]),
+            "qlora_loftq_residual": (i32, [vp, wp, vp, vp]),
+            "qlora_loftq_split": (i32, [vp, i64, vp, vp, i64, i64, i64, i32, vp, vp, vp]),
+            "qlora_quantize_status": (i32, [vp]),
+            "qlora_selftest_wait_timeout": (i32, [vp, sz, i32, ctypes.c_uint32, vp]),
             "qlora_linear_bwd_adam": (i32, [wp, vp, vp, vp, i64, vp, vp, i32, vp, ctypes.POINTER(_AdamState),
                                             ctypes.POINTER(_AdamHparams), ctypes.POINTER(_LinearOpts), vp, sz,
                                             vp]),
@@ -251,6 +259,21 @@ def qlora_quantize_nf4(W0: torch.Tensor, stream=None, out: NF4Weight | None = No
                                            _ptr(out.dq_scales), out.dq_format, _stream(stream)),
                "qlora_quantize_nf4_ex")
     return out
+
+
+def qlora_quantize_status(stream=None) -> int:
+    """Synchronise the stream and read (then clear) the quantisers' device status
+    word: 0, or QLORA_ERR_TIMEOUT if a bounded wait in a quantisation gave up."""
+    return lib().qlora_quantize_status(_stream(stream))
+
+
+def qlora_selftest_wait_timeout(workspace: "Workspace", kind: int, limit_us: int, stream=None) -> None:
+    """Run one bounded wait that can only run out (kind 0: an mbarrier, kind 1: a
+    workspace counter), with a limit of limit_us; afterwards workspace.status()
+    reports QLORA_ERR_TIMEOUT."""
+    buf = workspace.get(1280, stream)
+    _check(lib().qlora_selftest_wait_timeout(_ptr(buf), buf.numel(), kind, limit_us, _stream(stream)),
+           "qlora_selftest_wait_timeout")
 
 
 def qlora_quantize_int(W0: torch.Tensor, bits: int, stream=None, out=None):
@@ -423,16 +446,39 @@ def requantize_merged(w: NF4Weight, A: torch.Tensor, B: torch.Tensor, stream=Non
     return qlora_quantize_nf4(qlora_merge(w, A, B, torch.float32, stream=stream), stream=stream)
 
 
+def qlora_loftq_residual(W0: torch.Tensor, w: NF4Weight, stream=None, out=None) -> torch.Tensor:
+    """R = fl32(W0 - deq(Wq)), fp32 (in, out), for a weight quantised from W0."""
+    if out is None:
+        out = torch.empty((w.n_in, w.n_out), dtype=torch.float32, device=W0.device)
+    ws = w.c_struct()
+    _check(lib().qlora_loftq_residual(_ptr(W0), ctypes.byref(ws), _ptr(out), _stream(stream)),
+           "qlora_loftq_residual")
+    return out
+
+
+def qlora_loftq_split(U: torch.Tensor, S: torch.Tensor, Vh: torch.Tensor, r: int, stream=None):
+    """The adapters (A bf16 (in, r), B bf16 (r, out)) from the leading r singular
+    triplets of U diag(S) Vh (fp32 device tensors, U (in, k), Vh (k, out))."""
+    n_in, n_out = U.shape[0], Vh.shape[1]
+    A = torch.empty((n_in, r), dtype=torch.bfloat16, device=U.device)
+    B = torch.empty((r, n_out), dtype=torch.bfloat16, device=U.device)
+    _check(lib().qlora_loftq_split(_ptr(U), U.shape[1], _ptr(S), _ptr(Vh), Vh.shape[1], n_in, n_out, r, _ptr(A),
+                                   _ptr(B), _stream(stream)), "qlora_loftq_split")
+    return A, B
+
+
 def loftq_init(W0: torch.Tensor, r: int, stream=None):
     """Quantise W0 and start the adapters from the rank-r truncated SVD of the
     quantisation residual R = W0 - deq(Q(W0)) = U S V^T, split as A = U_r S_r^1/2,
     B = S_r^1/2 V_r^T (bf16), instead of B = 0.  Returns (NF4Weight, A, B).
-    The SVD is torch.linalg.svd on the device (a library decomposition, run once
-    at initialisation)."""
-    w = qlora_quantize_nf4(W0, stream=stream)
-    R = W0.float() - qlora_dequantize(w, torch.float32, stream=stream)
-    U, S, Vh = torch.linalg.svd(R, full_matrices=False)
-    root = S[:r].sqrt()
-    A = (U[:, :r] * root[None, :]).to(torch.bfloat16).contiguous()
-    B = (root[:, None] * Vh[:r, :]).to(torch.bfloat16).contiguous()
+    The quantiser, the residual and the split are library kernels; the SVD is
+    torch.linalg.svd on the device (a library decomposition, run once at
+    initialisation)."""
+    if stream is not None and not isinstance(stream, torch.cuda.Stream):
+        raise TypeError("loftq_init takes a torch.cuda.Stream (the SVD runs on it too)")
+    with torch.cuda.stream(stream) if stream is not None else _nullcontext():
+        w = qlora_quantize_nf4(W0)
+        R = qlora_loftq_residual(W0, w)
+        U, S, Vh = torch.linalg.svd(R, full_matrices=False)
+        A, B = qlora_loftq_split(U.contiguous(), S.contiguous(), Vh.contiguous(), r)
     return w, A, B

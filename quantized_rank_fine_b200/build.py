@@ -22,7 +22,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libqlora.so")
 SOURCES = ["api.cu", "quantize.cu", "dequant.cu", "skinny.cu", "gemm.cu", "gemv.cu", "xa_small.cu", "noalloc.cu",
-           "intq.cu"]
+           "intq.cu", "selftest.cu"]
 HEADERS = ["common.cuh", "kernels.h", "sm100.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

@@ -248,6 +248,28 @@ qlora_status qlora_ws_status(void* ws, void* stream) {
   return QLORA_OK;
 }
 
+qlora_status qlora_quantize_status(void* stream) {
+  QLORA_TRY(check_device());
+  uint32_t flags = 0;
+  QLORA_CUDA(qlora::quantize_status_take(static_cast<cudaStream_t>(stream), &flags));
+  return flags != 0 ? QLORA_ERR_TIMEOUT : QLORA_OK;
+}
+
+qlora_status qlora_selftest_wait_timeout(void* ws, size_t ws_bytes, int kind, uint32_t limit_us, void* stream) {
+  if (kind != 0 && kind != 1) return QLORA_ERR_INVALID_ARG;
+  if (limit_us < 1 || limit_us > 1000000u) return QLORA_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < qlora::kWsFixedBytes) return QLORA_ERR_WORKSPACE;
+  QLORA_TRY(check_device());
+  QLORA_TRY(check_ptr(ws));
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  // the last of the GEMM's counters: zero, and advanced by nothing here
+  const uint32_t* counter =
+      reinterpret_cast<const uint32_t*>(base + qlora::kWsStatusBytes) + (qlora::kMaxGemmCtas - 1);
+  QLORA_CUDA(qlora::launch_selftest_wait(reinterpret_cast<uint32_t*>(base), counter, kind,
+                                         static_cast<uint64_t>(limit_us) * 1000u, static_cast<cudaStream_t>(stream)));
+  return QLORA_OK;
+}
+
 qlora_status qlora_quantize_nf4(const float* W0, int64_t in, int64_t out, uint8_t* codes, uint8_t* dq_codes,
                                 float* dq_scales, void* stream) {
   return qlora_quantize_nf4_ex(W0, in, out, codes, dq_codes, dq_scales, QLORA_DQ_E4M3, stream);
@@ -306,6 +328,32 @@ qlora_status qlora_dequantize(const qlora_nf4_weight* w, void* W_out, int out_dt
   QLORA_TRY(check_ptr(W_out));
   QLORA_CUDA(qlora::launch_dequantize(w->codes, w->dq_codes, w->dq_scales, w->in * w->out, out_dtype == QLORA_BF16,
                                       W_out, static_cast<cudaStream_t>(stream), w->dq_format));
+  return QLORA_OK;
+}
+
+qlora_status qlora_loftq_residual(const float* W0, const qlora_nf4_weight* w, float* R, void* stream) {
+  if (!W0 || !R) return QLORA_ERR_INVALID_ARG;
+  QLORA_TRY(check_weight_shape(w));
+  QLORA_TRY(check_device());
+  QLORA_TRY(check_weight(w));
+  QLORA_TRY(check_ptr(W0));
+  QLORA_TRY(check_ptr(R));
+  QLORA_CUDA(qlora::launch_dequantize(w->codes, w->dq_codes, w->dq_scales, w->in * w->out, false, R,
+                                      static_cast<cudaStream_t>(stream), w->dq_format, W0));
+  return QLORA_OK;
+}
+
+qlora_status qlora_loftq_split(const float* U, int64_t ldu, const float* S, const float* Vh, int64_t ldv, int64_t in,
+                               int64_t out, int r, uint16_t* A, uint16_t* B, void* stream) {
+  if (!U || !S || !Vh || !A || !B) return QLORA_ERR_INVALID_ARG;
+  if (in < 1 || out < 1 || r < 1 || ldu < r || ldv < out || in > (int64_t(1) << 40) / (ldu > r ? ldu : r) ||
+      static_cast<int64_t>(r) > (int64_t(1) << 40) / (ldv > out ? ldv : out) || (in + out) * r >= (int64_t(1) << 40))
+    return QLORA_ERR_SHAPE;
+  QLORA_TRY(check_device());
+  for (const void* p : {static_cast<const void*>(U), static_cast<const void*>(S), static_cast<const void*>(Vh),
+                        static_cast<const void*>(A), static_cast<const void*>(B)})
+    QLORA_TRY(check_ptr(p));
+  QLORA_CUDA(qlora::launch_loftq_split(U, ldu, S, Vh, ldv, in, out, r, A, B, static_cast<cudaStream_t>(stream)));
   return QLORA_OK;
 }
 

@@ -85,6 +85,7 @@ enum : uint32_t {
   kFlagTimeoutProducer = 1u << 0,
   kFlagTimeoutMma = 1u << 1,
   kFlagTimeoutEpilogue = 1u << 2,
+  kFlagTimeoutSelftest = 1u << 3,
 };
 
 __device__ __forceinline__ void raise_flag(uint32_t* status, uint32_t bit) {

@@ -9,6 +9,11 @@
 //   so the result is bit-exact.
 // merge ("QLoRA (low-rank adapters on a quantized model)", "How it works" step 5):
 //   W = w' + A B with fp32 accumulation over the rank.
+// LoftQ-style initialisation (same page, "Going further": start A and B from an
+// SVD of W0 - Q(W0)): the quantisation residual R = fl32(W0 - w'), one mode of
+// the dequantisation kernel; and the symmetric split of a caller's rank-r SVD
+// U diag(S) Vh into the adapters, A = bf16(fl32(U fl32(sqrt S))) and
+// B = bf16(fl32(fl32(sqrt S) Vh)).
 //
 // Both are HBM-bound streaming kernels: each thread handles 16 consecutive
 // weights (8 code bytes, one 64-byte fp32 or 32-byte bf16 output run), so every
@@ -22,10 +27,15 @@ namespace {
 
 constexpr int kDqThreads = 256;
 
-template <bool kBf16>
+// Output of the dequantisation kernel: fp32 w', bf16(w'), or the residual
+// fl32(W0 - w') of the weight W0 the codes were quantised from.
+enum DqMode { kDqF32 = 0, kDqBf16 = 1, kDqResidual = 2 };
+
+template <int kMode>
 __global__ void __launch_bounds__(kDqThreads)
 dequantize_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ dq_codes,
-                  const float* __restrict__ dq_scales, int64_t n16, void* __restrict__ out, int fmt) {
+                  const float* __restrict__ dq_scales, int64_t n16, void* __restrict__ out, int fmt,
+                  const float* __restrict__ W0) {
   __shared__ float lv[16];
   if (threadIdx.x < 16) lv[threadIdx.x] = fmt == kFmtInt16 ? static_cast<float>(static_cast<int>(threadIdx.x) - 8)
                                                            : nf4_level(threadIdx.x);
@@ -44,7 +54,16 @@ dequantize_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__
     w[2 * i] = mul_rn(lv[byte & 0xF], a);
     w[2 * i + 1] = mul_rn(lv[byte >> 4], a);
   }
-  if constexpr (kBf16) {
+  if constexpr (kMode == kDqResidual) {
+    const float4* w0 = reinterpret_cast<const float4*>(W0) + 4 * t;
+    float4* o = reinterpret_cast<float4*>(out) + 4 * t;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 v = __ldcs(w0 + i);
+      __stcs(o + i, make_float4(__fsub_rn(v.x, w[4 * i]), __fsub_rn(v.y, w[4 * i + 1]),
+                                __fsub_rn(v.z, w[4 * i + 2]), __fsub_rn(v.w, w[4 * i + 3])));
+    }
+  } else if constexpr (kMode == kDqBf16) {
     uint4* o = reinterpret_cast<uint4*>(out) + 2 * t;
     uint4 p0, p1;
     p0.x = pack_bf16x2(w[0], w[1]);   p0.y = pack_bf16x2(w[2], w[3]);
@@ -142,19 +161,50 @@ merge_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ dq_c
   }
 }
 
+// A (in x r) and B (r x out) from the leading r singular triplets: thread e
+// writes element e of A (e < in r) or element e - in r of B.
+__global__ void __launch_bounds__(256)
+loftq_split_kernel(const float* __restrict__ U, int64_t ldu, const float* __restrict__ S,
+                   const float* __restrict__ Vh, int64_t ldv, int64_t n_in, int64_t n_out, int r,
+                   uint16_t* __restrict__ A, uint16_t* __restrict__ B) {
+  const int64_t e = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  const int64_t na = n_in * r;
+  if (e < na) {
+    const int64_t i = e / r;
+    const int j = static_cast<int>(e - i * r);
+    A[e] = static_cast<uint16_t>(pack_bf16x2(mul_rn(U[i * ldu + j], __fsqrt_rn(S[j])), 0.0f));
+  } else if (e < na + static_cast<int64_t>(r) * n_out) {
+    const int64_t f = e - na;
+    const int j = static_cast<int>(f / n_out);
+    const int64_t o = f - static_cast<int64_t>(j) * n_out;
+    B[f] = static_cast<uint16_t>(pack_bf16x2(mul_rn(__fsqrt_rn(S[j]), Vh[j * ldv + o]), 0.0f));
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_loftq_split(const float* U, int64_t ldu, const float* S, const float* Vh, int64_t ldv,
+                               int64_t n_in, int64_t n_out, int r, uint16_t* A, uint16_t* B, cudaStream_t stream) {
+  const int64_t n = (n_in + n_out) * r;
+  loftq_split_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(U, ldu, S, Vh, ldv, n_in, n_out,
+                                                                                 r, A, B);
+  count_launch();
+  return cudaGetLastError();
+}
 
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* dq_codes,
                               const float* dq_scales, int64_t n, bool bf16, void* out,
-                              cudaStream_t stream, int fmt) {
+                              cudaStream_t stream, int fmt, const float* W0) {
   const int64_t n16 = n / 16;
   if (n16 == 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>((n16 + kDqThreads - 1) / kDqThreads);
   timing_before(QLORA_KERNEL_DEQUANTIZE, stream);
-  if (bf16)
-    dequantize_kernel<true><<<grid, kDqThreads, 0, stream>>>(codes, dq_codes, dq_scales, n16, out, fmt);
+  if (W0)
+    dequantize_kernel<kDqResidual><<<grid, kDqThreads, 0, stream>>>(codes, dq_codes, dq_scales, n16, out, fmt, W0);
+  else if (bf16)
+    dequantize_kernel<kDqBf16><<<grid, kDqThreads, 0, stream>>>(codes, dq_codes, dq_scales, n16, out, fmt, nullptr);
   else
-    dequantize_kernel<false><<<grid, kDqThreads, 0, stream>>>(codes, dq_codes, dq_scales, n16, out, fmt);
+    dequantize_kernel<kDqF32><<<grid, kDqThreads, 0, stream>>>(codes, dq_codes, dq_scales, n16, out, fmt, nullptr);
   timing_after(QLORA_KERNEL_DEQUANTIZE, stream);
   count_launch();
   return cudaGetLastError();

@@ -44,8 +44,13 @@ constexpr int kFmtE4M3 = 0, kFmtU8 = 1, kFmtInt16 = 2;
 // dq_u8 / u8: the absmax codes are linear uint8 (s = max / 255) instead of E4M3.
 cudaError_t launch_quantize_nf4(const float* W0, int64_t n, uint8_t* codes, uint8_t* dq_codes,
                                 float* dq_scales, cudaStream_t stream, bool dq_u8 = false);
+// With W0 != nullptr the output is the fp32 residual fl32(W0 - w') instead (bf16 ignored).
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* dq_codes, const float* dq_scales,
-                              int64_t n, bool bf16, void* out, cudaStream_t stream, int fmt = kFmtE4M3);
+                              int64_t n, bool bf16, void* out, cudaStream_t stream, int fmt = kFmtE4M3,
+                              const float* W0 = nullptr);
+// A = bf16(U[:, :r] fl32(sqrt S)), B = bf16(fl32(sqrt S) Vh[:r, :]); row strides ldu, ldv (elements).
+cudaError_t launch_loftq_split(const float* U, int64_t ldu, const float* S, const float* Vh, int64_t ldv,
+                               int64_t n_in, int64_t n_out, int r, uint16_t* A, uint16_t* B, cudaStream_t stream);
 cudaError_t launch_merge(const uint8_t* codes, const uint8_t* dq_codes, const float* dq_scales,
                          const uint16_t* A, const uint16_t* B, int r, int64_t n_in, int64_t n_out,
                          bool bf16, void* out, cudaStream_t stream, int fmt = kFmtE4M3);
@@ -121,6 +126,15 @@ size_t fwd_gemm_split_bytes(int64_t M, int64_t n_in, int64_t n_out, int r);
 size_t dx_gemm_split_bytes(int64_t M, int64_t n_in, int64_t n_out, int r);
 // Most CTAs the GEMMs use (0: one per SM); a testing and tuning knob.
 void set_gemm_ctas(int ctas);
+
+// Synchronise `stream` and read (then clear) the quantiser's device status word.
+cudaError_t quantize_status_take(cudaStream_t stream, uint32_t* flags);
+
+// One bounded wait that nothing completes (kind 0: an mbarrier without
+// arrivals; kind 1: `counter`, left at 0, awaited to reach 1), giving up after
+// limit_ns and raising kFlagTimeoutSelftest in `status`.
+cudaError_t launch_selftest_wait(uint32_t* status, const uint32_t* counter, int kind, uint64_t limit_ns,
+                                 cudaStream_t stream);
 
 // Smallest workspace a forward/backward call accepts (no split tiles); the
 // size qlora_workspace_bytes returns also holds the split region.

@@ -12,12 +12,15 @@
 // The array is a file-scope __device__ variable: every GPU that loads the
 // library holds its kStaticWsBytes until the process exits.  In host code the
 // array's name is only a host-side stand-in, so its device address is looked up
-// with cudaGetSymbolAddress, once per device, on the first call made with that
-// device current; that first call should come before any stream capture.  All
-// calls share the array and it keeps the previous call's contents, so each call
-// first zeroes the part that must start at zero (the status word).  Two calls
-// whose work overlaps on the GPU (different streams, or different host threads)
-// race on the array.
+// with cudaGetSymbolAddress on the device that is current: on every call made
+// outside a stream capture (cheap, and correct again after the device's
+// context was reset), and from a per-device cache during a capture, which
+// therefore needs one earlier call on that device.  All calls share the array
+// and it keeps the previous call's contents, so each call first zeroes the
+// GEMM's split counters, which must start at zero; the status word is left as
+// it is until qlora_static_ws_status reads and clears it.  Two calls whose work
+// overlaps on the GPU (different streams, or different host threads) race on
+// the array.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -34,13 +37,20 @@ static __device__ __align__(256) unsigned char g_static_ws[kStaticWsBytes];
 std::mutex g_setup_mutex;
 void* g_static_ws_addr[64] = {};
 
-// Device address of g_static_ws on the current device (looked up once).
-qlora_status static_ws_address(void** out) {
+// Device address of g_static_ws on the current device: looked up again outside
+// a capture of `stream`, taken from the per-device cache inside one.
+qlora_status static_ws_address(void** out, cudaStream_t stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_CUDA;
   if (dev < 0 || dev >= 64) return QLORA_ERR_UNSUPPORTED_DEVICE;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (!g_static_ws_addr[dev]) {
+  if (cs == cudaStreamCaptureStatusNone || !g_static_ws_addr[dev]) {
+    if (cs != cudaStreamCaptureStatusNone) return QLORA_ERR_INVALID_ARG;   // no earlier call on this device
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_static_ws) != cudaSuccess || !ptr) {
       cudaGetLastError();
@@ -58,15 +68,25 @@ extern "C" qlora_status qlora_linear_fwd_static_ws(const qlora_nf4_weight* w, co
                                                    const uint16_t* A, const uint16_t* B, int r, uint16_t* Y,
                                                    uint16_t* V_save, void* stream) {
   if (!w) return QLORA_ERR_INVALID_ARG;
-  // the smallest workspace the forward accepts: the GEMM keeps its tiles whole
-  // (the split region would not fit the fixed array at the usual sizes)
+  // the smallest workspace the forward accepts (everything but the GEMM's split
+  // partial tiles): the GEMM keeps its tiles whole here
   const size_t need = qlora::ws_min_bytes(QLORA_OP_FWD, M, w->in, w->out, r);
   if (need == 0) return QLORA_ERR_SHAPE;
   if (need > kStaticWsBytes) return QLORA_ERR_WORKSPACE;   // larger than the fixed array
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   void* ws = nullptr;
-  const qlora_status st = static_ws_address(&ws);
+  const qlora_status st = static_ws_address(&ws, s);
   if (st != QLORA_OK) return st;
-  if (cudaMemsetAsync(ws, 0, qlora::kWsFixedBytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+  if (cudaMemsetAsync(static_cast<unsigned char*>(ws) + qlora::kWsStatusBytes, 0, qlora::kWsCounterBytes, s) !=
+      cudaSuccess)
     return QLORA_ERR_CUDA;
   return qlora_linear_fwd(w, X, M, A, B, r, Y, V_save, ws, need, stream);
+}
+
+extern "C" qlora_status qlora_static_ws_status(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* ws = nullptr;
+  const qlora_status st = static_ws_address(&ws, s);
+  if (st != QLORA_OK) return st;
+  return qlora_ws_status(ws, stream);
 }

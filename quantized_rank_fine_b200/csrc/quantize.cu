@@ -52,6 +52,11 @@ constexpr uint32_t kHalfBytes = kHalfBlocks * kBlock * 4;   // 32 KB of fp32
 constexpr int kCells = 65;
 constexpr float kRoundBase = 12582912.0f;            // 1.5 * 2^23: integers land in the low bits
 
+// Status word of the quantiser (it takes no workspace): a bounded wait for a
+// bulk copy that gives up raises a bit here; qlora_quantize_status reads and
+// clears it.  One per device (a __device__ variable of the module).
+__device__ uint32_t g_quantize_status;
+
 // Fast code of q; `near` accumulates whether q is within 2^-19 of the cell's threshold.
 __device__ __forceinline__ uint32_t fast_code(float q, const uint32_t* __restrict__ lut, bool& near) {
   const float f = fmaf(q, 32.0f, 32.0f + kRoundBase);
@@ -139,7 +144,7 @@ quantize_nf4_kernel(const float* __restrict__ W0, int64_t nblocks, int64_t ngrou
       if (h * kHalfBlocks >= nblk) break;          // a short last group
       const int b = static_cast<int>(j % kQBuf);
       const uint32_t ph = static_cast<uint32_t>((j / kQBuf) & 1);
-      const bool got = sm100::mbar_wait(bar0 + 8 * b, ph, nullptr, 0);
+      const bool got = sm100::mbar_wait(bar0 + 8 * b, ph, &g_quantize_status, kFlagTimeoutProducer);
       if (!__syncthreads_and(got)) {
         failed_at = j;
         break;
@@ -226,7 +231,8 @@ quantize_nf4_kernel(const float* __restrict__ W0, int64_t nblocks, int64_t ngrou
     for (int64_t k = failed_at; k < failed_at + kQBuf; ++k) {
       const int64_t gk = blockIdx.x + (k >> 1) * gridDim.x;
       if (gk >= ngroups || gk * kGroup + (k & 1) * kHalfBlocks >= nblocks) continue;
-      sm100::mbar_wait(bar0 + 8 * static_cast<int>(k % kQBuf), static_cast<uint32_t>((k / kQBuf) & 1), nullptr, 0);
+      sm100::mbar_wait(bar0 + 8 * static_cast<int>(k % kQBuf), static_cast<uint32_t>((k / kQBuf) & 1),
+                       &g_quantize_status, kFlagTimeoutProducer);
     }
   }
   __syncthreads();
@@ -257,6 +263,18 @@ cudaError_t launch_quantize_nf4(const float* W0, int64_t n, uint8_t* codes, uint
   timing_after(QLORA_KERNEL_QUANTIZE, stream);
   count_launch();
   return cudaGetLastError();
+}
+
+// Synchronise `stream`, then report (and clear) the quantiser's status word.
+cudaError_t quantize_status_take(cudaStream_t stream, uint32_t* flags) {
+  *flags = 0;
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(flags, g_quantize_status, sizeof(uint32_t));
+  if (e == cudaSuccess && *flags != 0) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyToSymbol(g_quantize_status, &zero, sizeof(uint32_t));
+  }
+  return e;
 }
 
 }  // namespace qlora

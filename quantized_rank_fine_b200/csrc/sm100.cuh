@@ -59,18 +59,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity, uin
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 
-// Wait until the phase with the given parity has completed; false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t* status,
-                                          uint32_t flag) {
+// Wait until the phase with the given parity has completed; false (with `flag`
+// raised in the status word) once `limit_ns` of global time have passed.
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, uint32_t* status, uint32_t flag,
+                                                uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_timer() - t0 > kWaitLimitNs) {
+  while (!mbar_try_wait(bar, parity, limit_ns < 0x100000u ? static_cast<uint32_t>(limit_ns) : 0x100000u)) {
+    if (global_timer() - t0 > limit_ns) {
       raise_flag(status, flag);
       return false;
     }
   }
   return true;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t* status, uint32_t flag) {
+  return mbar_wait_limit(bar, parity, status, flag, kWaitLimitNs);
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -344,20 +349,24 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   return v;
 }
 
-// Wait until *p >= target (acquire); false after the wait limit, with the flag
-// raised in the status word.
-__device__ __forceinline__ bool wait_counter(const uint32_t* p, uint32_t target, uint32_t* status,
-                                             uint32_t flag) {
+// Wait until *p >= target (acquire); false after `limit_ns`, with the flag raised
+// in the status word.
+__device__ __forceinline__ bool wait_counter_limit(const uint32_t* p, uint32_t target, uint32_t* status,
+                                                   uint32_t flag, uint64_t limit_ns) {
   if (ld_acquire_gpu(p) >= target) return true;
   const uint64_t t0 = global_timer();
   while (ld_acquire_gpu(p) < target) {
     __nanosleep(128);
-    if (global_timer() - t0 > kWaitLimitNs) {
+    if (global_timer() - t0 > limit_ns) {
       raise_flag(status, flag);
       return false;
     }
   }
   return true;
+}
+
+__device__ __forceinline__ bool wait_counter(const uint32_t* p, uint32_t target, uint32_t* status, uint32_t flag) {
+  return wait_counter_limit(p, target, status, flag, kWaitLimitNs);
 }
 
 // ---------------------------------------------------------------- dependent launches

@@ -184,3 +184,19 @@ def test_int16_weight_descriptor_checks(L):
     assert L.qlora_dequantize(ctypes.byref(w_int), FAKE, 0, None) != 1
     w_nf4 = q._Weight(0x10000, 0, 0x10000, 256, 256, q.QLORA_DQ_E4M3)
     assert L.qlora_dequantize(ctypes.byref(w_nf4), FAKE, 0, None) == 1
+
+
+def test_selftest_and_status_calls_check_arguments_first(L):
+    """The failure-path self-test rejects a bad kind, limit or workspace before it
+    looks for a device; the status calls report an error (and do not crash) when
+    there is no usable device."""
+    fake = ctypes.c_void_p(4096)
+    assert L.qlora_selftest_wait_timeout(fake, 4096, 2, 50, None) == 1        # unknown kind
+    assert L.qlora_selftest_wait_timeout(fake, 4096, 0, 0, None) == 1         # limit 0
+    assert L.qlora_selftest_wait_timeout(fake, 4096, 1, 1000001, None) == 1   # limit above 1 s
+    assert L.qlora_selftest_wait_timeout(None, 4096, 0, 50, None) == 4        # no workspace
+    assert L.qlora_selftest_wait_timeout(fake, 1279, 0, 50, None) == 4        # shorter than the prefix
+    import torch
+    if not torch.cuda.is_available():
+        assert L.qlora_quantize_status(None) != 0
+        assert L.qlora_static_ws_status(None) != 0

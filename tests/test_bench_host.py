@@ -88,14 +88,17 @@ def test_reference_arm_torchrun_world2():
 
 
 def test_workload_defaults_and_bytes(monkeypatch):
-    """Per-workload defaults, and the stack's activation bytes counting each
-    shared X once (q, k, v share one input, gate and up another)."""
-    monkeypatch.setattr(sys, "argv", ["bench.py", "--workload", "llama7b_stack_m2048_r16"])
+    """Per-workload defaults (the Llama-7B stack is the default workload, with
+    every row), and the stack's activation bytes counting each shared X once
+    (q, k, v share one input, gate and up another)."""
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--workload", "attn4096_m4096_r16"])
     a = bench.parse()
-    assert (a.steps, a.warmup, a.rows) == (20, 3, "")
+    assert (a.steps, a.warmup, a.rows) == (2000, 10, "all")
     monkeypatch.setattr(sys, "argv", ["bench.py"])
     a = bench.parse()
-    assert (a.steps, a.warmup, a.rows, a.workload) == (2000, 10, "all", "attn4096_m4096_r16")
+    assert (a.steps, a.warmup, a.rows, a.workload) == (20, 3, "all", "llama7b_stack_m2048_r16")
+    assert set(bench.ROW_NAMES) >= {"quantize", "gemv", "mlp_m8192"}
+    assert bench.weight_row_shape(bench.WORKLOADS["llama7b_stack_m2048_r16"]) == (4096, 11008)
     wl = bench.WORKLOADS["llama7b_stack_m2048_r16"]
     assert len(wl["shapes"]) == 224
     M = wl["M"]

@@ -62,3 +62,42 @@ def test_loftq_init_matches_oracle(n_in, n_out, r):
     assert_close(_f64(A.float() @ B.float()), A_ref @ B_ref, "A B")
     R = _f64(W0) - _f64(q.qlora_dequantize(w, torch.float32))
     assert np.linalg.norm(R - _f64(A.float() @ B.float())) < np.linalg.norm(R)
+
+
+@pytest.mark.parametrize("shape,fmt", [((512, 384), "nf4"), ((4096, 11008), "nf4"), ((320, 192), "u8"),
+                                       ((256, 512), "int16")])
+def test_loftq_residual_bitexact(shape, fmt):
+    """R = fl32(W0 - w') from the library kernel equals the oracle's residual
+    (exact in float64) rounded once to fp32, bit for bit, for NF4 weights with
+    either absmax code format and for the INT (one scale per 16) format."""
+    from oracle import intq
+    W0 = synth.normal(f"resid{shape}", shape, 0.02, device="cuda")
+    W0h = W0.cpu().numpy()
+    if fmt == "int16":
+        codes, scales = q.qlora_quantize_int(W0, 4)
+        w = q.int_weight(codes, scales, *shape)
+        ref = W0h.astype(np.float64) - intq.dequantize_int(codes.cpu().numpy(), scales.cpu().numpy(), *shape)
+    else:
+        w = q.qlora_quantize_nf4(W0, dq_format=q.QLORA_DQ_U8 if fmt == "u8" else q.QLORA_DQ_E4M3)
+        deq = nf4.dequantize(w.codes.cpu().numpy(), w.dq_codes.cpu().numpy(), w.dq_scales.cpu().numpy(), *shape,
+                             dq_format="u8" if fmt == "u8" else "e4m3")
+        ref = W0h.astype(np.float64) - deq.astype(np.float64)
+        if fmt == "nf4":
+            np.testing.assert_array_equal(ref, loftq.residual(W0h))
+    R = q.qlora_loftq_residual(W0, w)
+    torch.cuda.synchronize()
+    assert np.array_equal(R.cpu().numpy().view(np.uint32), nf4.fl32(ref).view(np.uint32))
+
+
+@pytest.mark.parametrize("n_in,n_out,k,r", [(512, 384, 384, 8), (1024, 1024, 1024, 16), (4096, 11008, 64, 64)])
+def test_loftq_split_bitexact(n_in, n_out, k, r):
+    """A and B from given fp32 factors (U with k > r columns, Vh with k rows)
+    equal the oracle's stored-precision split bit for bit."""
+    U = synth.normal(f"splitU{n_in}", (n_in, k), 1.0 / np.sqrt(n_in), device="cuda")
+    S = synth.normal(f"splitS{k}", (k,), 1.0, device="cuda").abs().sort(descending=True).values.contiguous()
+    Vh = synth.normal(f"splitV{n_out}", (k, n_out), 1.0 / np.sqrt(n_out), device="cuda")
+    A, B = q.qlora_loftq_split(U, S, Vh, r)
+    torch.cuda.synchronize()
+    Ar, Br = loftq.split_adapters(U.cpu().numpy(), S.cpu().numpy(), Vh.cpu().numpy(), r)
+    assert np.array_equal(A.float().cpu().numpy().view(np.uint32), Ar.view(np.uint32))
+    assert np.array_equal(B.float().cpu().numpy().view(np.uint32), Br.view(np.uint32))

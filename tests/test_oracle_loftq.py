@@ -75,3 +75,53 @@ def test_small_corrections_are_mostly_lost():
     big = loftq.lost_fraction(Wq, A, 30 * B, W_big)
     assert small > 0.5          # most of a small correction is lost
     assert big < small / 2      # a larger one is kept much better
+
+
+def test_split_adapters_exact_on_representable_values():
+    """Square roots and products that are exact in fp32 and bf16 (singular values
+    16, 4, 2.25, 0.25; factors with a few significant bits): the split gives
+    U s and s Vt exactly, as computed here with rationals."""
+    from fractions import Fraction
+    S = np.array([16.0, 4.0, 2.25, 0.25, 9.0], np.float32)
+    roots = [Fraction(4), Fraction(2), Fraction(3, 2), Fraction(1, 2)]
+    rng = np.random.default_rng(3)
+    vals = np.array([1.0, -1.0, 0.5, -0.75, 0.125, 1.5, -0.375, 0.0], np.float32)
+    U = vals[rng.integers(0, len(vals), (6, 5))]
+    Vt = vals[rng.integers(0, len(vals), (5, 7))]
+    A, B = loftq.split_adapters(U, S, Vt, 4)
+    for i in range(6):
+        for j in range(4):
+            assert Fraction(float(A[i, j])) == Fraction(float(U[i, j])) * roots[j]
+    for j in range(4):
+        for o in range(7):
+            assert Fraction(float(B[j, o])) == roots[j] * Fraction(float(Vt[j, o]))
+    assert A.shape == (6, 4) and B.shape == (4, 7)
+
+
+def test_split_adapters_product_and_gram_within_bf16_rounding():
+    """On an exact SVD of a random matrix (fp32 factors), A B equals the rank-r
+    truncation U_r diag(S_r) Vt_r, and A^T A equals diag(S_r), each within the
+    rounding of bf16 storage (relative 2^-8 per factor)."""
+    rng = np.random.default_rng(4)
+    R = rng.normal(size=(96, 80))
+    U, S, Vt = np.linalg.svd(R, full_matrices=False)
+    U32, S32, Vt32 = U.astype(np.float32), S.astype(np.float32), Vt.astype(np.float32)
+    r = 12
+    A, B = loftq.split_adapters(U32, S32, Vt32, r)
+    ref = (U32[:, :r].astype(np.float64) * S32[:r].astype(np.float64)) @ Vt32[:r].astype(np.float64)
+    bound = 2 * 2.0 ** -8 * (np.abs(U32[:, :r]) * S32[:r]) @ np.abs(Vt32[:r])
+    assert np.all(np.abs(A.astype(np.float64) @ B.astype(np.float64) - ref) <= bound + 1e-12)
+    gram = A.astype(np.float64).T @ A.astype(np.float64)
+    np.testing.assert_allclose(np.diag(gram), S[:r], rtol=2 * 2.0 ** -8)
+
+
+def test_split_adapters_agrees_with_the_float64_split():
+    """The stored-precision split of the oracle's own SVD is the float64 split of
+    loftq_init rounded: within 2^-7 relative, element by element."""
+    W0 = _w0()
+    R = loftq.residual(W0)
+    U, S, Vt = np.linalg.svd(R, full_matrices=False)
+    A, B = loftq.split_adapters(U.astype(np.float32), S.astype(np.float32), Vt.astype(np.float32), 8)
+    A64, B64 = loftq.loftq_init(W0, 8)
+    assert np.all(np.abs(A - A64) <= 2.0 ** -7 * np.abs(A64) + 1e-30)
+    assert np.all(np.abs(B - B64) <= 2.0 ** -7 * np.abs(B64) + 1e-30)
