@@ -30,8 +30,12 @@
 //              K-steps (one thread per 64 weights per step): codes from shared
 //              memory -> 16-entry bf16 table per 64-weight block (NF4) or per
 //              16-weight group (INT) -> byte-permute lookup -> 16-byte stores in
-//              the UMMA canonical layout; then the epilogue (TMEM -> registers
-//              -> global), all 8 warps.
+//              the UMMA canonical layout; then the epilogue, all 8 warps:
+//              TMEM -> registers -> bf16 -> a 32 x 32 block in shared memory
+//              (64-byte swizzle) -> one TMA tensor store per block, so every
+//              output line is written whole.  The staging blocks live in the
+//              dequantised-weight regions of the ring, which no one else
+//              touches while the dequant warps run the epilogue.
 // Barriers per stage: `loaded` (this CTA's TMA bytes), `ready` (in the even CTA:
 // the 4 dequant warps of each CTA that took the stage, each after its CTA's
 // stage has landed and its weight half is written) and `free` (the pair MMAs'
@@ -207,15 +211,18 @@ template <bool kDX, bool kInt>
 __global__ void __launch_bounds__(kThreads, 1)
 nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_ext_a,
                 const __grid_constant__ CUtensorMap tm_ext_b, const __grid_constant__ CUtensorMap tm_codes,
-                const GemmArgs p) {
+                const __grid_constant__ CUtensorMap tm_out, const GemmArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 3);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 4);
   const uint32_t loaded0 = smem_addr(bars), ready0 = smem_addr(bars + kStages);
   const uint32_t free0 = smem_addr(bars + 2 * kStages), tmem_full = smem_addr(bars + 3 * kStages);
   const uint32_t tmem_empty = smem_addr(bars + 3 * kStages + 1);
   const uint32_t mma_drained = smem_addr(bars + 3 * kStages + 2);
+  // the 8 epilogue warps of this CTA are done staging an item's output in the
+  // dequantised-weight regions (they may then be refilled)
+  const uint32_t staging_free = smem_addr(bars + 3 * kStages + 3);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();         // 0: issues the pair's MMAs
@@ -236,6 +243,7 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
     mbar_init(tmem_full, 1);
     mbar_init(tmem_empty, 2 * kDeqWarps);
     mbar_init(mma_drained, 1);
+    mbar_init(staging_free, kDeqWarps);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -247,6 +255,7 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
     tma_prefetch_desc(&tm_ext_a);
     tma_prefetch_desc(&tm_ext_b);
     tma_prefetch_desc(&tm_codes);
+    tma_prefetch_desc(&tm_out);
   }
   // both CTAs' barriers initialised and TMEM allocated before any cross-CTA use
   tc_fence_before();
@@ -267,6 +276,7 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int g = 0;        // K-steps issued so far (ring position)
+      int sf_done = 0;  // epilogues (staging_free phases) seen complete
       bool alive = true;
       WorkItem w;
       for (int it = 0; alive && work_item(p, S, it, w); ++it) {
@@ -291,6 +301,17 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
             else tma_load_2d(c_dst, &tm_codes, bar, kb * (kBK / 2), nh);
           } else {
             const int j = kb - nkb_w;
+            // the adapter's weight tile lands in the dequantised-weight region,
+            // which the previous item's epilogue may still use as output staging:
+            // wait for the epilogues of items 0 .. it-1, phase by phase (in order,
+            // so that no parity is mistaken for the one two phases later)
+            bool ok = true;
+            for (; ok && sf_done < it; ++sf_done)
+              ok = mbar_wait(staging_free, static_cast<uint32_t>(sf_done & 1), p.status, kFlagTimeoutProducer);
+            if (!ok) {
+              alive = false;
+              break;
+            }
             mbar_arrive_expect_tx(bar, kABytes + kBBytes);
             tma_load_2d(a_dst, &tm_ext_a, bar, j * kBK, ma);
             tma_load_2d(a_dst + kABytes / 2, &tm_ext_a, bar, j * kBK, ma + kBM);
@@ -389,6 +410,10 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
     // of column block cb sits at ((cb * 2 + half) * 4 + quarter) * 256 + q * 32 + lane,
     // so each warp store covers 512 contiguous bytes
     const uint32_t slot_lane = ((half * 4 + quarter) * 8) * 32 + lane;
+    // this warp's two 2 KB output staging blocks: in the dequantised-weight
+    // region of stage (warp - 2) / 2, the warp's half of it
+    const uint32_t stage_out = smem_addr(smem + ((warp - 2) >> 1) * kStageBytes + kABytes) +
+                               static_cast<uint32_t>((warp - 2) & 1) * (kBBytes / 2);
 
     int g = 0;
     bool alive = true;
@@ -508,7 +533,9 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
           for (int c = pair + 1; c < c_end; ++c)
             have = have && wait_counter(p.counters + 2 * c + rank, kDeqWarps, p.status, kFlagTimeoutEpilogue);
         }
-        const int64_t row = m0 + half * kBM + kHalfN * rank + quarter * 32 + lane;
+        // the warp's 32 rows; each 32-column block goes out through shared
+        // memory as one TMA store (rows and columns past the output are clipped)
+        const int64_t row0 = m0 + half * kBM + kHalfN * rank + quarter * 32;
 #pragma unroll 1
         for (int cb = 0; cb < kBN / 32; ++cb) {
           uint32_t v[32];
@@ -532,26 +559,41 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
             }
           }
           const int64_t col = n0 + cb * 32;
-          if (row < p.M && col < p.N) {
-            uint4* dst = reinterpret_cast<uint4*>(p.D + row * p.N + col);
+          const uint32_t buf = stage_out + static_cast<uint32_t>(cb & 1) * 2048u;
+          // the store issued from this block two rounds ago has read it
+          if (lane == 0 && cb >= 2) bulk_wait_read<1>();
+          __syncwarp();
+          // row `lane` of the block, 64 bytes as four 16-byte chunks, chunk c at
+          // c ^ ((row >> 1) & 3) (the 64-byte swizzle of the tensor map)
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint4 o;
-              o.x = pack_bf16x2(acc[8 * q + 0], acc[8 * q + 1]);
-              o.y = pack_bf16x2(acc[8 * q + 2], acc[8 * q + 3]);
-              o.z = pack_bf16x2(acc[8 * q + 4], acc[8 * q + 5]);
-              o.w = pack_bf16x2(acc[8 * q + 6], acc[8 * q + 7]);
-              dst[q] = o;
-            }
+          for (int q = 0; q < 4; ++q)
+            st_shared_v4(buf + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4), pack_bf16x2(acc[8 * q + 0], acc[8 * q + 1]),
+                         pack_bf16x2(acc[8 * q + 2], acc[8 * q + 3]), pack_bf16x2(acc[8 * q + 4], acc[8 * q + 5]),
+                         pack_bf16x2(acc[8 * q + 6], acc[8 * q + 7]));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && row0 < p.M && col < p.N) {
+            tma_store_2d(&tm_out, buf, static_cast<int32_t>(col), static_cast<int32_t>(row0));
+            bulk_commit();
           }
         }
+        // both staging blocks read before the dequant warps reuse the region
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
       }
+      // no warp writes the next item's weight tiles into a region another warp
+      // may still be staging from: every warp arrives, then waits (bounded) for all
+      __syncwarp();
+      if (lane == 0) mbar_arrive(staging_free);
+      if (!__all_sync(0xffffffffu, mbar_wait(staging_free, it & 1, p.status, kFlagTimeoutEpilogue))) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tmem_empty_lead);
     }
   }
 
+  // every output store of this thread has completed
+  if (warp >= 2 && lane == 0) bulk_wait<0>();
   // Both CTAs are done with TMEM (the even CTA's MMAs have all completed: every
   // epilogue waited for the last commit or gave up) before the pair frees it.
   tc_fence_before();
@@ -685,7 +727,7 @@ size_t plan_ws_bytes(const GemmPlan& P) {
 
 template <bool kDX, bool kInt>
 cudaError_t launch_gemm(const CUtensorMap& act, const CUtensorMap& ea, const CUtensorMap& eb, const CUtensorMap& cm,
-                        GemmArgs a, uint32_t* counters, void* partials, size_t partial_bytes,
+                        const CUtensorMap& om, GemmArgs a, uint32_t* counters, void* partials, size_t partial_bytes,
                         cudaStream_t stream) {
   const cudaError_t pe = prepare_kernel<kDX, kInt>();
   if (pe != cudaSuccess) return pe;
@@ -712,7 +754,7 @@ cudaError_t launch_gemm(const CUtensorMap& act, const CUtensorMap& ea, const CUt
   cfg.numAttrs = 2;
   const int which = kDX ? QLORA_KERNEL_DX_GEMM : QLORA_KERNEL_FWD_GEMM;
   timing_before(which, stream);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, nf4_gemm_kernel<kDX, kInt>, act, ea, eb, cm, a);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, nf4_gemm_kernel<kDX, kInt>, act, ea, eb, cm, om, a);
   timing_after(which, stream);
   count_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
@@ -724,34 +766,40 @@ cudaError_t launch_gemm(const CUtensorMap& act, const CUtensorMap& ea, const CUt
 cudaError_t launch_fwd_gemm(const WeightView& w, const uint16_t* X, const uint16_t* V, const uint16_t* B,
                             int64_t M, int r, uint16_t* Y, uint32_t* status, uint32_t* counters,
                             void* partials, size_t partial_bytes, cudaStream_t stream) {
-  CUtensorMap act, ea, eb, cm;
+  CUtensorMap act, ea, eb, cm, om;
   // activations in 128-row boxes; codes as a (in x out/2) byte matrix: 64 rows x
-  // 64 bytes (one CTA's 128 columns) per K-step, 64-byte swizzle
+  // 64 bytes (one CTA's 128 columns) per K-step, 64-byte swizzle; Y stored in
+  // 32 x 32 blocks, 64-byte swizzle
   if (!make_map(&act, X, M, w.in, 64, 128) || !make_map(&ea, V, M, r, 64, 128) ||
       !make_map(&eb, B, r, w.out, 64, 64) ||
-      !make_map_t(&cm, w.codes, w.in, w.out / 2, 64, 64, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, CU_TENSOR_MAP_SWIZZLE_64B))
+      !make_map_t(&cm, w.codes, w.in, w.out / 2, 64, 64, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map_t(&om, Y, M, w.out, 32, 32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   GemmArgs a{w.codes, w.dq_codes, w.dq_scales, w.out, M, w.out, w.in, r, Y, status, w.fmt == kFmtU8 ? 1 : 0,
              0, 0, 0, nullptr, nullptr};
-  return w.fmt == kFmtInt16 ? launch_gemm<false, true>(act, ea, eb, cm, a, counters, partials, partial_bytes, stream)
-                            : launch_gemm<false, false>(act, ea, eb, cm, a, counters, partials, partial_bytes, stream);
+  return w.fmt == kFmtInt16
+             ? launch_gemm<false, true>(act, ea, eb, cm, om, a, counters, partials, partial_bytes, stream)
+             : launch_gemm<false, false>(act, ea, eb, cm, om, a, counters, partials, partial_bytes, stream);
 }
 
 // dX = dY deq(W)^T + U A^T.
 cudaError_t launch_dx_gemm(const WeightView& w, const uint16_t* dY, const uint16_t* U, const uint16_t* A,
                            int64_t M, int r, uint16_t* dX, uint32_t* status, uint32_t* counters,
                            void* partials, size_t partial_bytes, cudaStream_t stream) {
-  CUtensorMap act, ea, eb, cm;
+  CUtensorMap act, ea, eb, cm, om;
   // activations in 128-row boxes; codes as a (in x out/2) byte matrix: 128 rows
-  // (one CTA's columns of dX) x 32 bytes per K-step, 32-byte swizzle
+  // (one CTA's columns of dX) x 32 bytes per K-step, 32-byte swizzle; dX stored
+  // in 32 x 32 blocks, 64-byte swizzle
   if (!make_map(&act, dY, M, w.out, 64, 128) || !make_map(&ea, U, M, r, 64, 128) ||
       !make_map(&eb, A, w.in, r, 64, 128) ||
-      !make_map_t(&cm, w.codes, w.in, w.out / 2, 32, 128, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, CU_TENSOR_MAP_SWIZZLE_32B))
+      !make_map_t(&cm, w.codes, w.in, w.out / 2, 32, 128, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, CU_TENSOR_MAP_SWIZZLE_32B) ||
+      !make_map_t(&om, dX, M, w.in, 32, 32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   GemmArgs a{w.codes, w.dq_codes, w.dq_scales, w.out, M, w.in, w.out, r, dX, status, w.fmt == kFmtU8 ? 1 : 0,
              0, 0, 0, nullptr, nullptr};
-  return w.fmt == kFmtInt16 ? launch_gemm<true, true>(act, ea, eb, cm, a, counters, partials, partial_bytes, stream)
-                            : launch_gemm<true, false>(act, ea, eb, cm, a, counters, partials, partial_bytes, stream);
+  return w.fmt == kFmtInt16
+             ? launch_gemm<true, true>(act, ea, eb, cm, om, a, counters, partials, partial_bytes, stream)
+             : launch_gemm<true, false>(act, ea, eb, cm, om, a, counters, partials, partial_bytes, stream);
 }
 
 size_t fwd_gemm_split_bytes(int64_t M, int64_t n_in, int64_t n_out, int r) {
