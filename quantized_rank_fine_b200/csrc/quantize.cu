@@ -128,9 +128,14 @@ quantize_nf4_kernel(const float* __restrict__ W0, int64_t nblocks, int64_t ngrou
   if (tid == 0) {
     for (int b = 0; b < kQBuf; ++b) sm100::mbar_init(bar0 + 8 * b, 1);
     sm100::fence_mbar_init();
+    // W0 may be written by the kernel this one follows (programmatic dependent
+    // launch): the set-up above overlaps its tail, the copies wait for it
+    sm100::grid_dependency_wait();
     for (int j = 0; j < kQBuf; ++j) issue_half(j, W0, nblocks, ngroups, buf0, bar0);
   }
   __syncthreads();
+  // the outputs are written only after the kernel before has completed
+  sm100::grid_dependency_wait();
 
   const int quarter = lane & 3;            // which 16 weights of its block
   const int bsub = lane >> 2;              // block among the 8 of an iteration
@@ -257,12 +262,22 @@ cudaError_t launch_quantize_nf4(const float* W0, int64_t n, uint8_t* codes, uint
     set[dev] = true;
   }
   const int64_t grid = std::min<int64_t>(ngroups, 2 * (dev < 64 ? sms[dev] : 148));
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kQThreads);
+  cfg.dynamicSmemBytes = kQBuf * kHalfBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
   timing_before(QLORA_KERNEL_QUANTIZE, stream);
-  quantize_nf4_kernel<<<static_cast<unsigned>(grid), kQThreads, kQBuf * kHalfBytes, stream>>>(
-      W0, nblocks, ngroups, codes, dq_codes, dq_scales, dq_u8);
+  const cudaError_t e =
+      cudaLaunchKernelEx(&cfg, quantize_nf4_kernel, W0, nblocks, ngroups, codes, dq_codes, dq_scales, dq_u8);
   timing_after(QLORA_KERNEL_QUANTIZE, stream);
   count_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // Synchronise `stream`, then report (and clear) the quantiser's status word.
