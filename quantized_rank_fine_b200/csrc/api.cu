@@ -474,8 +474,8 @@ static qlora_status bwd_impl(const qlora_nf4_weight* w, const uint16_t* X, const
     V = Vw;
   }
   QLORA_CUDA(qlora::launch_dybt(dY, B, M, w->out, r, U, status, s, lo.scale, lo.drop));
-  QLORA_CUDA(qlora::launch_vtdy(V, dY, M, w->out, r, dB, status, s, nullptr, lo.accumulate));
-  QLORA_CUDA(qlora::launch_xtu(X, U, M, w->in, r, dA, status, s, nullptr, lo.accumulate));
+  QLORA_CUDA(qlora::launch_dbda(V, dY, X, U, M, w->in, w->out, r, dA, dB, status, s, nullptr, nullptr,
+                                lo.accumulate));
   if (dX) {
     const SplitRegion sr = split_region(ws, ws_bytes, L);
     QLORA_CUDA(qlora::launch_dx_gemm(wv, dY, U, A, M, r, dX, status, sr.counters, sr.partials, sr.partial_bytes, s));
@@ -552,20 +552,19 @@ qlora_status qlora_linear_bwd_adam(const qlora_nf4_weight* w, const uint16_t* X,
   pB.v = st->vB;
   pB.p16 = B;
 
-  // Every read of A or B comes before its update: U and V read them first, the
-  // B step follows U, dX reads A before the A step.
+  // Every read of A or B comes before its update: V, U and dX read them first,
+  // then one launch takes the B and A steps.
   if (!V) {
     uint16_t* Vw = reinterpret_cast<uint16_t*>(base + L.v_off);
     QLORA_CUDA(qlora::launch_xa(X, A, M, w->in, r, Vw, status, s, lo.scale, lo.drop));
     V = Vw;
   }
   QLORA_CUDA(qlora::launch_dybt(dY, B, M, w->out, r, U, status, s, lo.scale, lo.drop));
-  QLORA_CUDA(qlora::launch_vtdy(V, dY, M, w->out, r, nullptr, status, s, &pB));
   if (dX) {
     const SplitRegion sr = split_region(ws, ws_bytes, L);
     QLORA_CUDA(qlora::launch_dx_gemm(wv, dY, U, A, M, r, dX, status, sr.counters, sr.partials, sr.partial_bytes, s));
   }
-  QLORA_CUDA(qlora::launch_xtu(X, U, M, w->in, r, nullptr, status, s, &pA));
+  QLORA_CUDA(qlora::launch_dbda(V, dY, X, U, M, w->in, w->out, r, nullptr, nullptr, status, s, &pA, &pB));
   return QLORA_OK;
 }
 

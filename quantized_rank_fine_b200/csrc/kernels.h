@@ -91,11 +91,11 @@ cudaError_t launch_xa(const uint16_t* X, const uint16_t* A, int64_t M, int64_t n
 cudaError_t launch_dybt(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t n_out, int r,
                         uint16_t* U, uint32_t* status, cudaStream_t stream, float scale = 1.0f,
                         Dropout drop = {});
-cudaError_t launch_xtu(const uint16_t* X, const uint16_t* U, int64_t M, int64_t n_in, int r, float* dA,
-                       uint32_t* status, cudaStream_t stream, const AdamParams* adam = nullptr,
-                       bool accumulate = false);
-cudaError_t launch_vtdy(const uint16_t* V, const uint16_t* dY, int64_t M, int64_t n_out, int r,
-                        float* dB, uint32_t* status, cudaStream_t stream, const AdamParams* adam = nullptr,
+// dB (r x out, fp32, stored from dB^T = dY^T V) and dA = X^T U (in x r, fp32) in
+// one launch; with adam_a / adam_b the Adam step replaces the stores.
+cudaError_t launch_dbda(const uint16_t* V, const uint16_t* dY, const uint16_t* X, const uint16_t* U, int64_t M,
+                        int64_t n_in, int64_t n_out, int r, float* dA, float* dB, uint32_t* status,
+                        cudaStream_t stream, const AdamParams* adam_a = nullptr, const AdamParams* adam_b = nullptr,
                         bool accumulate = false);
 
 // Small-M forward (M <= kGemvMaxTokens): base + adapter in one kernel, the

@@ -9,13 +9,16 @@
 // by streaming the big operand (X or dY) from HBM once.  A CTA owns 128 output
 // rows and one slice of the reduction: TMA brings 128 x 64 (Aop) and 64 x 64
 // (Bop) bf16 tiles into a 3-stage shared-memory ring (128-byte swizzle, K- or
-// MN-major as the operand sits in memory; two CTAs per SM), one thread issues
+// MN-major as the operand sits in memory; two fit on an SM), one thread issues
 // tcgen05.mma into a 128 x r fp32 TMEM accumulator, and four warps move the
-// result out.  The reduction is split across CTAs so that the whole grid is
-// resident at once; the splits of a row tile form one thread-block cluster.
+// result out.  The reduction is split across CTAs so that the grid holds about
+// one CTA per SM; the splits of a row tile form one thread-block cluster.
 // Each split stores its TMEM rows straight into the shared memory of the CTA
 // that owns those rows (distributed shared memory); after one cluster barrier
 // the owners add the splits in order (deterministic, no workspace, no atomics).
+// One launch may carry two independent products of the same operand layouts
+// (dA and dB, which both reduce over the tokens): the row tiles of the second
+// follow those of the first in the grid, and both use the same split count.
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -114,10 +117,16 @@ __device__ __forceinline__ void store_pair(const SkArgs& p, int64_t row, int col
 
 // A_MN: Aop stored with the row index contiguous (MN-major), else k contiguous.
 // B_MN: Bop stored with the column index contiguous (MN-major), else k contiguous.
+// Row tiles [0, rt0) compute product 0 (tm_a0, tm_b0, p0), the rest product 1.
 template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(kSkThreads, 2)
-skinny_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                 const SkArgs p) {
+skinny_tc_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_b0,
+                 const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_b1,
+                 const __grid_constant__ SkArgs p0, const __grid_constant__ SkArgs p1, const int rt0) {
+  const bool second = static_cast<int>(blockIdx.x) >= rt0;
+  const SkArgs& p = second ? p1 : p0;
+  const CUtensorMap* tm_a = second ? &tm_a1 : &tm_a0;
+  const CUtensorMap* tm_b = second ? &tm_b1 : &tm_b0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* recv = reinterpret_cast<float*>(smem + kSkStages * kSkStage);       // [S][cap][64]
@@ -127,7 +136,7 @@ skinny_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
   const uint32_t tmem_full = smem_addr(bars + 2 * kSkStages);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kRowsT;
+  const int64_t row0 = static_cast<int64_t>(second ? static_cast<int>(blockIdx.x) - rt0 : blockIdx.x) * kRowsT;
   const int split = blockIdx.y;
   const int col0 = blockIdx.z * kColsT;
   const int cols = min(kColsT, p.r - col0);
@@ -152,8 +161,8 @@ skinny_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tm_a);
-    tma_prefetch_desc(&tm_b);
+    tma_prefetch_desc(tm_a);
+    tma_prefetch_desc(tm_b);
   }
   tc_fence_before();
   __syncthreads();
@@ -176,13 +185,13 @@ skinny_tc_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
         const int32_t k0 = static_cast<int32_t>(kbeg + kb * kKT);
         mbar_arrive_expect_tx(bar, kSkStage);
         if (!A_MN) {
-          tma_load_2d(a_dst, &tm_a, bar, k0, static_cast<int32_t>(row0));
+          tma_load_2d(a_dst, tm_a, bar, k0, static_cast<int32_t>(row0));
         } else {
-          tma_load_2d(a_dst, &tm_a, bar, static_cast<int32_t>(row0), k0);
-          tma_load_2d(a_dst + 8192, &tm_a, bar, static_cast<int32_t>(row0 + 64), k0);
+          tma_load_2d(a_dst, tm_a, bar, static_cast<int32_t>(row0), k0);
+          tma_load_2d(a_dst + 8192, tm_a, bar, static_cast<int32_t>(row0 + 64), k0);
         }
-        if (!B_MN) tma_load_2d(b_dst, &tm_b, bar, k0, col0);
-        else tma_load_2d(b_dst, &tm_b, bar, col0, k0);
+        if (!B_MN) tma_load_2d(b_dst, tm_b, bar, k0, col0);
+        else tma_load_2d(b_dst, tm_b, bar, col0, k0);
       }
     }
   } else if (warp == 1) {
@@ -310,7 +319,9 @@ bool bf16_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-constexpr int kResident = 2 * 148;   // CTAs that fit on the GPU at once
+// CTAs of one launch: one per SM.  Two fit on an SM, so the next rank-r launch
+// (a programmatic dependent) is resident and waiting while this one drains.
+constexpr int kResident = 148;
 
 struct Plan {
   int splits;
@@ -318,12 +329,13 @@ struct Plan {
   dim3 grid;
 };
 
-Plan plan(int64_t rows, int r, int64_t k_total) {
-  const int64_t rt = (rows + kRowsT - 1) / kRowsT;
+// Split count for one product (rows x r, reduction k_total) or two of the same
+// rank and reduction length (rows1 > 0): as many reduction slices as give one
+// CTA per SM (kResident), each slice at least two K-steps long.
+Plan plan(int64_t rows, int r, int64_t k_total, int64_t rows1 = 0) {
+  const int64_t rt = (rows + kRowsT - 1) / kRowsT + (rows1 + kRowsT - 1) / kRowsT;
   const int ct = (r + kColsT - 1) / kColsT;
   const int64_t ktiles = (k_total + kKT - 1) / kKT;
-  // as many reduction slices as keep the whole grid resident (one wave), each
-  // slice at least two K-steps long
   int64_t s = kResident / (rt * ct);
   s = std::min<int64_t>(s, std::max<int64_t>(1, ktiles / 2));
   s = std::max<int64_t>(1, std::min<int64_t>(s, kMaxSplits));
@@ -332,10 +344,21 @@ Plan plan(int64_t rows, int r, int64_t k_total) {
   return Plan{static_cast<int>(s), kps, dim3(static_cast<unsigned>(rt), static_cast<unsigned>(s), ct)};
 }
 
+// One product of the launch: its operand maps and what is stored where.
+struct Product {
+  CUtensorMap ta, tb;
+  int64_t rows;
+  void* out;
+  int out_kind;
+  const AdamParams* adam;
+  float scale;
+  Dropout drop;
+};
+
+// Launch product x (and product y, if given: same rank r and reduction k_total).
 template <bool A_MN, bool B_MN>
-cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows, int r, int64_t k_total, void* out,
-                int out_kind, uint32_t* status, cudaStream_t stream, const AdamParams* adam = nullptr,
-                float scale = 1.0f, bool accumulate = false, Dropout drop = {}) {
+cudaError_t run(const Product& x, const Product* y, int r, int64_t k_total, uint32_t* status, cudaStream_t stream,
+                bool accumulate) {
   static bool set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -347,9 +370,14 @@ cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows, int 
     if (e != cudaSuccess) return e;
     set[dev] = true;
   }
-  const Plan pl = plan(rows, r, k_total);
-  SkArgs a{rows, r, k_total, pl.kps, out, out_kind, status, adam ? 1 : 0, adam ? *adam : AdamParams{}, scale,
-           accumulate ? 1 : 0, drop.keep, drop.keep_scale};
+  const Plan pl = plan(x.rows, r, k_total, y ? y->rows : 0);
+  auto args = [&](const Product& q) {
+    return SkArgs{q.rows, r, k_total, pl.kps, q.out, q.out_kind, status, q.adam ? 1 : 0,
+                  q.adam ? *q.adam : AdamParams{}, q.scale, accumulate ? 1 : 0, q.drop.keep, q.drop.keep_scale};
+  };
+  const SkArgs a0 = args(x), a1 = y ? args(*y) : a0;
+  const int rt0 = static_cast<int>((x.rows + kRowsT - 1) / kRowsT);
+  const Product& yy = y ? *y : x;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = pl.grid;
   cfg.blockDim = dim3(kSkThreads);
@@ -365,7 +393,7 @@ cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows, int 
   cfg.attrs = at;
   cfg.numAttrs = 2;
   timing_before(QLORA_KERNEL_RANK_R, stream);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, skinny_tc_kernel<A_MN, B_MN>, ta, tb, a);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, skinny_tc_kernel<A_MN, B_MN>, x.ta, x.tb, yy.ta, yy.tb, a0, a1, rt0);
   timing_after(QLORA_KERNEL_RANK_R, stream);
   count_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
@@ -376,33 +404,50 @@ cudaError_t run(const CUtensorMap& ta, const CUtensorMap& tb, int64_t rows, int 
 // V = X A: Aop = X (M x in, k contiguous); Bop[j][k] = A[k][j] (j contiguous).
 cudaError_t launch_xa(const uint16_t* X, const uint16_t* A, int64_t M, int64_t n_in, int r, uint16_t* V,
                       uint32_t* status, cudaStream_t stream, float scale, Dropout drop) {
-  CUtensorMap ta, tb;
-  if (!bf16_map(&ta, X, M, n_in, 64, 128) || !bf16_map(&tb, A, n_in, r, 64, 64)) return cudaErrorInvalidValue;
-  return run<false, true>(ta, tb, M, r, n_in, V, 0, status, stream, nullptr, scale, false, drop);
+  Product x{};
+  if (!bf16_map(&x.ta, X, M, n_in, 64, 128) || !bf16_map(&x.tb, A, n_in, r, 64, 64)) return cudaErrorInvalidValue;
+  x.rows = M;
+  x.out = V;
+  x.out_kind = 0;
+  x.scale = scale;
+  x.drop = drop;
+  return run<false, true>(x, nullptr, r, n_in, status, stream, false);
 }
 
 // U = dY B^T: Aop = dY (M x out, k contiguous); Bop = B (r x out, k contiguous).
 cudaError_t launch_dybt(const uint16_t* dY, const uint16_t* B, int64_t M, int64_t n_out, int r, uint16_t* U,
                         uint32_t* status, cudaStream_t stream, float scale, Dropout drop) {
-  CUtensorMap ta, tb;
-  if (!bf16_map(&ta, dY, M, n_out, 64, 128) || !bf16_map(&tb, B, r, n_out, 64, 64)) return cudaErrorInvalidValue;
-  return run<false, false>(ta, tb, M, r, n_out, U, 0, status, stream, nullptr, scale, false, drop);
-}
-
-// dA = X^T U: Aop[i][m] = X[m][i] (i contiguous); Bop[j][m] = U[m][j] (j contiguous).
-cudaError_t launch_xtu(const uint16_t* X, const uint16_t* U, int64_t M, int64_t n_in, int r, float* dA,
-                       uint32_t* status, cudaStream_t stream, const AdamParams* adam, bool accumulate) {
-  CUtensorMap ta, tb;
-  if (!bf16_map(&ta, X, M, n_in, 64, 64) || !bf16_map(&tb, U, M, r, 64, 64)) return cudaErrorInvalidValue;
-  return run<true, true>(ta, tb, n_in, r, M, dA, 1, status, stream, adam, 1.0f, accumulate);
+  Product x{};
+  if (!bf16_map(&x.ta, dY, M, n_out, 64, 128) || !bf16_map(&x.tb, B, r, n_out, 64, 64)) return cudaErrorInvalidValue;
+  x.rows = M;
+  x.out = U;
+  x.out_kind = 0;
+  x.scale = scale;
+  x.drop = drop;
+  return run<false, false>(x, nullptr, r, n_out, status, stream, false);
 }
 
 // dB^T = dY^T V: Aop[o][m] = dY[m][o] (o contiguous); Bop[j][m] = V[m][j]; stored as dB (r x out).
-cudaError_t launch_vtdy(const uint16_t* V, const uint16_t* dY, int64_t M, int64_t n_out, int r, float* dB,
-                        uint32_t* status, cudaStream_t stream, const AdamParams* adam, bool accumulate) {
-  CUtensorMap ta, tb;
-  if (!bf16_map(&ta, dY, M, n_out, 64, 64) || !bf16_map(&tb, V, M, r, 64, 64)) return cudaErrorInvalidValue;
-  return run<true, true>(ta, tb, n_out, r, M, dB, 2, status, stream, adam, 1.0f, accumulate);
+// dA = X^T U: Aop[i][m] = X[m][i] (i contiguous); Bop[j][m] = U[m][j] (j contiguous).
+// Both reduce over the M tokens, so they share one launch: dB's row tiles first.
+cudaError_t launch_dbda(const uint16_t* V, const uint16_t* dY, const uint16_t* X, const uint16_t* U, int64_t M,
+                        int64_t n_in, int64_t n_out, int r, float* dA, float* dB, uint32_t* status,
+                        cudaStream_t stream, const AdamParams* adam_a, const AdamParams* adam_b, bool accumulate) {
+  Product b{}, a{};
+  if (!bf16_map(&b.ta, dY, M, n_out, 64, 64) || !bf16_map(&b.tb, V, M, r, 64, 64) ||
+      !bf16_map(&a.ta, X, M, n_in, 64, 64) || !bf16_map(&a.tb, U, M, r, 64, 64))
+    return cudaErrorInvalidValue;
+  b.rows = n_out;
+  b.out = dB;
+  b.out_kind = 2;
+  b.adam = adam_b;
+  b.scale = 1.0f;
+  a.rows = n_in;
+  a.out = dA;
+  a.out_kind = 1;
+  a.adam = adam_a;
+  a.scale = 1.0f;
+  return run<true, true>(b, &a, r, M, status, stream, accumulate);
 }
 
 }  // namespace qlora
