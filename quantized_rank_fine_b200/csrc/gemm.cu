@@ -265,9 +265,12 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
   // the even CTA's barriers, as seen from either CTA of the pair
   const uint32_t ready_lead = mapa_shared(ready0, 0);
   const uint32_t tmem_empty_lead = mapa_shared(tmem_empty, 0);
-  // Launched as a programmatic dependent: the set-up above overlaps the kernel
-  // before; nothing in global memory is touched until that kernel has finished.
-  grid_dependency_wait();
+  // Launched as a programmatic dependent of the rank-r kernel of the same call
+  // (V before the forward, U or dA/dB before dX).  That kernel lets this one start
+  // only after its own wait for the kernel before it, so everything this kernel
+  // reads except that kernel's output (V or U, read by the adapter steps) is
+  // final: the activations and weights stream at once, and only the adapter
+  // steps and the first global write wait for the rank-r kernel to finish.
   grid_launch_dependents();
 
   int owned_end = 0;    // > 0: this pair owns a split tile whose other parts pairs b+1 .. owned_end-1 hold
@@ -301,6 +304,7 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
             else tma_load_2d(c_dst, &tm_codes, bar, kb * (kBK / 2), nh);
           } else {
             const int j = kb - nkb_w;
+            grid_dependency_wait();   // V or U is written by the kernel before
             // the adapter's weight tile lands in the dequantised-weight region,
             // which the previous item's epilogue may still use as output staging:
             // wait for the epilogues of items 0 .. it-1, phase by phase (in order,
@@ -503,6 +507,7 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
       if (!alive) break;
 
       // ---------------------------------------------------------- epilogue of the item
+      grid_dependency_wait();   // no global write before the kernel before has finished
       if (!__all_sync(0xffffffffu, mbar_wait(tmem_full, it & 1, p.status, kFlagTimeoutEpilogue))) break;
       tc_fence_after();
       if (w.kb0 > 0) {
@@ -536,6 +541,18 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
         // the warp's 32 rows; each 32-column block goes out through shared
         // memory as one TMA store (rows and columns past the output are clipped)
         const int64_t row0 = m0 + half * kBM + kHalfN * rank + quarter * 32;
+        // The other pairs' partials of column block cb, summed in pair order; the
+        // first pair's values are only loaded here and added one block later, so
+        // their L2 round trip overlaps the previous block's store.
+        const bool merge = have && c_end > pair + 1;
+        float4 pre[8];
+        auto fetch = [&](int cb) {
+          const float4* src = reinterpret_cast<const float4*>(p.partials) +
+                              static_cast<size_t>(2 * (pair + 1) + rank) * (kSlotFloats / 4) + cb * 2048 + slot_lane;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) pre[q] = __ldcg(src + q * 32);
+        };
+        if (merge) fetch(0);
 #pragma unroll 1
         for (int cb = 0; cb < kBN / 32; ++cb) {
           uint32_t v[32];
@@ -544,8 +561,15 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
           float acc[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) acc[i] = __uint_as_float(v[i]);
-          if (have) {
-            for (int c = pair + 1; c < c_end; ++c) {
+          if (merge) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              acc[4 * q] += pre[q].x;
+              acc[4 * q + 1] += pre[q].y;
+              acc[4 * q + 2] += pre[q].z;
+              acc[4 * q + 3] += pre[q].w;
+            }
+            for (int c = pair + 2; c < c_end; ++c) {
               const float4* src = reinterpret_cast<const float4*>(p.partials) +
                                   static_cast<size_t>(2 * c + rank) * (kSlotFloats / 4) + cb * 2048 + slot_lane;
 #pragma unroll
@@ -557,6 +581,7 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
                 acc[4 * q + 3] += x.w;
               }
             }
+            if (cb + 1 < kBN / 32) fetch(cb + 1);
           }
           const int64_t col = n0 + cb * 32;
           const uint32_t buf = stage_out + static_cast<uint32_t>(cb & 1) * 2048u;

@@ -115,7 +115,10 @@ cudaError_t launch_gemv(const WeightView& w, const uint16_t* X, const uint16_t* 
 // K-steps of the last tiles are shared between CTAs: `counters` (the
 // workspace's kMaxGemmCtas counters, zero) and `partials` (one 256 x 256 fp32
 // tile per CTA, *_gemm_split_bytes) hold their hand-over.  With partials ==
-// nullptr, or fewer bytes, every tile stays whole.
+// nullptr, or fewer bytes, every tile stays whole.  Launch them only right after
+// the rank-r kernel that writes V or U (launch_xa, launch_dybt, launch_dbda):
+// they read their other inputs before that kernel has finished, which is safe
+// because it starts them only once the kernels before it have finished.
 cudaError_t launch_fwd_gemm(const WeightView& w, const uint16_t* X, const uint16_t* V, const uint16_t* B,
                             int64_t M, int r, uint16_t* Y, uint32_t* status, uint32_t* counters,
                             void* partials, size_t partial_bytes, cudaStream_t stream);
