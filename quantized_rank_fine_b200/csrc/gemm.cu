@@ -516,8 +516,7 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
 #pragma unroll 1
         for (int cb = 0; cb < kBN / 32; ++cb) {
           uint32_t v[32];
-          tmem_ld_32x32b_x32(taddr + cb * 32, v);
-          tmem_ld_wait();
+          tmem_ld_32x32b_x32(taddr + cb * 32, v);   // returns once the values are in v
           float4* dst = slot + cb * 2048 + slot_lane;
 #pragma unroll
           for (int q = 0; q < 8; ++q)
@@ -556,8 +555,7 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
 #pragma unroll 1
         for (int cb = 0; cb < kBN / 32; ++cb) {
           uint32_t v[32];
-          tmem_ld_32x32b_x32(taddr + cb * 32, v);
-          tmem_ld_wait();
+          tmem_ld_32x32b_x32(taddr + cb * 32, v);   // returns once the values are in v
           float acc[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) acc[i] = __uint_as_float(v[i]);
@@ -672,6 +670,10 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int 
 // ---------------------------------------------------------------- schedule
 
 constexpr int kMinSplitSteps = 16;    // shortest share of the split region per pair (K-steps)
+// What one more work item costs a pair, in K-steps of MMA time: the epilogue
+// drains the accumulator and the dequant warps refill the pipeline while the MMAs
+// wait (5-7 us measured, at about 0.7 us per K-step).
+constexpr int kItemCostSteps = 10;
 int g_ctas_override = 0;              // qlora_gemm_set_ctas (0: as many pairs as fit)
 
 struct GemmPlan {
@@ -737,6 +739,9 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int r, bool split_allowed) {
   if (!split_allowed || T % C == 0) return whole;
   const int waves = T / C, rest = T % C;
   if (waves == 0) {
+    // Fewer tiles than pairs: split them only if the shorter range per pair more
+    // than pays for the extra work item each pair then runs.
+    if (static_cast<int64_t>(T) * S / C + kItemCostSteps >= S) return whole;
     const int pairs = static_cast<int>(std::min<int64_t>(C, static_cast<int64_t>(T) * S / kMinSplitSteps));
     if (pairs <= T) return whole;
     return {pairs, tiles_n, 0, T};

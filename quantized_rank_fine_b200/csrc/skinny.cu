@@ -236,14 +236,16 @@ skinny_tc_kernel(const __grid_constant__ CUtensorMap tm_a0, const __grid_constan
     for (int c = 0; c < n_mma; c += 16) {
       uint32_t v[16];
       if (ok && nkb > 0) {
+        // load and wait in one statement: the registers are valid only after the wait
         asm volatile(
             "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-            "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+            "tcgen05.wait::ld.sync.aligned;"
             : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
               "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
               "=r"(v[15])
-            : "r"(taddr + c));
-        tmem_ld_wait();
+            : "r"(taddr + c)
+            : "memory");
       } else {
 #pragma unroll
         for (int i = 0; i < 16; ++i) v[i] = 0u;   // an empty slice contributes zeros

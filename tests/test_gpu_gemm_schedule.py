@@ -11,8 +11,10 @@ K-steps inside a split, ragged M.
 Each case is compared with the float64 oracle (relative Frobenius <= 1e-2,
 max-abs <= 2e-2 of max |ref|) on every output.  The full-size layers of
 test_gpu_linear run the uncapped grid: at M = 4096 the 4096 x 4096 layer has
-74 whole pair tiles and 54 split ones, and at M = 2048 (the stack) every
-4096-wide output tile is split between two pairs."""
+74 whole pair tiles and 54 split ones.  With fewer tiles than pairs the tiles are
+split only when that saves more than the extra work item costs: at M = 2048 (the
+stack) the 4096 x 4096 layers run their 64 tiles whole, the 11008-deep down
+projection splits its 64 tiles over the 74 pairs."""
 
 import pytest
 import torch
@@ -47,7 +49,7 @@ def _partials_offset(op, M, r):
 # (M, in, out, r, CTAs): the forward GEMM has N = out, K = in; dX has N = in, K = out.
 # The GEMM runs CTA pairs on 512 x 256 tiles, so CTAs / 2 pairs share the work.
 CASES = [
-    (600, 2048, 768, 24, 14),   # fwd: 6 tiles, all split over 7 pairs; dX: 7 whole tiles, then 9 split
+    (600, 2048, 768, 24, 24),   # fwd: 6 tiles, all split over 12 pairs; dX: 16 tiles, all split over 12 pairs
     (256, 4096, 256, 16, 8),    # fwd: one tile's 65 K-steps over 4 pairs (the owner adds 3 partials)
     (256, 256, 4096, 72, 8),    # dX: one tile over 4 pairs, its two adapter K-steps in the last share
     (1100, 2048, 1536, 40, 10), # fwd and dX: whole tiles, then split ones; M ragged (76 rows in the last tile)
