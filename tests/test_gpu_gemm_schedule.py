@@ -55,6 +55,8 @@ CASES = [
     (1100, 2048, 1536, 40, 10), # fwd and dX: whole tiles, then split ones; M ragged (76 rows in the last tile)
     (777, 1024, 1280, 64, 6),   # fwd: 6 whole tiles, then 4 split over 3 pairs; M ragged
     (1500, 1024, 1280, 64, 10), # dX: 5 whole tiles, then 7 split over 5 pairs; M ragged
+    (9000, 64, 128, 64, 8),     # fwd and dX: 18 whole tiles of 2 or 3 K-steps (one adapter step) over 4
+                                # pairs, four or five items a pair back to back; M ragged
 ]
 
 
