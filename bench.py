@@ -505,25 +505,37 @@ def time_weight_rows(wl, pk, want):
 
     iters = 30
     if "quantize" in want:
-        t = timed(lambda i: q.qlora_quantize_nf4(W0s[i % reps], out=ws_[i % reps]), q.KERNEL_QUANTIZE, iters)
+        qf = lambda i: q.qlora_quantize_nf4(W0s[i % reps], out=ws_[i % reps])
+        t = timed(qf, q.KERNEL_QUANTIZE, iters)
         b = n * (4 + 0.5 + 1 / 64) + 4 * math.ceil(n / 64 / 256)
-        rows["quantize"] = {"shape": [n_in, n_out], "ms": t, **hbm_fracs(b, t, pk), "bytes_per_weight": 4.516}
+        tb = graph_per_call(qf, iters)
+        bb = hbm_fracs(b, tb, pk)
+        rows["quantize"] = {"shape": [n_in, n_out], "ms": t, **hbm_fracs(b, t, pk), "bytes_per_weight": 4.516,
+                            "back_to_back": {"ms_per_call": tb, "gbs": bb["gbs"], "frac_hbm": bb["frac_hbm"],
+                                             "note": "graph of back-to-back quantisations of the rotating "
+                                                     "weights, device time per call"}}
     if "dequantize" in want:
         outs = [torch.empty((n_in, n_out), dtype=torch.bfloat16, device="cuda") for _ in range(reps)]
-        t = timed(lambda i: q.qlora_dequantize(ws_[i % reps], torch.bfloat16, out=outs[i % reps]),
-                  q.KERNEL_DEQUANTIZE, iters)
+        df = lambda i: q.qlora_dequantize(ws_[i % reps], torch.bfloat16, out=outs[i % reps])
+        t = timed(df, q.KERNEL_DEQUANTIZE, iters)
         b = n * (0.5 + 1 / 64 + 2) + 4 * math.ceil(n / 64 / 256)
-        rows["dequantize_bf16"] = {"shape": [n_in, n_out], "ms": t, **hbm_fracs(b, t, pk)}
+        tb = graph_per_call(df, iters)
+        bb = hbm_fracs(b, tb, pk)
+        rows["dequantize_bf16"] = {"shape": [n_in, n_out], "ms": t, **hbm_fracs(b, t, pk),
+                                   "back_to_back": {"ms_per_call": tb, "gbs": bb["gbs"], "frac_hbm": bb["frac_hbm"]}}
         del outs
     if "merge" in want:
         r = wl["r"]
         A = synth.normal("rowsA", (n_in, r), 1 / math.sqrt(n_in), torch.bfloat16, "cuda")
         B = synth.normal("rowsB", (r, n_out), 0.01, torch.bfloat16, "cuda")
         outs32 = [torch.empty((n_in, n_out), dtype=torch.float32, device="cuda") for _ in range(reps)]
-        t = timed(lambda i: q.qlora_merge(ws_[i % reps], A, B, torch.float32, out=outs32[i % reps]),
-                  q.KERNEL_MERGE, iters)
+        mf = lambda i: q.qlora_merge(ws_[i % reps], A, B, torch.float32, out=outs32[i % reps])
+        t = timed(mf, q.KERNEL_MERGE, iters)
         b = n * (0.5 + 1 / 64 + 4) + 2 * r * (n_in + n_out)
-        rows["merge_f32"] = {"shape": [n_in, n_out], "r": r, "ms": t, **hbm_fracs(b, t, pk)}
+        tb = graph_per_call(mf, iters)
+        bb = hbm_fracs(b, tb, pk)
+        rows["merge_f32"] = {"shape": [n_in, n_out], "r": r, "ms": t, **hbm_fracs(b, t, pk),
+                             "back_to_back": {"ms_per_call": tb, "gbs": bb["gbs"], "frac_hbm": bb["frac_hbm"]}}
         del outs32
     del W0s, ws_
     torch.cuda.synchronize()
@@ -713,6 +725,37 @@ def time_train_step(wl):
         raise RuntimeError("a kernel wait timed out in the training-step row")
     out["adam_overhead_ms"] = out["fwd_bwd_adam"]["ms_per_step"] - out["fwd_bwd"]["ms_per_step"]
     return out
+
+
+def graph_per_call(fn, iters):
+    """Device time (ms) per call of a CUDA graph of `iters` back-to-back calls of
+    fn(i): the throughput of a sequence of launches, where each kernel's set-up
+    overlaps the one before (programmatic dependent launch)."""
+    import torch
+    for i in range(3):
+        fn(i)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side, capture_error_mode="relaxed"):
+            for i in range(iters):
+                fn(i)
+    torch.cuda.current_stream().wait_stream(side)
+    graph.replay()
+    torch.cuda.synchronize()
+    best = None
+    for _ in range(3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        t = e0.elapsed_time(e1) / iters
+        best = t if best is None else min(best, t)
+    del graph
+    return best
 
 
 def graph_timed(fn, which, iters):
