@@ -128,9 +128,9 @@ nf4_gemv_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;                                                  // kGvStages x (codes, X)
   uint8_t* lut = smem + kGvStages * kStageBytes;                         // [256][32] x 4 bytes
-  float* aslice = reinterpret_cast<float*>(lut + kLutBytes);             // [8 warps][32] absmax'
+  float* aslice = reinterpret_cast<float*>(lut + kLutBytes);             // [8 warps][2][32] absmax'
   float* part = reinterpret_cast<float*>(ring);                          // [M][256] after the loop
-  float* recv = aslice + kGvConsumers * 32;                              // [S][cap] float4
+  float* recv = aslice + kGvConsumers * 64;                              // [S][cap] float4
   __shared__ __align__(8) uint64_t bars[2 * kGvStages];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -224,13 +224,58 @@ nf4_gemv_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
       }
     };
     const uint32_t lut_lane = smem_addr(lut) + lane * 4;
-    float* asl = aslice + warp * 32;
+    float* asl = aslice + warp * 64;   // two slices: the stages of a pair
     constexpr uint32_t kLo = 0x0F0F0F0Fu;
     // 16, 2^28 and 128 as run-time values (p.M < 2^16): multiplies by them stay
     // multiply-adds on the FMA pipe rather than shifts on the integer pipe
     const uint32_t k16 = 16u | (static_cast<uint32_t>(p.M) >> 16);
     const uint32_t k2p28 = (1u << 28) | (static_cast<uint32_t>(p.M) >> 16);
     const uint32_t k128 = 128u | (static_cast<uint32_t>(p.M) >> 16);
+
+    // One 16-row step (h = 0, 1 of this warp's row half) of the weight stage at
+    // ctile, with the absmax' slice asl_s of that stage.
+    auto hstep = [&](const uint8_t* ctile, const float* asl_s, int h) {
+      const uint8_t* xtile = ctile + kCodeBytes;
+      const int r0 = half * 32 + h * 16;   // first row of the 16-row step within the stage
+      const int kb = cg * 32 + 4 * g;      // byte of this lane's 8 columns within the row
+      const uint32_t c0 = ld_sw128(ctile, r0 + 2 * t, kb);
+      const uint32_t c1 = ld_sw128(ctile, r0 + 2 * t + 1, kb);
+      const uint32_t c2 = ld_sw128(ctile, r0 + 2 * t + 8, kb);
+      const uint32_t c3 = ld_sw128(ctile, r0 + 2 * t + 9, kb);
+      // byte j: (row k code, row k+1 code) of column 8g+2j (even) or 8g+2j+1 (odd);
+      // c * 16 = c << 4 and umulhi(c, 2^28) = c >> 4
+      const uint32_t e01 = (c0 & kLo) | ((c1 * k16) & ~kLo);
+      const uint32_t o01 = (__umulhi(c0, k2p28) & kLo) | (c1 & ~kLo);
+      const uint32_t e89 = (c2 & kLo) | ((c3 * k16) & ~kLo);
+      const uint32_t o89 = (__umulhi(c2, k2p28) & kLo) | (c3 & ~kLo);
+      // x' fragment: token a*8+g, k slots (2t, 2t+1) and (2t+8, 2t+9)
+      const float2 s01 = *reinterpret_cast<const float2*>(asl_s + h * 16 + 2 * t);
+      const float2 s89 = *reinterpret_cast<const float2*>(asl_s + h * 16 + 2 * t + 8);
+      uint32_t bx[MT][2];
+#pragma unroll
+      for (int a = 0; a < MT; ++a) {
+        const int m = a * 8 + g;
+        bx[a][0] = 0u;
+        bx[a][1] = 0u;
+        if (m < p.M) {
+          const uint32_t x01 = ld_sw128(xtile, m, 2 * (r0 + 2 * t));
+          const uint32_t x89 = ld_sw128(xtile, m, 2 * (r0 + 2 * t + 8));
+          bx[a][0] = pack_bf16x2(mul_rn(bf16_lo(x01), s01.x), mul_rn(bf16_hi(x01), s01.y));
+          bx[a][1] = pack_bf16x2(mul_rn(bf16_lo(x89), s89.x), mul_rn(bf16_hi(x89), s89.y));
+        }
+      }
+      auto tile_j = [&](auto jc) {
+        constexpr int j = decltype(jc)::value;
+        const uint32_t a0 = lut_pair<j>(lut_lane, e01, k128), a1 = lut_pair<j>(lut_lane, o01, k128);
+        const uint32_t a2 = lut_pair<j>(lut_lane, e89, k128), a3 = lut_pair<j>(lut_lane, o89, k128);
+#pragma unroll
+        for (int a = 0; a < MT; ++a) mma_bf16_16816(acc[a][j], a0, a1, a2, a3, bx[a][0], bx[a][1]);
+      };
+      tile_j(std::integral_constant<int, 0>{});
+      tile_j(std::integral_constant<int, 1>{});
+      tile_j(std::integral_constant<int, 2>{});
+      tile_j(std::integral_constant<int, 3>{});
+    };
 
     // One stage; (qc, qs) hold its absmax code and scale and are reloaded with
     // those of stage i + 2 once used.  False if the wait for the stage timed out.
@@ -273,62 +318,49 @@ nf4_gemv_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
         return true;
       }
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int r0 = half * 32 + h * 16;   // first row of the 16-row step within the stage
-        const int kb = cg * 32 + 4 * g;      // byte of this lane's 8 columns within the row
-        const uint32_t c0 = ld_sw128(ctile, r0 + 2 * t, kb);
-        const uint32_t c1 = ld_sw128(ctile, r0 + 2 * t + 1, kb);
-        const uint32_t c2 = ld_sw128(ctile, r0 + 2 * t + 8, kb);
-        const uint32_t c3 = ld_sw128(ctile, r0 + 2 * t + 9, kb);
-        // byte j: (row k code, row k+1 code) of column 8g+2j (even) or 8g+2j+1 (odd);
-        // c * 16 = c << 4 and umulhi(c, 2^28) = c >> 4
-        const uint32_t e01 = (c0 & kLo) | ((c1 * k16) & ~kLo);
-        const uint32_t o01 = (__umulhi(c0, k2p28) & kLo) | (c1 & ~kLo);
-        const uint32_t e89 = (c2 & kLo) | ((c3 * k16) & ~kLo);
-        const uint32_t o89 = (__umulhi(c2, k2p28) & kLo) | (c3 & ~kLo);
-        // x' fragment: token a*8+g, k slots (2t, 2t+1) and (2t+8, 2t+9)
-        const float2 s01 = *reinterpret_cast<const float2*>(asl + h * 16 + 2 * t);
-        const float2 s89 = *reinterpret_cast<const float2*>(asl + h * 16 + 2 * t + 8);
-        uint32_t bx[MT][2];
-#pragma unroll
-        for (int a = 0; a < MT; ++a) {
-          const int m = a * 8 + g;
-          bx[a][0] = 0u;
-          bx[a][1] = 0u;
-          if (m < p.M) {
-            const uint32_t x01 = ld_sw128(xtile, m, 2 * (r0 + 2 * t));
-            const uint32_t x89 = ld_sw128(xtile, m, 2 * (r0 + 2 * t + 8));
-            bx[a][0] = pack_bf16x2(mul_rn(bf16_lo(x01), s01.x), mul_rn(bf16_hi(x01), s01.y));
-            bx[a][1] = pack_bf16x2(mul_rn(bf16_lo(x89), s89.x), mul_rn(bf16_hi(x89), s89.y));
-          }
-        }
-        auto tile_j = [&](auto jc) {
-          constexpr int j = decltype(jc)::value;
-          const uint32_t a0 = lut_pair<j>(lut_lane, e01, k128), a1 = lut_pair<j>(lut_lane, o01, k128);
-          const uint32_t a2 = lut_pair<j>(lut_lane, e89, k128), a3 = lut_pair<j>(lut_lane, o89, k128);
-#pragma unroll
-          for (int a = 0; a < MT; ++a) mma_bf16_16816(acc[a][j], a0, a1, a2, a3, bx[a][0], bx[a][1]);
-        };
-        tile_j(std::integral_constant<int, 0>{});
-        tile_j(std::integral_constant<int, 1>{});
-        tile_j(std::integral_constant<int, 2>{});
-        tile_j(std::integral_constant<int, 3>{});
-      }
+      for (int h = 0; h < 2; ++h) hstep(ctile, asl, h);
       __syncwarp();   // every lane is done with this stage and with the absmax' slice
       if (lane == 0) mbar_arrive(empty0 + 8 * s);
       return true;
     };
-
-    // two register sets, so that no load result is moved before it is used
+    // Two weight stages at once: both waits first, then the four 16-row steps in
+    // one stretch of code, so that the table lookups and products of both stages
+    // overlap.  (qa, sa) and (qb, sb) hold the absmax data of stages i and i + 1.
     uint32_t qa, qb;
     float sa, sb;
+    auto stage2 = [&](int i) -> bool {
+      const int s0 = i % kGvStages, s1 = (i + 1) % kGvStages;
+      asl[lane] = absmax_deq(static_cast<uint8_t>(qa), sa, p.dq_u8 != 0);
+      asl[32 + lane] = absmax_deq(static_cast<uint8_t>(qb), sb, p.dq_u8 != 0);
+      load_scale(i + 2, qa, sa);
+      load_scale(i + 3, qb, sb);
+      __syncwarp();   // both slices are complete
+      const bool got = mbar_wait(full0 + 8 * s0, (i / kGvStages) & 1, p.status, kFlagTimeoutMma) &&
+                       mbar_wait(full0 + 8 * s1, ((i + 1) / kGvStages) & 1, p.status, kFlagTimeoutMma);
+      if (!__all_sync(0xffffffffu, got)) return false;
+      const uint8_t* t0 = ring + s0 * kStageBytes;
+      const uint8_t* t1 = ring + s1 * kStageBytes;
+      hstep(t0, asl, 0);
+      hstep(t0, asl, 1);
+      hstep(t1, asl + 32, 0);
+      hstep(t1, asl + 32, 1);
+      __syncwarp();   // every lane is done with both stages and both slices
+      if (lane == 0) {
+        mbar_arrive(empty0 + 8 * s0);
+        mbar_arrive(empty0 + 8 * s1);
+      }
+      return true;
+    };
+
+    // two register sets, so that no load result is moved before it is used
     load_scale(0, qa, sa);
     load_scale(1, qb, sb);
     named_barrier_sync(1, kGvConsumers * 32);   // level table complete
-    for (int i = 0; i < nall; i += 2) {
-      if (!stage(i, qa, sa)) break;
-      if (i + 1 < nall && !stage(i + 1, qb, sb)) break;
-    }
+    int i = 0;
+    for (; i + 1 < nstage; i += 2)
+      if (!stage2(i)) break;
+    // an odd last weight stage, then the adapter stages, one at a time
+    for (bool ok = i + 1 >= nstage; ok && i < nall; ++i) ok = stage(i, (i & 1) ? qb : qa, (i & 1) ? sb : sa);
   }
   __syncthreads();   // ring no longer read or written: it becomes the partial buffer
 
@@ -393,7 +425,7 @@ nf4_gemv_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
 }
 
 // + 1 KB to align the ring to the swizzle atom
-constexpr size_t kGvSmemBytes = 1024 + kGvStages * kStageBytes + kLutBytes + kGvConsumers * 32 * 4 + kRecvBytes;
+constexpr size_t kGvSmemBytes = 1024 + kGvStages * kStageBytes + kLutBytes + kGvConsumers * 64 * 4 + kRecvBytes;
 
 // Clusters of each size (1 .. kMaxCluster CTAs) that can be resident at once,
 // queried once per device (the kernels' attributes are set on the way); all
