@@ -24,8 +24,11 @@
 //     sum_k (x_k a'_k) l_k.  The B fragment is x'[m][k] = bf16(x[m][k] * a'(k, block)),
 //     built in registers from the X tile and the block's absmax'; the weight
 //     operand is the bf16 NF4 level itself.  Each lane computes a' of one row of
-//     its warp's block per stage from an absmax code and scale it loaded three
+//     its warp's block per stage from an absmax code and scale it loaded two
 //     stages earlier, so nothing runs before the first stage but the level table.
+//   * A consumer warp takes the weight stages two at a time: it waits for both,
+//     then runs their four 16-row steps as one stretch of code, so the table
+//     lookups and products of the two stages overlap.
 //   * The adapter term V B rides on the same MMAs as r extra k rows of the last
 //     K-split, [X | V] [deq(Wq); B]: its producer loads, per 16 adapter rows, the
 //     tile's 16 x 256 block of B (TMA, 128-byte swizzle) and the 16 matching
