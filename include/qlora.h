@@ -140,6 +140,36 @@ QLORA_API qlora_status qlora_quantize_nf4_ex(const float* W0, int64_t in, int64_
                                              uint8_t* dq_codes, float* dq_scales, int dq_format, void* stream);
 
 /*
+ * One weight of a batch quantisation: W0 [device] fp32 (in, out) and its outputs,
+ * as in qlora_quantize_nf4.
+ */
+typedef struct qlora_quantize_job {
+  const float* W0;
+  int64_t in;
+  int64_t out;
+  uint8_t* codes;
+  uint8_t* dq_codes;
+  float* dq_scales;
+} qlora_quantize_job;
+
+/*
+ * qlora_quantize_nf4_ex for n weights (a model's linears quantised in one pass):
+ * the same codes, absmax codes and scales, bit for bit, as n separate calls.  Up
+ * to 32 weights share one launch, whose persistent grid runs through all of their
+ * groups in one sequence, so the weights do not each end with a partly idle wave.
+ *   jobs  [host] n descriptors (read during the call only); every job must meet
+ *         qlora_quantize_nf4's requirements.
+ * QLORA_ERR_INVALID_ARG for n < 0, a NULL jobs array with n > 0, a NULL pointer
+ * in a job or an unknown dq_format; QLORA_ERR_SHAPE for a job's bad shape: these
+ * are checked for every job before anything is launched.  Whether each pointer
+ * is 16-byte aligned device memory of the current device is checked for the 32
+ * jobs of a launch just before that launch (QLORA_ERR_INVALID_ARG or
+ * QLORA_ERR_ALIGNMENT; the launches before it stay issued).  n = 0 does nothing.
+ */
+QLORA_API qlora_status qlora_quantize_nf4_batch(const qlora_quantize_job* jobs, int n, int dq_format,
+                                                void* stream);
+
+/*
  * The second base quantiser, of the pages' simulation ("QLoRA (low-rank adapters
  * on a quantized model)", "The code, line by line": symmetric uniform integers,
  * one scale per 16 consecutive entries of the flattened (in, out) matrix; no NF4

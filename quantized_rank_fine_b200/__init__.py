@@ -39,7 +39,7 @@ EXPORTS = (
     "qlora_linear_fwd_static_ws", "qlora_linear_bwd_adam", "qlora_linear_fwd_ex", "qlora_linear_bwd_ex",
     "qlora_gemm_set_ctas", "qlora_quantize_nf4_ex", "qlora_quantize_int", "qlora_dequantize_int",
     "qlora_static_ws_status", "qlora_quantize_status", "qlora_selftest_wait_timeout",
-    "qlora_loftq_residual", "qlora_loftq_split",
+    "qlora_loftq_residual", "qlora_loftq_split", "qlora_quantize_nf4_batch",
 )
 
 # Weight formats (NF4Weight.dq_format): NF4 with E4M3 or linear uint8 absmax
@@ -63,6 +63,11 @@ class QLoRAError(RuntimeError):
 class _Weight(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("dq_codes", ctypes.c_void_p), ("dq_scales", ctypes.c_void_p),
                 ("in_", ctypes.c_int64), ("out", ctypes.c_int64), ("dq_format", ctypes.c_int32)]
+
+
+class _QuantizeJob(ctypes.Structure):
+    _fields_ = [("W0", ctypes.c_void_p), ("in_", ctypes.c_int64), ("out", ctypes.c_int64),
+                ("codes", ctypes.c_void_p), ("dq_codes", ctypes.c_void_p), ("dq_scales", ctypes.c_void_p)]
 
 
 class _AdamHparams(ctypes.Structure):
@@ -107,6 +112,7 @@ def lib() -> ctypes.CDLL:
             "qlora_launch_count": (ctypes.c_uint64, []),
             "qlora_gemm_set_ctas": (i32, [i32]),
             "qlora_quantize_nf4_ex": (i32, [vp, i64, i64, vp, vp, vp, i32, vp]),
+            "qlora_quantize_nf4_batch": (i32, [ctypes.POINTER(_QuantizeJob), i32, i32, vp]),
             "qlora_quantize_int": (i32, [vp, i64, i64, i32, vp, vp, vp]),
             "qlora_dequantize_int": (i32, [vp, vp, i64, i64, vp, i32, vp]),
             "qlora_linear_fwd_static_ws": (i32, [wp, vp, i64, vp, vp, i32, vp, vp, vp]),
@@ -259,6 +265,28 @@ def qlora_quantize_nf4(W0: torch.Tensor, stream=None, out: NF4Weight | None = No
                                            _ptr(out.dq_scales), out.dq_format, _stream(stream)),
                "qlora_quantize_nf4_ex")
     return out
+
+
+def qlora_quantize_nf4_batch(W0s, stream=None, outs=None, dq_format: int = QLORA_DQ_E4M3) -> list:
+    """Several fp32 (in, out) weights on the GPU -> one NF4Weight each, in as few
+    launches as the library needs (qlora_quantize_nf4_batch); the same bytes as
+    quantising them one by one."""
+    if outs is None:
+        outs = []
+        for W0 in W0s:
+            n_in, n_out = W0.shape
+            n, dev = n_in * n_out, W0.device
+            outs.append(NF4Weight(torch.empty(n // 2, dtype=torch.uint8, device=dev),
+                                  torch.empty(n // BLOCK, dtype=torch.uint8, device=dev),
+                                  torch.empty((n // BLOCK + GROUP - 1) // GROUP, dtype=torch.float32, device=dev),
+                                  n_in, n_out))
+    jobs = (_QuantizeJob * max(1, len(W0s)))()
+    for i, (W0, o) in enumerate(zip(W0s, outs)):
+        o.dq_format = dq_format
+        jobs[i] = _QuantizeJob(_ptr(W0), W0.shape[0], W0.shape[1], _ptr(o.codes), _ptr(o.dq_codes),
+                               _ptr(o.dq_scales))
+    _check(lib().qlora_quantize_nf4_batch(jobs, len(W0s), dq_format, _stream(stream)), "qlora_quantize_nf4_batch")
+    return outs
 
 
 def qlora_quantize_status(stream=None) -> int:

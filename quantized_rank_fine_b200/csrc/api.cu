@@ -2,7 +2,9 @@
 // Declarations, argument meaning, layouts and error behaviour: include/qlora.h.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
+#include <vector>
 #include <string.h>
 
 #include <atomic>
@@ -287,6 +289,37 @@ qlora_status qlora_quantize_nf4_ex(const float* W0, int64_t in, int64_t out, uin
   QLORA_TRY(check_ptr(dq_scales));
   QLORA_CUDA(qlora::launch_quantize_nf4(W0, in * out, codes, dq_codes, dq_scales, static_cast<cudaStream_t>(stream),
                                         dq_format == QLORA_DQ_U8));
+  return QLORA_OK;
+}
+
+qlora_status qlora_quantize_nf4_batch(const qlora_quantize_job* jobs, int n, int dq_format, void* stream) {
+  if (n < 0 || (n > 0 && !jobs)) return QLORA_ERR_INVALID_ARG;
+  if (dq_format != QLORA_DQ_E4M3 && dq_format != QLORA_DQ_U8) return QLORA_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    const qlora_quantize_job& j = jobs[i];
+    if (!j.W0 || !j.codes || !j.dq_codes || !j.dq_scales) return QLORA_ERR_INVALID_ARG;
+    if (j.in < 1 || j.out < 1 || j.in > (int64_t(1) << 40) / j.out || (j.in * j.out) % QLORA_BLOCK != 0)
+      return QLORA_ERR_SHAPE;
+  }
+  if (n == 0) return QLORA_OK;
+  QLORA_TRY(check_device());
+  // The pointers of each launch's weights are checked just before that launch, so
+  // that the host checks of the next ones overlap the device work (a pointer
+  // error stops the batch there: the launches before it have been issued).
+  std::vector<qlora::QuantizeJob> q(static_cast<size_t>(n));
+  for (int c = 0; c < n; c += qlora::kQMaxJobs) {
+    const int cn = std::min(qlora::kQMaxJobs, n - c);
+    for (int i = c; i < c + cn; ++i) {
+      const qlora_quantize_job& j = jobs[i];
+      QLORA_TRY(check_ptr(j.W0));
+      QLORA_TRY(check_ptr(j.codes));
+      QLORA_TRY(check_ptr(j.dq_codes));
+      QLORA_TRY(check_ptr(j.dq_scales));
+      q[i] = qlora::QuantizeJob{j.W0, j.in * j.out, j.codes, j.dq_codes, j.dq_scales};
+    }
+    QLORA_CUDA(qlora::launch_quantize_nf4_batch(q.data() + c, cn, static_cast<cudaStream_t>(stream),
+                                                dq_format == QLORA_DQ_U8));
+  }
   return QLORA_OK;
 }
 

@@ -582,8 +582,13 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
             if (cb + 1 < kBN / 32) fetch(cb + 1);
           }
           const int64_t col = n0 + cb * 32;
+          // Only blocks that are stored touch the staging buffers, so that every
+          // write to a buffer follows the commit of the store that last read it
+          // (the blocks past the output's last column or row are a suffix of the
+          // warp's blocks and are skipped whole).
+          if (row0 >= p.M || col >= p.N) continue;
           const uint32_t buf = stage_out + static_cast<uint32_t>(cb & 1) * 2048u;
-          // the store issued from this block two rounds ago has read it
+          // the store issued from this buffer two blocks ago has read it
           if (lane == 0 && cb >= 2) bulk_wait_read<1>();
           __syncwarp();
           // row `lane` of the block, 64 bytes as four 16-byte chunks, chunk c at
@@ -595,7 +600,7 @@ nf4_gemm_kernel(const __grid_constant__ CUtensorMap tm_act, const __grid_constan
                          pack_bf16x2(acc[8 * q + 6], acc[8 * q + 7]));
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0 && row0 < p.M && col < p.N) {
+          if (lane == 0) {
             tma_store_2d(&tm_out, buf, static_cast<int32_t>(col), static_cast<int32_t>(row0));
             bulk_commit();
           }

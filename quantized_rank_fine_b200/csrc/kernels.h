@@ -44,6 +44,17 @@ constexpr int kFmtE4M3 = 0, kFmtU8 = 1, kFmtInt16 = 2;
 // dq_u8 / u8: the absmax codes are linear uint8 (s = max / 255) instead of E4M3.
 cudaError_t launch_quantize_nf4(const float* W0, int64_t n, uint8_t* codes, uint8_t* dq_codes,
                                 float* dq_scales, cudaStream_t stream, bool dq_u8 = false);
+// Several weights (n weights each, a multiple of 64): up to kQMaxJobs per launch,
+// whose groups the persistent grid walks as one sequence.
+constexpr int kQMaxJobs = 32;
+struct QuantizeJob {
+  const float* W0;
+  int64_t n;
+  uint8_t* codes;
+  uint8_t* dq_codes;
+  float* dq_scales;
+};
+cudaError_t launch_quantize_nf4_batch(const QuantizeJob* jobs, int n, cudaStream_t stream, bool dq_u8 = false);
 // With W0 != nullptr the output is the fp32 residual fl32(W0 - w') instead (bf16 ignored).
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* dq_codes, const float* dq_scales,
                               int64_t n, bool bf16, void* out, cudaStream_t stream, int fmt = kFmtE4M3,

@@ -11,6 +11,9 @@
 //
 // Layout: a persistent grid of two 256-thread CTAs per SM walks the groups
 // (16,384 weights = 64 KB of fp32 each), every group as two halves of 128 blocks.
+// One launch can take several weights (a batch of up to kQMaxJobs): their groups
+// are numbered one after the other, so the CTAs run through all of them without a
+// tail per weight.
 // A bulk asynchronous copy streams each half-group into one of three 32 KB
 // shared-memory buffers, two halves ahead of the one being encoded, so HBM is
 // read continuously with no thread involvement.  Warp w owns blocks 16w .. 16w+15
@@ -85,23 +88,51 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
                : "memory");
 }
 
-// Work item j of this CTA: half (j & 1) of its group number j >> 1.
-__device__ __forceinline__ void issue_half(int64_t j, const float* W0, int64_t nblocks, int64_t ngroups,
-                                           uint32_t buf0, uint32_t bar0) {
-  const int64_t g = blockIdx.x + (j >> 1) * gridDim.x;
-  if (g >= ngroups) return;
-  const int64_t blk = g * kGroup + (j & 1) * kHalfBlocks;
-  if (blk >= nblocks) return;
-  const int64_t nb = min(static_cast<int64_t>(kHalfBlocks), nblocks - blk);
-  const uint32_t bytes = static_cast<uint32_t>(nb * kBlock * 4);
-  const int b = static_cast<int>(j % kQBuf);
-  sm100::mbar_arrive_expect_tx(bar0 + 8 * b, bytes);
-  bulk_load(buf0 + b * kHalfBytes, W0 + blk * kBlock, bytes, bar0 + 8 * b);
+// The weights of one launch.  Group gg of the launch is group gg - group0[j] of
+// weight j, for the j with group0[j] <= gg < group0[j + 1].
+// NJ is the capacity: 1 for a single weight (a small parameter block, so that a
+// launch per weight costs no more than before), kQMaxJobs for a batch.
+template <int NJ>
+struct QJobs {
+  int n;
+  int64_t group0[NJ + 1];
+  int64_t nblocks[NJ];
+  const float* W0[NJ];
+  uint8_t* codes[NJ];
+  uint8_t* dq_codes[NJ];
+  float* dq_scales[NJ];
+};
+
+// The weight of group gg, searched upward from `j` (a CTA's groups only increase,
+// so each search starts where the previous one ended).
+template <int NJ>
+__device__ __forceinline__ int job_of(const QJobs<NJ>& q, int64_t gg, int j = 0) {
+  while (j + 1 < q.n && q.group0[j + 1] <= gg) ++j;
+  return j;
 }
 
+// Work item i of this CTA: half (i & 1) of its group number i >> 1.  `jc` is the
+// weight of the item issued before (items are issued in increasing order).
+template <int NJ>
+__device__ __forceinline__ void issue_half(int64_t i, const QJobs<NJ>& q, uint32_t buf0, uint32_t bar0, int& jc) {
+  const int64_t gg = blockIdx.x + (i >> 1) * gridDim.x;
+  if (gg >= q.group0[q.n]) return;
+  const int j = jc = job_of(q, gg, jc);
+  const int64_t blk = (gg - q.group0[j]) * kGroup + (i & 1) * kHalfBlocks;
+  const int b = static_cast<int>(i % kQBuf);
+  if (blk >= q.nblocks[j]) {   // the empty second half of a short group: complete the phase
+    sm100::mbar_arrive(bar0 + 8 * b);
+    return;
+  }
+  const int64_t nb = min(static_cast<int64_t>(kHalfBlocks), q.nblocks[j] - blk);
+  const uint32_t bytes = static_cast<uint32_t>(nb * kBlock * 4);
+  sm100::mbar_arrive_expect_tx(bar0 + 8 * b, bytes);
+  bulk_load(buf0 + b * kHalfBytes, q.W0[j] + blk * kBlock, bytes, bar0 + 8 * b);
+}
+
+template <int NJ>
 __global__ void __launch_bounds__(kQThreads, 2)
-quantize_nf4_kernel(const float* __restrict__ W0, int64_t nblocks, int64_t ngroups, uint8_t* __restrict__ codes,
-                    uint8_t* __restrict__ dq_codes, float* __restrict__ dq_scales, bool dq_u8) {
+quantize_nf4_kernel(const __grid_constant__ QJobs<NJ> q, bool dq_u8) {
   extern __shared__ __align__(128) uint8_t qsmem[];
   __shared__ uint32_t lut[kCells];
   __shared__ float thr_exact[16];
@@ -125,13 +156,14 @@ quantize_nf4_kernel(const float* __restrict__ W0, int64_t nblocks, int64_t ngrou
     lut[tid] = (__float_as_uint(thr) & ~0xFu) | base;
   }
   if (tid < 16) thr_exact[tid] = tid < 15 ? c_nf4_threshold[tid] : 2.0f;
+  int jissue = 0, jgroup = 0;   // the weights of the last copy issued (thread 0) and of the current group
   if (tid == 0) {
     for (int b = 0; b < kQBuf; ++b) sm100::mbar_init(bar0 + 8 * b, 1);
     sm100::fence_mbar_init();
     // W0 may be written by the kernel this one follows (programmatic dependent
     // launch): the set-up above overlaps its tail, the copies wait for it
     sm100::grid_dependency_wait();
-    for (int j = 0; j < kQBuf; ++j) issue_half(j, W0, nblocks, ngroups, buf0, bar0);
+    for (int j = 0; j < kQBuf; ++j) issue_half(j, q, buf0, bar0, jissue);
   }
   __syncthreads();
   // the outputs are written only after the kernel before has completed
@@ -142,11 +174,22 @@ quantize_nf4_kernel(const float* __restrict__ W0, int64_t nblocks, int64_t ngrou
   // rotated chunk order: the 8 lanes of a quarter-warp read 8 different 16-byte bank groups
   const int rot = (quarter >> 1) + 2 * (bsub & 1);
   int64_t j = 0, failed_at = -1;
-  for (int64_t g = blockIdx.x; g < ngroups; g += gridDim.x) {
+  const int64_t ngroups = q.group0[q.n];
+  for (int64_t gg = blockIdx.x; gg < ngroups; gg += gridDim.x) {
+    // group g of weight jb
+    const int jb = jgroup = job_of(q, gg, jgroup);
+    const int64_t g = gg - q.group0[jb];
     const int64_t blk0 = g * kGroup;
-    const int nblk = static_cast<int>(nblocks - blk0 < kGroup ? nblocks - blk0 : kGroup);
+    const int nblk = static_cast<int>(q.nblocks[jb] - blk0 < kGroup ? q.nblocks[jb] - blk0 : kGroup);
+    uint8_t* __restrict__ codes = q.codes[jb];
+    uint8_t* __restrict__ dq_codes = q.dq_codes[jb];
+    float* __restrict__ dq_scales = q.dq_scales[jb];
+    // Every group is two work items.  The second half of a short group (a weight's
+    // last) is empty: its barrier phase completes without a copy and nothing is
+    // encoded, so the item numbering of the copies and of this loop stay in step
+    // across the weights of the launch.
     for (int h = 0; h < 2; ++h, ++j) {
-      if (h * kHalfBlocks >= nblk) break;          // a short last group
+      const bool empty = h * kHalfBlocks >= nblk;
       const int b = static_cast<int>(j % kQBuf);
       const uint32_t ph = static_cast<uint32_t>((j / kQBuf) & 1);
       const bool got = sm100::mbar_wait(bar0 + 8 * b, ph, &g_quantize_status, kFlagTimeoutProducer);
@@ -155,56 +198,58 @@ quantize_nf4_kernel(const float* __restrict__ W0, int64_t nblocks, int64_t ngrou
         break;
       }
       const float* gs = reinterpret_cast<const float*>(qsmem + b * kHalfBytes);
+      if (!empty) {
 #pragma unroll
-      for (int it = 0; it < 2; ++it) {
-        const int hb = warp * 16 + it * 8 + bsub;     // block within the half
-        const int lb = h * kHalfBlocks + hb;          // block within the group
-        float4 v[4];
-        int ci[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          ci[c] = (c + rot) & 3;
-          v[c] = (lb < nblk) ? *reinterpret_cast<const float4*>(gs + hb * kBlock + quarter * 16 + 4 * ci[c])
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        float m = 0.0f;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          m = fmaxf(m, fmaxf(fmaxf(fabsf(v[c].x), fabsf(v[c].y)), fmaxf(fabsf(v[c].z), fabsf(v[c].w))));
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-        if (lb < nblk) {
-          float rcp = (m > 0.0f) ? __frcp_rn(m) : 0.0f;
-          const bool exact_all = !(rcp <= 3.0e38f);   // a subnormal absmax: exact path only
-          if (exact_all) rcp = 0.0f;
-          uint64_t word = 0;
-          uint32_t near_chunks = 0;                   // bit ci: that chunk may sit across a threshold
-#pragma unroll
+        for (int it = 0; it < 2; ++it) {
+          const int hb = warp * 16 + it * 8 + bsub;     // block within the half
+          const int lb = h * kHalfBlocks + hb;          // block within the group
+          float4 v[4];
+          int ci[4];
+  #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            bool nr = exact_all;
-            const uint32_t c4 = fast_code(__fmul_rn(v[c].x, rcp), lut, nr) |
-                                (fast_code(__fmul_rn(v[c].y, rcp), lut, nr) << 4) |
-                                (fast_code(__fmul_rn(v[c].z, rcp), lut, nr) << 8) |
-                                (fast_code(__fmul_rn(v[c].w, rcp), lut, nr) << 12);
-            word |= static_cast<uint64_t>(c4) << (16 * ci[c]);
-            near_chunks |= (nr ? 1u : 0u) << ci[c];
+            ci[c] = (c + rot) & 3;
+            v[c] = (lb < nblk) ? *reinterpret_cast<const float4*>(gs + hb * kBlock + quarter * 16 + 4 * ci[c])
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
           }
-          // redo (rarely) the chunks with a quotient that may sit across its threshold
-          while (near_chunks) {
-            const int cc = __ffs(near_chunks) - 1;
-            near_chunks &= near_chunks - 1;
-            const float4 w4 = *reinterpret_cast<const float4*>(gs + hb * kBlock + quarter * 16 + 4 * cc);
-            const uint32_t c4 = exact_code(w4.x, m, thr_exact) | (exact_code(w4.y, m, thr_exact) << 4) |
-                                (exact_code(w4.z, m, thr_exact) << 8) | (exact_code(w4.w, m, thr_exact) << 12);
-            word = (word & ~(0xFFFFull << (16 * cc))) | (static_cast<uint64_t>(c4) << (16 * cc));
+          float m = 0.0f;
+  #pragma unroll
+          for (int c = 0; c < 4; ++c)
+            m = fmaxf(m, fmaxf(fmaxf(fabsf(v[c].x), fabsf(v[c].y)), fmaxf(fabsf(v[c].z), fabsf(v[c].w))));
+          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+          if (lb < nblk) {
+            float rcp = (m > 0.0f) ? __frcp_rn(m) : 0.0f;
+            const bool exact_all = !(rcp <= 3.0e38f);   // a subnormal absmax: exact path only
+            if (exact_all) rcp = 0.0f;
+            uint64_t word = 0;
+            uint32_t near_chunks = 0;                   // bit ci: that chunk may sit across a threshold
+  #pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              bool nr = exact_all;
+              const uint32_t c4 = fast_code(__fmul_rn(v[c].x, rcp), lut, nr) |
+                                  (fast_code(__fmul_rn(v[c].y, rcp), lut, nr) << 4) |
+                                  (fast_code(__fmul_rn(v[c].z, rcp), lut, nr) << 8) |
+                                  (fast_code(__fmul_rn(v[c].w, rcp), lut, nr) << 12);
+              word |= static_cast<uint64_t>(c4) << (16 * ci[c]);
+              near_chunks |= (nr ? 1u : 0u) << ci[c];
+            }
+            // redo (rarely) the chunks with a quotient that may sit across its threshold
+            while (near_chunks) {
+              const int cc = __ffs(near_chunks) - 1;
+              near_chunks &= near_chunks - 1;
+              const float4 w4 = *reinterpret_cast<const float4*>(gs + hb * kBlock + quarter * 16 + 4 * cc);
+              const uint32_t c4 = exact_code(w4.x, m, thr_exact) | (exact_code(w4.y, m, thr_exact) << 4) |
+                                  (exact_code(w4.z, m, thr_exact) << 8) | (exact_code(w4.w, m, thr_exact) << 12);
+              word = (word & ~(0xFFFFull << (16 * cc))) | (static_cast<uint64_t>(c4) << (16 * cc));
+            }
+            *reinterpret_cast<uint2*>(codes + (blk0 + lb) * (kBlock / 2) + quarter * 8) =
+                make_uint2(static_cast<uint32_t>(word), static_cast<uint32_t>(word >> 32));
+            if (quarter == 0) amax[lb] = m;
           }
-          *reinterpret_cast<uint2*>(codes + (blk0 + lb) * (kBlock / 2) + quarter * 8) =
-              make_uint2(static_cast<uint32_t>(word), static_cast<uint32_t>(word >> 32));
-          if (quarter == 0) amax[lb] = m;
         }
       }
       __syncthreads();   // buffer b fully read
-      if (tid == 0) issue_half(j + kQBuf, W0, nblocks, ngroups, buf0, bar0);
+      if (tid == 0) issue_half(j + kQBuf, q, buf0, bar0, jissue);
     }
     if (failed_at >= 0) break;
 
@@ -235,7 +280,9 @@ quantize_nf4_kernel(const float* __restrict__ W0, int64_t nblocks, int64_t ngrou
   if (failed_at >= 0 && tid == 0) {
     for (int64_t k = failed_at; k < failed_at + kQBuf; ++k) {
       const int64_t gk = blockIdx.x + (k >> 1) * gridDim.x;
-      if (gk >= ngroups || gk * kGroup + (k & 1) * kHalfBlocks >= nblocks) continue;
+      if (gk >= ngroups) continue;
+      const int jk = job_of(q, gk);
+      if ((gk - q.group0[jk]) * kGroup + (k & 1) * kHalfBlocks >= q.nblocks[jk]) continue;
       sm100::mbar_wait(bar0 + 8 * static_cast<int>(k % kQBuf), static_cast<uint32_t>((k / kQBuf) & 1),
                        &g_quantize_status, kFlagTimeoutProducer);
     }
@@ -245,17 +292,33 @@ quantize_nf4_kernel(const float* __restrict__ W0, int64_t nblocks, int64_t ngrou
 
 }  // namespace
 
-cudaError_t launch_quantize_nf4(const float* W0, int64_t n, uint8_t* codes, uint8_t* dq_codes,
-                                float* dq_scales, cudaStream_t stream, bool dq_u8) {
-  const int64_t nblocks = n / kBlock;
-  const int64_t ngroups = (nblocks + kGroup - 1) / kGroup;
+namespace {
+
+// One launch over jobs [0, n) (n <= NJ).
+template <int NJ>
+cudaError_t launch_jobs(const QuantizeJob* jobs, int n, cudaStream_t stream, bool dq_u8) {
+  QJobs<NJ> q{};
+  q.n = 0;
+  q.group0[0] = 0;
+  for (int i = 0; i < n; ++i) {
+    const int64_t nblocks = jobs[i].n / kBlock;
+    if (nblocks == 0) continue;
+    const int k = q.n++;
+    q.nblocks[k] = nblocks;
+    q.W0[k] = jobs[i].W0;
+    q.codes[k] = jobs[i].codes;
+    q.dq_codes[k] = jobs[i].dq_codes;
+    q.dq_scales[k] = jobs[i].dq_scales;
+    q.group0[k + 1] = q.group0[k] + (nblocks + kGroup - 1) / kGroup;
+  }
+  const int64_t ngroups = q.group0[q.n];
   if (ngroups == 0) return cudaSuccess;
   static bool set[64] = {};
   static int sms[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(quantize_nf4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(quantize_nf4_kernel<NJ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(kQBuf * kHalfBytes));
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
@@ -273,11 +336,26 @@ cudaError_t launch_quantize_nf4(const float* W0, int64_t n, uint8_t* codes, uint
   cfg.attrs = at;
   cfg.numAttrs = 1;
   timing_before(QLORA_KERNEL_QUANTIZE, stream);
-  const cudaError_t e =
-      cudaLaunchKernelEx(&cfg, quantize_nf4_kernel, W0, nblocks, ngroups, codes, dq_codes, dq_scales, dq_u8);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, quantize_nf4_kernel<NJ>, q, dq_u8);
   timing_after(QLORA_KERNEL_QUANTIZE, stream);
   count_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_nf4(const float* W0, int64_t n, uint8_t* codes, uint8_t* dq_codes,
+                                float* dq_scales, cudaStream_t stream, bool dq_u8) {
+  const QuantizeJob job{W0, n, codes, dq_codes, dq_scales};
+  return launch_jobs<1>(&job, 1, stream, dq_u8);
+}
+
+cudaError_t launch_quantize_nf4_batch(const QuantizeJob* jobs, int n, cudaStream_t stream, bool dq_u8) {
+  for (int i = 0; i < n; i += kQMaxJobs) {
+    const cudaError_t e = launch_jobs<kQMaxJobs>(jobs + i, std::min(kQMaxJobs, n - i), stream, dq_u8);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 // Synchronise `stream`, then report (and clear) the quantiser's status word.

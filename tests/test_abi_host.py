@@ -68,6 +68,19 @@ def test_quantize_rejects_before_launch(L):
     assert L.qlora_quantize_nf4(FAKE, 0, 64, FAKE, FAKE, FAKE, None) == 2
 
 
+def test_batch_quantize_rejects_before_launch(L):
+    job = q._QuantizeJob(0x10000, 64, 64, 0x10000, 0x10000, 0x10000)
+    bad_ptr = q._QuantizeJob(0x10000, 64, 64, None, 0x10000, 0x10000)
+    bad_shape = q._QuantizeJob(0x10000, 3, 7, 0x10000, 0x10000, 0x10000)
+    jobs = (q._QuantizeJob * 2)(job, bad_ptr)
+    assert L.qlora_quantize_nf4_batch(jobs, -1, 0, None) == 1          # negative count
+    assert L.qlora_quantize_nf4_batch(None, 2, 0, None) == 1           # no descriptors
+    assert L.qlora_quantize_nf4_batch(jobs, 1, 7, None) == 1           # unknown absmax format
+    assert L.qlora_quantize_nf4_batch(jobs, 2, 0, None) == 1           # a NULL output in job 1
+    assert L.qlora_quantize_nf4_batch((q._QuantizeJob * 2)(job, bad_shape), 2, 0, None) == 2
+    assert L.qlora_quantize_nf4_batch(None, 0, 0, None) == 0           # nothing to do
+
+
 def test_linear_rejects_before_launch(L):
     w = q._Weight(0x10000, 0x10000, 0x10000, 256, 256)
     wp = ctypes.byref(w)

@@ -137,3 +137,20 @@ def test_workspace_without_split_region_keeps_tiles_whole():
         # at most one bf16 rounding step apart (2^-7 relative) where the fp32 sums straddle a boundary
         assert_close(whole[k], split[k].double().cpu().numpy(), f"{k} whole vs split", rel_fro=2e-3, max_abs=1e-2)
     assert torch.equal(whole["dA"], split["dA"]) and torch.equal(whole["dB"], split["dB"])
+
+
+@pytest.mark.parametrize("n_out", [128, 192])
+def test_partial_column_tile_repeated(n_out):
+    """A pair tile wider than the output: each warp stores a prefix of its 32-column
+    blocks and skips the rest, and the staging buffers of the stored blocks must not
+    be touched again until their TMA stores have read them.  Short items (two K-steps)
+    back to back make a late store likely; ten forwards must give the same bytes,
+    and the first matches the oracle."""
+    t, w = layer_on_gpu(64, n_out, 131062, 64, tag="partcol")   # 256 tiles: 3-4 items a pair
+    ws = q.Workspace()
+    first = run_fwd_bwd(t, w, ws)
+    full_check(t, w, first)
+    for _ in range(10):
+        Y, _ = q.qlora_linear_fwd(w, t["X"], t["A"], t["B"], ws)
+        torch.cuda.synchronize()
+        assert torch.equal(Y, first["Y"])

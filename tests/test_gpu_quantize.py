@@ -38,6 +38,37 @@ def test_quantize_bitexact_shapes(shape):
     assert np.array_equal(deq.cpu().numpy().view(np.uint32), nf4.dequantize(*gpu, *shape).view(np.uint32))
 
 
+@pytest.mark.parametrize("dq_format", [q.QLORA_DQ_E4M3, q.QLORA_DQ_U8])
+def test_batch_quantize_equals_single(dq_format):
+    """The batch quantiser (one launch per 32 weights, the weights' groups walked
+    as one sequence) gives the bytes of one call per weight: 40 weights of mixed
+    shapes (short last groups, a single block, 4096 x 11008), so a batch spans
+    two launches; the outputs sit between canary guard regions."""
+    shapes = [(4096, 11008), (64, 96), (1, 64), (512, 768), (7, 640), (320, 192)] * 6 + [(256, 256)] * 4
+    W0s = [synth.normal(f"qbatch{i}", shp, 0.02, device="cuda") for i, shp in enumerate(shapes)]
+    outs, guards = [], []
+    for shp in shapes:
+        n = shp[0] * shp[1]
+        (b0, codes), (b1, dqc), (b2, dqs) = (guarded((n // 2,), torch.uint8), guarded((n // 64,), torch.uint8),
+                                             guarded(((n // 64 + 255) // 256,), torch.float32))
+        outs.append(q.NF4Weight(codes, dqc, dqs, *shp))
+        guards += [b0, b1, b2]
+    q.qlora_quantize_nf4_batch(W0s, outs=outs, dq_format=dq_format)
+    assert q.qlora_quantize_status() == 0
+    assert_guards(guards, "batch quantize")
+    for i, (W0, w) in enumerate(zip(W0s, outs)):
+        one = q.qlora_quantize_nf4(W0, dq_format=dq_format)
+        for a, b in ((w.codes, one.codes), (w.dq_codes, one.dq_codes), (w.dq_scales, one.dq_scales)):
+            assert torch.equal(a, b), f"job {i} {shapes[i]}"
+        assert w.dq_format == dq_format
+    # and the oracle on a few of them
+    for i in (1, 3, 4):
+        gpu = (outs[i].codes.cpu().numpy(), outs[i].dq_codes.cpu().numpy(), outs[i].dq_scales.cpu().numpy())
+        assert_quant_equal(gpu, nf4.quantize_nf4(W0s[i].cpu().numpy(),
+                                                 dq_format="u8" if dq_format == q.QLORA_DQ_U8 else "e4m3"),
+                           f"batch job {i}")
+
+
 def test_quantize_edge_cases():
     """All-zero blocks, -0.0, a single non-zero, dominant +-values, huge and tiny
     magnitudes, a subnormal absmax, and values at / next to every decision
