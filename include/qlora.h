@@ -153,8 +153,10 @@ typedef struct qlora_quantize_job {
 } qlora_quantize_job;
 
 /*
- * qlora_quantize_nf4_ex for n weights (a model's linears quantised in one pass):
- * the same codes, absmax codes and scales, bit for bit, as n separate calls.  Up
+ * qlora_quantize_nf4_ex for n weights ("How it works" step 1 for every frozen
+ * linear of a model; "What QLoRA adds over LoRA": adapters on every linear
+ * layer): the same codes, absmax codes and scales, bit for bit, as n separate
+ * calls.  Up
  * to 32 weights share one launch, whose persistent grid runs through all of their
  * groups in one sequence, so the weights do not each end with a partly idle wave.
  *   jobs  [host] n descriptors (read during the call only); every job must meet

@@ -107,6 +107,7 @@ struct QJobs {
 // so each search starts where the previous one ended).
 template <int NJ>
 __device__ __forceinline__ int job_of(const QJobs<NJ>& q, int64_t gg, int j = 0) {
+  if constexpr (NJ == 1) return 0;
   while (j + 1 < q.n && q.group0[j + 1] <= gg) ++j;
   return j;
 }
@@ -190,6 +191,10 @@ quantize_nf4_kernel(const __grid_constant__ QJobs<NJ> q, bool dq_u8) {
     // across the weights of the launch.
     for (int h = 0; h < 2; ++h, ++j) {
       const bool empty = h * kHalfBlocks >= nblk;
+      // one weight: its short group is this CTA's last, nothing follows the empty half
+      if constexpr (NJ == 1) {
+        if (empty) break;
+      }
       const int b = static_cast<int>(j % kQBuf);
       const uint32_t ph = static_cast<uint32_t>((j / kQBuf) & 1);
       const bool got = sm100::mbar_wait(bar0 + 8 * b, ph, &g_quantize_status, kFlagTimeoutProducer);
