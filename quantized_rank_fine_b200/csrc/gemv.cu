@@ -37,6 +37,8 @@
 //   * V comes from the kernel launched just before (X A).  Launched as a
 //     programmatic dependent, this kernel streams all of its codes while that
 //     one finishes; only the last split's producer waits for it, before it loads V.
+//     It lets its own dependent (the next call's first kernel, which waits for
+//     this one to finish before it reads anything) become resident at once.
 //   * The K-splits of a tile form one thread-block cluster; the split count is
 //     the one that needs the fewest waves x rows per CTA given how many clusters
 //     of each size the device holds at once.  Each CTA sums its row halves into
@@ -138,6 +140,7 @@ nf4_gemv_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_const
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
+  grid_launch_dependents();
   const int tile = blockIdx.x, split = blockIdx.y;
   const int64_t k_begin = static_cast<int64_t>(split) * p.Kc;
   const int rows = static_cast<int>(p.K - k_begin < p.Kc ? p.K - k_begin : p.Kc);   // multiple of 64

@@ -15,9 +15,11 @@
 //   * Each CTA stores every element of its partial into the receive buffer of
 //     the CTA that owns the element (distributed shared memory); after one
 //     cluster barrier the owners add the splits in order and write bf16 V.
-//   * The kernel lets the dependent small-M forward start at once (programmatic
-//     dependent launch): that kernel streams the 4-bit weights meanwhile and
-//     waits for V only when it reaches the adapter rows.
+//   * Launched as a programmatic dependent of the kernel before it, so that its
+//     CTAs are resident when that kernel ends; it reads nothing in global memory
+//     before that kernel has finished.  It then lets the dependent small-M forward
+//     start at once: that kernel streams the 4-bit weights meanwhile and waits
+//     for V only when it reaches the adapter rows.
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -49,6 +51,10 @@ struct XaArgs {
 };
 
 __global__ void __launch_bounds__(kXaThreads) xa_small_kernel(const XaArgs p) {
+  // Everything before this kernel has finished once the wait returns, so the
+  // dependent launched right after (which reads its own inputs at once) sees
+  // them complete.
+  grid_dependency_wait();
   grid_launch_dependents();
   extern __shared__ __align__(16) uint8_t smem[];
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem);                       // [M][kXPitch]
@@ -190,13 +196,15 @@ cudaError_t launch_xa_small(const uint16_t* X, const uint16_t* A, int64_t M, int
   cfg.blockDim = dim3(kXaThreads);
   cfg.dynamicSmemBytes = kXaSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = 1;
   at[0].val.clusterDim.y = static_cast<unsigned>(S);
   at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   timing_before(QLORA_KERNEL_RANK_R, stream);
   const cudaError_t e = cudaLaunchKernelEx(&cfg, xa_small_kernel, a);
   timing_after(QLORA_KERNEL_RANK_R, stream);
