@@ -435,9 +435,10 @@ constexpr size_t kGvSmemBytes = 1024 + kGvStages * kStageBytes + kLutBytes + kGv
 
 // Clusters of each size (1 .. kMaxCluster CTAs) that can be resident at once,
 // queried once per device (the kernels' attributes are set on the way); all
-// zero if the device cannot run the kernel.
+// zero if the device cannot run the kernel.  `sms`: the device's SM count.
 struct ClusterFit {
   int max_active[kMaxCluster + 1];
+  int sms;
 };
 
 const ClusterFit& cluster_fit() {
@@ -474,16 +475,27 @@ const ClusterFit& cluster_fit() {
       break;
     f.max_active[S] = n1 < n2 ? n1 : n2;
   }
+  if (cudaDeviceGetAttribute(&f.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) f.sms = 0;
   cudaGetLastError();
   fits[dev] = f;
   done[dev] = true;
   return fits[dev];
 }
 
-// K-splits S (the cluster size) and rows per split Kc for a K x N weight: the
-// split that minimises waves x rows per CTA (each CTA streams its rows at about
-// the same rate), fewer splits on a tie.  False if no cluster size fits.
-bool gemv_plan(int64_t K, int64_t N, const ClusterFit& fit, int& S, int& Kc) {
+// K-splits S (the cluster size) and rows per split Kc for a K x N weight at M
+// tokens, fewer splits on a tie.  False if no cluster size fits.
+//   * M <= 8: the split that minimises waves x rows per CTA.  A CTA streams its
+//     stages at about the same rate whether or not it shares its SM, so more
+//     CTAs stream more at once.
+//   * M > 8 (two token tiles, twice the products per stage): the consumer warps
+//     are issue-bound and an SM streams at about the same rate with one CTA or
+//     two; a CTA alone on its SM takes a stage in about 7/13 of the time two CTAs
+//     sharing an SM take.  The split minimises the stages an SM streams: a wave
+//     of more CTAs than SMs puts two on some SMs, and those set its length.
+// (Both rules measured on the 4096 x 4096 weight: at M = 1, 8 splits of 8 stages
+// take 11.7 us per forward against 9.6 us for 13 splits of 5; at M = 16, 15.6
+// against 17.0 us.)
+bool gemv_plan(int64_t K, int64_t N, int64_t M, const ClusterFit& fit, int& S, int& Kc) {
   const int64_t tiles = (N + kTileCols - 1) / kTileCols;
   const int64_t stages = K / kStageRows;
   int64_t best_cost = -1;
@@ -492,7 +504,8 @@ bool gemv_plan(int64_t K, int64_t N, const ClusterFit& fit, int& S, int& Kc) {
     const int64_t kc = ((K + s - 1) / s + kStageRows - 1) / kStageRows * kStageRows;
     if ((K + kc - 1) / kc != s) continue;   // another s gives the same split
     const int64_t waves = (tiles + fit.max_active[s] - 1) / fit.max_active[s];
-    const int64_t cost = waves * kc;
+    const int64_t wave_ctas = (tiles < fit.max_active[s] ? tiles : fit.max_active[s]) * s;
+    const int64_t cost = M <= 8 ? waves * kc : waves * (kc / kStageRows) * (wave_ctas > fit.sms ? 13 : 7);
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
       S = s;
@@ -519,13 +532,13 @@ PFN_cuTensorMapEncodeTiled_v12000 gemv_encoder() {
 
 bool gemv_supported(int64_t M, int64_t K, int64_t N) {
   int S, Kc;
-  return M >= 1 && M <= kGemvMaxTokens && gemv_plan(K, N, cluster_fit(), S, Kc);
+  return M >= 1 && M <= kGemvMaxTokens && gemv_plan(K, N, M, cluster_fit(), S, Kc);
 }
 
 cudaError_t launch_gemv(const WeightView& w, const uint16_t* X, const uint16_t* V, const uint16_t* B, int64_t M,
                         int r, uint16_t* Y, uint32_t* status, cudaStream_t stream) {
   int S, Kc;
-  if (w.fmt == kFmtInt16 || M < 1 || M > kGemvMaxTokens || !gemv_plan(w.in, w.out, cluster_fit(), S, Kc))
+  if (w.fmt == kFmtInt16 || M < 1 || M > kGemvMaxTokens || !gemv_plan(w.in, w.out, M, cluster_fit(), S, Kc))
     return cudaErrorInvalidValue;   // NF4 weights only
   auto enc = gemv_encoder();
   if (!enc) return cudaErrorInvalidValue;
