@@ -115,6 +115,17 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def gemm_peak(pk, timed_s, reasons):
+    """The bf16 peak the headline's fused GEMM is measured against: the sustained
+    figure (a seconds-long cuBLAS loop under the power cap) for a kernel timed
+    inside a long step, that is a timed region of 2 s or more or one whose clock
+    record shows the power cap holding the SM clock down; the burst figure
+    otherwise.  Returns (peak TFLOP/s, sustained?, power-capped?)."""
+    power_capped = "sw_power_cap" in (reasons or [])
+    sustained = timed_s >= 2.0 or power_capped
+    return (pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]), sustained, power_capped
+
+
 def flops_fwd_bwd(n_in, n_out, M, r):
     """Algorithmic flops of one forward + backward: 4 M in out + 6 M r (in + out)."""
     return 4 * M * n_in * n_out + 6 * M * r * (n_in + n_out)
@@ -953,13 +964,7 @@ def arm_ours(args, world, rank, local):
     gemm_flops = [flops_fwd_gemm(a, b, M, r) for a, b in wl["shapes"]] * n_gt
     achieved = sum(gemm_flops) / (sum(gemm_ms) / 1e3) / 1e12
     timed_s = ms / 1e3
-    # The sustained peak (a seconds-long cuBLAS loop under the power cap) is the
-    # denominator for a kernel timed inside a long step: a timed region of 2 s or
-    # more, or one in which the clock record shows the power cap holding the SM
-    # clock down.  The burst peak otherwise.  Both fractions are reported.
-    power_capped = "sw_power_cap" in (clk.get("reasons") or [])
-    sustained = timed_s >= 2.0 or power_capped
-    peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
+    peak, sustained, power_capped = gemm_peak(pk, timed_s, clk.get("reasons"))   # both fractions are reported
     traffic = None   # DRAM bytes per launch from the last ncu capture, if gemm.cu is unchanged since
     tp = os.path.join(ROOT, "profiles", "traffic.txt")
     if os.path.exists(tp):

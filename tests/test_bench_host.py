@@ -124,3 +124,14 @@ def test_code_hash_ignores_comments_not_code():
     assert bench.code_tokens(a) == bench.code_tokens(b)
     assert bench.code_tokens(a) != bench.code_tokens(c)
     assert '"a // b"' in bench.code_tokens(a)
+
+
+def test_gemm_peak_rule():
+    """The headline GEMM's denominator: burst for a short region at full clock,
+    sustained once the region is long or the power cap shows in the clock record."""
+    pk = {"bf16_tflops": 1648.3, "bf16_tflops_sustained": 1398.5}
+    assert bench.gemm_peak(pk, 0.5, []) == (1648.3, False, False)
+    assert bench.gemm_peak(pk, 0.5, None) == (1648.3, False, False)
+    assert bench.gemm_peak(pk, 1.1, ["sw_power_cap"]) == (1398.5, True, True)
+    assert bench.gemm_peak(pk, 2.5, []) == (1398.5, True, False)
+    assert bench.gemm_peak(pk, 0.5, ["hw_slowdown"]) == (1648.3, False, False)
