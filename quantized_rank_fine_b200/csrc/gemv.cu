@@ -39,9 +39,10 @@
 //     one finishes; only the last split's producer waits for it, before it loads V.
 //     It lets its own dependent (the next call's first kernel, which waits for
 //     this one to finish before it reads anything) become resident at once.
-//   * The K-splits of a tile form one thread-block cluster; the split count is
-//     the one that needs the fewest waves x rows per CTA given how many clusters
-//     of each size the device holds at once.  Each CTA sums its row halves into
+//   * The K-splits of a tile form one thread-block cluster; the split count
+//     follows from how many clusters of each size the device holds at once (see
+//     gemv_plan: the fewest waves x rows per CTA at up to 8 tokens, the fewest
+//     stages per SM above).  Each CTA sums its row halves into
 //     an fp32 [M][256] partial and stores each slice of it straight into the
 //     shared memory of the CTA that owns the slice (distributed shared memory);
 //     after one cluster barrier every owner adds its slices in split order
