@@ -478,7 +478,7 @@ def run_step(layers, ws):
         q.qlora_linear_bwd(w, t["X"], o["V"], t["dY"], t["A"], t["B"], ws, dX=o["dX"], dA=o["dA"], dB=o["dB"])
 
 
-ROW_NAMES = ("quantize", "dequantize", "merge", "gemv", "train_step", "int16", "mlp_m8192")
+ROW_NAMES = ("quantize", "dequantize", "merge", "gemv", "train_step", "int16", "mlp_m8192", "dense")
 
 
 def time_rows(wl, pk, which="all"):
@@ -506,7 +506,64 @@ def time_rows(wl, pk, which="all"):
             rows["int16"] = time_int16_rows(wl, pk)
         except Exception as e:   # a secondary row never takes the headline down
             rows["int16"] = {"error": f"{type(e).__name__}: {e}"}
+    if "dense" in want:
+        try:
+            rows["dense_context"] = time_dense_context(pk)
+        except Exception as e:   # context only: never takes the headline down
+            rows["dense_context"] = {"error": f"{type(e).__name__}: {e}"}
     return rows
+
+
+def time_dense_context(pk):
+    """Context, not the product: the unfused alternative to the fused forward.
+    cuBLAS (torch.matmul, bf16) on the dequantised bf16 weight, and the same after
+    qlora_dequantize each call, beside this library's forward (V = X A and the
+    fused dequant GEMM) on the same weights, at the attention projection (M = 4096,
+    r = 16) and the MLP projections (M = 8192, r = 64).  Device time per call of a
+    CUDA graph of back-to-back calls over weights rotated past L2; TFLOP/s count
+    2 M in out (the base product)."""
+    import torch
+    import quantized_rank_fine_b200 as q
+    import synth
+    out = {}
+    iters = 20
+    for n_in, n_out, M, r in ((4096, 4096, 4096, 16), (4096, 11008, 8192, 64), (11008, 4096, 8192, 64)):
+        reps = max(3, math.ceil(3 * L2_BYTES / (n_in * n_out * 2)))
+        wts = [q.qlora_quantize_nf4(synth.normal(f"denseW{i}", (n_in, n_out), 0.02, device="cuda"))
+               for i in range(reps)]
+        Ws = [q.qlora_dequantize(w, torch.bfloat16) for w in wts]
+        X = synth.normal(f"denseX{M}", (M, n_in), 1.0, torch.bfloat16, "cuda")
+        A = synth.normal("denseA", (n_in, r), 1 / math.sqrt(n_in), torch.bfloat16, "cuda")
+        B = synth.normal("denseB", (r, n_out), 0.01, torch.bfloat16, "cuda")
+        Y = torch.empty((M, n_out), dtype=torch.bfloat16, device="cuda")
+        V = torch.empty((M, r), dtype=torch.bfloat16, device="cuda")
+        ws = q.Workspace()
+        torch.cuda.synchronize()
+
+        def cublas(i):
+            torch.matmul(X, Ws[i % reps], out=Y)
+
+        def dequant_cublas(i):
+            q.qlora_dequantize(wts[i % reps], torch.bfloat16, out=Ws[i % reps])
+            torch.matmul(X, Ws[i % reps], out=Y)
+
+        def fused(i):
+            q.qlora_linear_fwd(wts[i % reps], X, A, B, ws, Y=Y, V=V)
+
+        flops = 2.0 * M * n_in * n_out
+        row = {}
+        for name, fn in (("cublas_on_dequantised_bf16", cublas), ("dequantize_then_cublas", dequant_cublas),
+                         ("libqlora_forward", fused)):
+            t = graph_per_call(fn, iters)
+            row[name] = {"ms": t, **tensor_fracs(flops, t, pk)}
+        if ws.status() != 0:
+            raise RuntimeError("a kernel wait timed out in the dense-context row")
+        out[f"{n_in}x{n_out}_m{M}_r{r}"] = row
+        del wts, Ws, X, Y, V, ws
+        torch.cuda.synchronize()
+    out["note"] = ("context only: cuBLAS through torch.matmul, not part of the path; TFLOP/s of the base "
+                   "product 2 M in out")
+    return out
 
 
 def weight_row_shape(wl):
