@@ -243,9 +243,9 @@ QLORA_API qlora_status qlora_linear_fwd(const qlora_nf4_weight* w, const uint16_
  *   larger than QLORA_STATIC_WS_BYTES.  The GEMM then always keeps its tiles
  *   whole, which can cost up to one wave of tiles against qlora_linear_fwd with
  *   a full-size workspace.
- *   The array's device address is looked up on every call made outside a stream
- *   capture and cached per device for calls inside one: a captured call needs an
- *   earlier uncaptured call on the same device (else QLORA_ERR_INVALID_ARG).
+ *   The array's device address is looked up on the current device with
+ *   cudaGetSymbolAddress, and kept per device for the cases where the lookup is
+ *   not made (QLORA_ERR_INVALID_ARG if no earlier call on the device made it).
  *   Every call shares the one array and zeroes its split counters first; calls
  *   whose work overlaps on the GPU (other streams, other threads) race and must
  *   not be issued.  A bounded wait that gives up inside a kernel sets the array's
@@ -259,8 +259,7 @@ QLORA_API qlora_status qlora_linear_fwd_static_ws(const qlora_nf4_weight* w, con
 /* qlora_ws_status for the array of qlora_linear_fwd_static_ws on the current
  * device: synchronise `stream`, then QLORA_ERR_TIMEOUT (and clear the word) if a
  * bounded wait in a kernel of a static-workspace call gave up since the last
- * check, else QLORA_OK.  Inside a stream capture it needs an earlier uncaptured
- * call on the device, like the forward. */
+ * check, else QLORA_OK.  It finds the array as the forward does. */
 QLORA_API qlora_status qlora_static_ws_status(void* stream);
 
 /*

@@ -12,10 +12,10 @@
 // The array is a file-scope __device__ variable: every GPU that loads the
 // library holds its kStaticWsBytes until the process exits.  In host code the
 // array's name is only a host-side stand-in, so its device address is looked up
-// with cudaGetSymbolAddress on the device that is current: on every call made
-// outside a stream capture (cheap, and correct again after the device's
-// context was reset), and from a per-device cache during a capture, which
-// therefore needs one earlier call on that device.  All calls share the array
+// with cudaGetSymbolAddress on the device that is current (cheap, and correct
+// again after the device's context was reset).  The lookup is skipped while
+// `stream` is capturing; the address kept per device by an earlier call is used
+// then.  All calls share the array
 // and it keeps the previous call's contents, so each call first zeroes the
 // GEMM's split counters, which must start at zero; the status word is left as
 // it is until qlora_static_ws_status reads and clears it.  Two calls whose work
